@@ -1,0 +1,375 @@
+"""fp64 CPU oracle for Spatial Sparse Attention (SSA).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, __graft_entry__.smoke() and the
+CPU-baseline leg of bench.py, never by the product path. It shares no code with
+the CUDA library. The arithmetic lives in ssa_oracle.c (plain C, fp64, OpenMP
+over rows); this module only marshals arrays, walks packed sequences and maps
+per-sequence block indices to global ones.
+
+Every function follows the formulation written at the top of ssa_oracle.c
+(Direct3D-S2 summary page, "Technical principles", SSA item; Direct3D-S2 model
+page, "What is Direct3D-S2?").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssa_oracle.c")
+_LIB = os.path.join(_HERE, "libssa_oracle.so")
+
+F32, BF16, F16, F64 = 0, 1, 2, 3
+_lib = None
+
+c_i32p = ctypes.POINTER(ctypes.c_int32)
+c_i64p = ctypes.POINTER(ctypes.c_int64)
+c_f32p = ctypes.POINTER(ctypes.c_float)
+c_f64p = ctypes.POINTER(ctypes.c_double)
+c_vp = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile ssa_oracle.c into libssa_oracle.so (gcc, -O2, OpenMP). Returns the path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-Wall", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        L = _lib
+        L.oracle_decode_f16.restype = ctypes.c_double
+        L.oracle_decode_f16.argtypes = [ctypes.c_uint16]
+        L.oracle_decode_bf16.restype = ctypes.c_double
+        L.oracle_decode_bf16.argtypes = [ctypes.c_uint16]
+        L.oracle_round_to.restype = ctypes.c_double
+        L.oracle_round_to.argtypes = [ctypes.c_double, ctypes.c_int]
+        L.oracle_partition.restype = ctypes.c_int64
+        L.oracle_partition.argtypes = [ctypes.c_int64, c_i32p, ctypes.c_int32, c_i32p, c_i32p,
+                                       c_i32p, c_i32p]
+        for f in (L.oracle_window, L.oracle_window_brute):
+            f.restype = ctypes.c_int64
+            f.argtypes = [ctypes.c_int64, c_i32p, ctypes.c_int32, c_i64p, c_i32p]
+        L.oracle_compress.restype = ctypes.c_int
+        L.oracle_compress.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, c_vp, c_vp, c_f32p, c_i32p, c_i32p,
+                                      ctypes.c_int32, c_f64p, c_f64p]
+        L.oracle_forward.restype = ctypes.c_int
+        L.oracle_forward.argtypes = [
+            ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
+            c_f32p, c_f32p, ctypes.c_int32, ctypes.c_int32, c_i32p, c_i32p, c_i32p,
+            ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_i32p,
+            c_f64p, c_f64p, c_f64p, c_f64p, c_i32p, c_f64p]
+        L.oracle_backward.restype = ctypes.c_int
+        L.oracle_backward.argtypes = [
+            ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
+            c_f32p, c_f32p, c_vp, ctypes.c_int32, ctypes.c_int32, c_i32p, c_i32p, c_i32p,
+            ctypes.c_int64, c_i64p, c_i32p, c_i32p, c_f64p, c_f64p, c_f64p]
+        L.oracle_backward_dq_rows.restype = ctypes.c_int
+        L.oracle_backward_dq_rows.argtypes = [
+            ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
+            c_f32p, c_f32p, c_vp, ctypes.c_int32, ctypes.c_int32, c_i32p, c_i32p, c_i32p,
+            ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_f64p, c_i32p]
+    return _lib
+
+
+# ----------------------------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------------------------
+
+def _ptr(a: Optional[np.ndarray], ctype):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctype)
+
+
+def _raw(t):
+    """(contiguous numpy view of the storage bits, dtype code) of a CPU tensor or array."""
+    try:
+        import torch
+        if isinstance(t, torch.Tensor):
+            t = t.detach().cpu().contiguous()
+            if t.dtype == torch.float64:
+                return t.numpy(), F64
+            if t.dtype == torch.float32:
+                return t.numpy(), F32
+            if t.dtype == torch.float16:
+                return t.numpy(), F16
+            if t.dtype == torch.bfloat16:
+                return t.view(torch.int16).numpy(), BF16
+            raise TypeError(t.dtype)
+    except ImportError:
+        pass
+    a = np.ascontiguousarray(t)
+    if a.dtype == np.float64:
+        return a, F64
+    if a.dtype == np.float32:
+        return a, F32
+    if a.dtype == np.float16:
+        return a, F16
+    raise TypeError(a.dtype)
+
+
+def _f32(t) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(t, torch.Tensor):
+            return np.ascontiguousarray(t.detach().cpu().float().numpy())
+    except ImportError:
+        pass
+    return np.ascontiguousarray(t, dtype=np.float32)
+
+
+def decode(bits: np.ndarray, dtype: int) -> np.ndarray:
+    L = lib()
+    f = L.oracle_decode_f16 if dtype == F16 else L.oracle_decode_bf16
+    return np.array([f(int(b)) for b in np.asarray(bits, dtype=np.uint16).ravel()])
+
+
+def round_to(x: np.ndarray, dtype: int) -> np.ndarray:
+    L = lib()
+    return np.array([L.oracle_round_to(float(v), dtype) for v in np.asarray(x).ravel()])
+
+
+# ----------------------------------------------------------------------------------------------
+# plan: partition + window lists
+# ----------------------------------------------------------------------------------------------
+
+def partition(coords: np.ndarray, block: int = 8):
+    """One sequence. Returns perm, tok_blk, blk_off, blk_coord (local indices)."""
+    c = np.ascontiguousarray(coords, dtype=np.int32)
+    n = len(c)
+    perm = np.empty(n, np.int32)
+    tok_blk = np.empty(n, np.int32)
+    blk_off = np.empty(n + 1, np.int32)
+    blk_coord = np.empty((max(n, 1), 3), np.int32)
+    mb = lib().oracle_partition(n, _ptr(c, c_i32p), block, _ptr(perm, c_i32p),
+                                _ptr(tok_blk, c_i32p), _ptr(blk_off, c_i32p),
+                                _ptr(blk_coord, c_i32p))
+    if mb < 0:
+        raise ValueError("oracle_partition failed")
+    return perm, tok_blk, blk_off[:mb + 1].copy(), blk_coord[:mb].copy()
+
+
+def window(coords: np.ndarray, r: int, brute: bool = False):
+    """One sequence. Returns (nbr_off int64 [n+1], nbr_idx int32 [nnz]), rows ascending."""
+    c = np.ascontiguousarray(coords, dtype=np.int32)
+    n = len(c)
+    f = lib().oracle_window_brute if brute else lib().oracle_window
+    off = np.zeros(n + 1, np.int64)
+    nnz = f(n, _ptr(c, c_i32p), r, _ptr(off, c_i64p), None)
+    if nnz == -2:
+        raise ValueError("duplicate coordinate")
+    if nnz < 0:
+        raise ValueError("oracle_window failed")
+    idx = np.empty(max(nnz, 1), np.int32)
+    f(n, _ptr(c, c_i32p), r, _ptr(off, c_i64p), _ptr(idx, c_i32p))
+    return off, idx[:nnz]
+
+
+def plan(coords: np.ndarray, cu_seqlens, block: int = 8, r: int = 2) -> Dict[str, np.ndarray]:
+    """Partition and window lists of a packed batch, with global token and block indices."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    perms, toks, offs, bcs, bseq, nos, nis = [], [], [], [], [], [], []
+    blk_base = np.zeros(len(cu), np.int64)
+    nnz_base = 0
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        perm, tok_blk, blk_off, blk_coord = partition(coords[lo:hi], block)
+        mb = len(blk_coord)
+        perms.append(perm.astype(np.int64) + lo)
+        toks.append(tok_blk.astype(np.int64) + blk_base[s])
+        offs.append(blk_off[:-1].astype(np.int64) + lo)
+        bcs.append(blk_coord)
+        bseq.append(np.full(mb, s, np.int32))
+        blk_base[s + 1] = blk_base[s] + mb
+        no, ni = window(coords[lo:hi], r)
+        nos.append(no[:-1] + nnz_base)
+        nis.append(ni.astype(np.int64) + lo)
+        nnz_base += int(no[-1])
+    mb_total = int(blk_base[-1])
+    return dict(
+        perm=np.concatenate(perms).astype(np.int32) if perms else np.zeros(0, np.int32),
+        tok_blk=np.concatenate(toks).astype(np.int32),
+        blk_off=np.concatenate(offs + [np.array([cu[-1]])]).astype(np.int32),
+        blk_coord=np.concatenate(bcs).astype(np.int32).reshape(mb_total, 3),
+        blk_seq=np.concatenate(bseq).astype(np.int32),
+        blk_base=blk_base,
+        nbr_off=np.concatenate(nos + [np.array([nnz_base])]).astype(np.int64),
+        nbr_idx=np.concatenate(nis).astype(np.int32),
+    )
+
+
+# ----------------------------------------------------------------------------------------------
+# forward / backward
+# ----------------------------------------------------------------------------------------------
+
+def _seq_plan(coords, lo, hi, block, r):
+    perm, tok_blk, blk_off, blk_coord = partition(coords[lo:hi], block)
+    no, ni = window(coords[lo:hi], r)
+    return perm, tok_blk, blk_off, len(blk_coord), no, ni
+
+
+def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None,
+            block: int = 8, round_compressed: bool = True, sel_in=None,
+            want_z: bool = False) -> Dict[str, object]:
+    """Oracle forward for the query rows `rows` (global indices; None = all tokens).
+
+    Returns out, o_cmp, o_sel, o_win ([R, H, D] float64), sel ([R, H, k] int32 global block
+    indices, -1 = empty slot) and, if want_z, z: list of [H, Mb_seq] scaled compressed logits.
+    """
+    coords = np.ascontiguousarray(coords, dtype=np.int32)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    q, dt = _raw(Q)
+    k, _ = _raw(K)
+    v, _ = _raw(V)
+    g = _f32(gates)
+    w = _f32(Wc)
+    N, H, D = q.shape
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    R = len(rows)
+    res = {name: np.zeros((R, H, D)) for name in ("out", "o_cmp", "o_sel", "o_win")}
+    res["sel"] = np.full((R, H, topk), -1, np.int32)
+    zs = [None] * R
+    seq_of = np.searchsorted(cu, rows, side="right") - 1
+    blk_base = 0
+    L = lib()
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        perm, tok_blk, blk_off, mb, no, ni = _seq_plan(coords, lo, hi, block, r)
+        pick = np.nonzero(seq_of == s)[0]
+        if len(pick):
+            local = np.ascontiguousarray(rows[pick] - lo)
+            n_r = len(local)
+            outs = {name: np.zeros((n_r, H, D)) for name in ("out", "o_cmp", "o_sel", "o_win")}
+            sel = np.zeros((n_r, H, topk), np.int32)
+            zc = np.zeros((n_r, H, max(mb, 1))) if want_z else None
+            sin = None
+            if sel_in is not None:
+                sin = np.ascontiguousarray(np.asarray(sel_in, dtype=np.int64)[pick], dtype=np.int64)
+                sin = np.where(sin >= 0, sin - blk_base, -1).astype(np.int32)
+            rc = L.oracle_forward(
+                hi - lo, H, D, dt,
+                q[lo:hi].ctypes.data, k[lo:hi].ctypes.data, v[lo:hi].ctypes.data,
+                _ptr(np.ascontiguousarray(g[lo:hi]), c_f32p), _ptr(w, c_f32p), topk,
+                int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
+                _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p),
+                n_r, _ptr(local, c_i64p), _ptr(sin, c_i32p),
+                _ptr(outs["out"], c_f64p), _ptr(outs["o_cmp"], c_f64p),
+                _ptr(outs["o_sel"], c_f64p), _ptr(outs["o_win"], c_f64p),
+                _ptr(sel, c_i32p), _ptr(zc, c_f64p))
+            if rc != 0:
+                raise RuntimeError("oracle_forward failed")
+            for name in outs:
+                res[name][pick] = outs[name]
+            res["sel"][pick] = np.where(sel >= 0, sel + blk_base, -1)
+            if want_z:
+                for t, p in enumerate(pick):
+                    zs[p] = zc[t, :, :mb].copy()
+        blk_base += mb
+    if want_z:
+        res["z"] = zs
+    res["rows"] = rows
+    return res
+
+
+def backward(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, block: int = 8,
+             round_compressed: bool = True):
+    """Full fp64 backward: (dQ, dK, dV) [N, H, D] of sum(dO * out), selection held fixed."""
+    coords = np.ascontiguousarray(coords, dtype=np.int32)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    q, dt = _raw(Q)
+    k, _ = _raw(K)
+    v, _ = _raw(V)
+    go, _ = _raw(dO)
+    g = _f32(gates)
+    w = _f32(Wc)
+    N, H, D = q.shape
+    dQ, dK, dV = (np.zeros((N, H, D)) for _ in range(3))
+    L = lib()
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        n = hi - lo
+        perm, tok_blk, blk_off, mb, no, ni = _seq_plan(coords, lo, hi, block, r)
+        sel = np.zeros((n, H, topk), np.int32)
+        gs = np.ascontiguousarray(g[lo:hi])
+        rc = L.oracle_forward(n, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data,
+                              v[lo:hi].ctypes.data, _ptr(gs, c_f32p), _ptr(w, c_f32p), topk,
+                              int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
+                              _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p),
+                              n, None, None, None, None, None, None, _ptr(sel, c_i32p), None)
+        if rc != 0:
+            raise RuntimeError("oracle_forward failed")
+        a, b, c = (np.zeros((n, H, D)) for _ in range(3))
+        rc = L.oracle_backward(n, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data,
+                               v[lo:hi].ctypes.data, _ptr(gs, c_f32p), _ptr(w, c_f32p),
+                               go[lo:hi].ctypes.data, topk, int(round_compressed),
+                               _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p), _ptr(blk_off, c_i32p),
+                               mb, _ptr(no, c_i64p), _ptr(ni, c_i32p), _ptr(sel, c_i32p),
+                               _ptr(a, c_f64p), _ptr(b, c_f64p), _ptr(c, c_f64p))
+        if rc != 0:
+            raise RuntimeError("oracle_backward failed")
+        dQ[lo:hi], dK[lo:hi], dV[lo:hi] = a, b, c
+    return dQ, dK, dV
+
+
+def backward_dq_rows(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, rows,
+                     block: int = 8, round_compressed: bool = True):
+    """dQ [R, H, D] for the given global rows, evaluated row by row (any size)."""
+    coords = np.ascontiguousarray(coords, dtype=np.int32)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    q, dt = _raw(Q)
+    k, _ = _raw(K)
+    v, _ = _raw(V)
+    go, _ = _raw(dO)
+    g = _f32(gates)
+    w = _f32(Wc)
+    N, H, D = q.shape
+    rows = np.asarray(rows, dtype=np.int64)
+    dQ = np.zeros((len(rows), H, D))
+    seq_of = np.searchsorted(cu, rows, side="right") - 1
+    L = lib()
+    for s in range(len(cu) - 1):
+        pick = np.nonzero(seq_of == s)[0]
+        if not len(pick):
+            continue
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        perm, tok_blk, blk_off, mb, no, ni = _seq_plan(coords, lo, hi, block, r)
+        local = np.ascontiguousarray(rows[pick] - lo)
+        out = np.zeros((len(local), H, D))
+        rc = L.oracle_backward_dq_rows(
+            hi - lo, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data, v[lo:hi].ctypes.data,
+            _ptr(np.ascontiguousarray(g[lo:hi]), c_f32p), _ptr(w, c_f32p), go[lo:hi].ctypes.data,
+            topk, int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
+            _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p), len(local),
+            _ptr(local, c_i64p), _ptr(out, c_f64p), None)
+        if rc != 0:
+            raise RuntimeError("oracle_backward_dq_rows failed")
+        dQ[pick] = out
+    return dQ
+
+
+def compress(coords, K, V, Wc, block: int = 8, round_compressed: bool = False):
+    """Compressed tokens (Kc, Vc) [Mb, H, D] of a single sequence."""
+    k, dt = _raw(K)
+    v, _ = _raw(V)
+    w = _f32(Wc)
+    N, H, D = k.shape
+    perm, tok_blk, blk_off, blk_coord = partition(coords, block)
+    mb = len(blk_coord)
+    Kc = np.zeros((mb, H, D))
+    Vc = np.zeros((mb, H, D))
+    lib().oracle_compress(mb, H, D, dt, k.ctypes.data, v.ctypes.data, _ptr(w, c_f32p),
+                          _ptr(perm, c_i32p), _ptr(blk_off, c_i32p), int(round_compressed),
+                          _ptr(Kc, c_f64p), _ptr(Vc, c_f64p))
+    return Kc, Vc

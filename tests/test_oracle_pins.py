@@ -1,0 +1,439 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each test checks the oracle against one of: a library routine for a special case
+(dense softmax attention via torch's scaled_dot_product_attention, numpy/torch
+float conversions), a closed form, an invariant of the method, a planted input
+with a known answer, a brute-force restatement on tiny inputs, or finite
+differences. A dropped term, a wrong sign or index, or a transposed operand in
+the oracle fails at least one of them.
+
+The method: Direct3D-S2 summary page, "Technical principles", SSA item
+(partition by 3D coordinates; block compression; top-k blocks by compression
+scores; local window; gated aggregation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+F32, BF16, F16, F64 = oracle.F32, oracle.BF16, oracle.F16, oracle.F64
+
+
+def _tiny_coords():
+    c, cu, g = workloads.make_coords(workloads.CONFIGS["tiny"])
+    return c, cu
+
+
+def _rand(shape, seed, dtype=np.float64):
+    return np.random.default_rng(seed).standard_normal(shape).astype(dtype)
+
+
+def _gates(N, H, g, seed=0):
+    if g is None:
+        return np.random.default_rng(seed).random((N, H, 3)).astype(np.float32)
+    return np.broadcast_to(np.asarray(g, np.float32), (N, H, 3)).copy()
+
+
+def dense_attention(q, k, v):
+    """softmax(q k^T / sqrt(D)) v per head via torch's library routine, fp64. [N,H,D] in/out."""
+    qt, kt, vt = (torch.from_numpy(np.ascontiguousarray(x)).permute(1, 0, 2) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)
+    return o.permute(1, 0, 2).numpy()
+
+
+def run(coords, q, k, v, gates, Wc, topk, r, **kw):
+    cu = np.array([0, len(coords)])
+    return oracle.forward(coords, cu, q, k, v, gates, Wc, topk, r, **kw)
+
+
+# ---------------------------------------------------------------------------------------------
+# storage-type decoding and rounding (checked against numpy / torch conversions)
+# ---------------------------------------------------------------------------------------------
+
+def test_decode_f16_every_bit_pattern():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.decode(bits, F16)
+    ref = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def test_decode_bf16_every_bit_pattern():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.decode(bits, BF16)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def test_round_to_f16_matches_numpy():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([
+        rng.standard_normal(3000) * 10.0 ** rng.integers(-8, 5, 3000),
+        (np.arange(-2000, 2000) + 0.5) * 2.0 ** -10,       # exact ties at the unit scale
+        (np.arange(-300, 300) + 0.5) * 2.0 ** -24,         # ties in the subnormal range
+        [65504.0, 65519.9, 65520.0, -70000.0, 0.0, -0.0],
+    ])
+    ours = oracle.round_to(x, F16)
+    ref = x.astype(np.float16).astype(np.float64)
+    assert np.array_equal(ours, ref)
+
+
+def test_round_to_bf16_matches_torch():
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal(5000) * 10.0 ** rng.integers(-30, 30, 5000)).astype(np.float32)
+    ours = oracle.round_to(x.astype(np.float64), BF16)
+    ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(ours, ref)
+
+
+# ---------------------------------------------------------------------------------------------
+# partition and window lists
+# ---------------------------------------------------------------------------------------------
+
+def test_partition_matches_plain_grouping():
+    c, _ = _tiny_coords()
+    c = c[np.random.default_rng(3).permutation(len(c))]
+    perm, tok_blk, blk_off, blk_coord = oracle.partition(c, 8)
+    groups = {}
+    for i, xyz in enumerate(c):
+        groups.setdefault(tuple(int(t) // 8 for t in xyz), []).append(i)
+    keys = sorted(groups)
+    assert [tuple(b) for b in blk_coord] == keys
+    assert list(perm) == [i for kk in keys for i in groups[kk]]
+    assert list(np.diff(blk_off)) == [len(groups[kk]) for kk in keys]
+    assert blk_off[-1] == len(c)
+    for b, kk in enumerate(keys):
+        assert all(tok_blk[i] == b for i in groups[kk])
+
+
+@pytest.mark.parametrize("r", [0, 1, 2, 3])
+def test_window_matches_pairwise_brute_force(r):
+    c, _ = _tiny_coords()
+    rng = np.random.default_rng(4 + r)
+    sub = c[rng.choice(len(c), 500, replace=False)]
+    off, idx = oracle.window(sub, r)
+    d = np.abs(sub[:, None, :] - sub[None, :, :]).max(axis=2)
+    for i in range(len(sub)):
+        ref = np.nonzero(d[i] <= r)[0]
+        assert np.array_equal(idx[off[i]:off[i + 1]], ref)
+    off_b, idx_b = oracle.window(sub, r, brute=True)
+    assert np.array_equal(off, off_b) and np.array_equal(idx, idx_b)
+
+
+def test_window_invariants():
+    c, _ = _tiny_coords()
+    r = 2
+    off, idx = oracle.window(c, r)
+    pairs = set()
+    for i in range(len(c)):
+        row = idx[off[i]:off[i + 1]]
+        assert i in row
+        assert len(row) <= (2 * r + 1) ** 3
+        assert np.all(np.diff(row) > 0)
+        pairs.update((i, int(j)) for j in row)
+    assert all((j, i) in pairs for (i, j) in pairs)
+
+
+def test_window_rejects_duplicates():
+    c = np.array([[1, 2, 3], [4, 5, 6], [1, 2, 3]], np.int32)
+    with pytest.raises(ValueError):
+        oracle.window(c, 1)
+
+
+# ---------------------------------------------------------------------------------------------
+# branches reduce to dense attention in their limiting cases
+# ---------------------------------------------------------------------------------------------
+
+def _tiny_inputs(seed=10, H=2, D=32):
+    c, _ = _tiny_coords()
+    N = len(c)
+    q, k, v = (_rand((N, H, D), seed + t) for t in range(3))
+    Wc = _rand((D, D), seed + 3) / np.sqrt(D)
+    return c, q, k, v, Wc.astype(np.float32)
+
+
+def test_selection_branch_is_dense_attention_when_k_covers_all_blocks():
+    c, q, k, v, Wc = _tiny_inputs()
+    mb = len(oracle.partition(c)[3])
+    res = run(c, q, k, v, _gates(len(c), 2, (0, 1, 0)), Wc, topk=mb + 3, r=1)
+    ref = dense_attention(q, k, v)
+    np.testing.assert_allclose(res["o_sel"], ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(res["out"], ref, rtol=0, atol=1e-12)
+    assert np.all(res["sel"][:, :, mb:] == -1)
+    assert np.all(np.sort(res["sel"][:, :, :mb], axis=2) == np.arange(mb))
+
+
+def test_window_branch_is_dense_attention_when_radius_covers_grid():
+    c, q, k, v, Wc = _tiny_inputs(seed=20)
+    res = run(c, q, k, v, _gates(len(c), 2, (0, 0, 1)), Wc, topk=4, r=40)
+    np.testing.assert_allclose(res["out"], dense_attention(q, k, v), rtol=0, atol=1e-12)
+
+
+def test_compressed_branch_is_dense_attention_on_a_lattice():
+    # one token per block (coordinates on multiples of 8) and Wc = I: compressed tokens are the
+    # tokens themselves, so the compressed branch is dense attention over all tokens.
+    g = np.arange(0, 64, 8)
+    c = np.stack(np.meshgrid(g, g, g, indexing="ij"), -1).reshape(-1, 3).astype(np.int32)
+    N, H, D = len(c), 2, 16
+    q, k, v = (_rand((N, H, D), 30 + t) for t in range(3))
+    res = run(c, q, k, v, _gates(N, H, (1, 0, 0)), np.eye(D, dtype=np.float32), topk=3, r=1,
+              round_compressed=False)
+    np.testing.assert_allclose(res["out"], dense_attention(q, k, v), rtol=0, atol=1e-12)
+
+
+def test_constant_values_give_closed_forms():
+    c, q, k, v, Wc = _tiny_inputs(seed=40)
+    ones = np.ones_like(v)
+    res = run(c, q, k, ones, _gates(len(c), 2, None), Wc, topk=4, r=2, round_compressed=False)
+    np.testing.assert_allclose(res["o_sel"], 1.0, atol=1e-13)
+    np.testing.assert_allclose(res["o_win"], 1.0, atol=1e-13)
+    colsum = Wc.astype(np.float64).sum(axis=0)      # 1^T . Wc: the compressed value of V = 1
+    np.testing.assert_allclose(res["o_cmp"], np.broadcast_to(colsum, res["o_cmp"].shape),
+                               atol=1e-12)
+
+
+def test_pooling_of_block_constant_keys():
+    c, _ = _tiny_coords()
+    N, H, D = len(c), 2, 8
+    perm, tok_blk, blk_off, blk_coord = oracle.partition(c)
+    mb = len(blk_coord)
+    cb = _rand((mb, H, D), 50)
+    k = cb[tok_blk]                      # every token carries its block's constant key
+    Wc = _rand((D, D), 51).astype(np.float32)
+    Kc, Vc = oracle.compress(c, k, k, Wc)
+    ref = np.einsum("bhd,de->bhe", cb, Wc.astype(np.float64))
+    np.testing.assert_allclose(Kc, ref, atol=1e-12)
+    np.testing.assert_allclose(Vc, ref, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# invariants
+# ---------------------------------------------------------------------------------------------
+
+def test_output_is_linear_in_the_gates():
+    c, q, k, v, Wc = _tiny_inputs(seed=60)
+    N = len(c)
+    # multiples of 1/16, so ga + gb is exact in fp32
+    ga = np.floor(_gates(N, 2, None, seed=1) * 16) / 16
+    gb = np.floor(_gates(N, 2, None, seed=2) * 16) / 16
+    ra = run(c, q, k, v, ga, Wc, 4, 2)["out"]
+    rb = run(c, q, k, v, gb, Wc, 4, 2)["out"]
+    rab = run(c, q, k, v, ga + gb, Wc, 4, 2)["out"]
+    np.testing.assert_allclose(rab, ra + rb, atol=1e-12)
+
+
+def test_permutation_equivariance():
+    c, q, k, v, Wc = _tiny_inputs(seed=70)
+    N = len(c)
+    g = _gates(N, 2, None)
+    base = run(c, q, k, v, g, Wc, 4, 2)
+    p = np.random.default_rng(71).permutation(N)
+    shuf = run(c[p], q[p], k[p], v[p], g[p], Wc, 4, 2)
+    np.testing.assert_allclose(shuf["out"], base["out"][p], atol=1e-12)
+    # blocks are indexed by coordinate, not by token order: the selection is unchanged
+    assert np.array_equal(shuf["sel"], base["sel"][p])
+
+
+def test_translation_by_whole_blocks():
+    c, q, k, v, Wc = _tiny_inputs(seed=80)
+    g = _gates(len(c), 2, None)
+    base = run(c, q, k, v, g, Wc, 4, 2)
+    moved = run(c + np.array([8, 16, 24], np.int32), q, k, v, g, Wc, 4, 2)
+    np.testing.assert_allclose(moved["out"], base["out"], atol=1e-12)
+    assert np.array_equal(moved["sel"], base["sel"])
+
+
+# ---------------------------------------------------------------------------------------------
+# planted top-k
+# ---------------------------------------------------------------------------------------------
+
+def planted_case(dtype=np.float64, H=2, D=16, seed=90):
+    """Every query is e = 1; every key of block b is alpha_b * 1; Wc = I.
+
+    Then Kc_b = alpha_b * 1 and the compressed logit is z_b = alpha_b * D / sqrt(D), so the
+    expected ranking is by alpha (ties -> lower block index), independent of any arithmetic.
+    Alphas are multiples of 1/8 (exact in every storage type); two blocks are tied on purpose.
+    """
+    c, _ = _tiny_coords()
+    N = len(c)
+    perm, tok_blk, blk_off, blk_coord = oracle.partition(c)
+    mb = len(blk_coord)
+    rng = np.random.default_rng(seed)
+    alpha = np.stack([rng.permutation(mb) for _ in range(H)], axis=1).astype(np.float64)
+    alpha = (alpha - mb / 2) / 8.0
+    alpha[7, 0] = alpha[3, 0]                   # planted tie in head 0: block 3 must win it
+    q = np.ones((N, H, D), dtype)
+    k = np.repeat(alpha[tok_blk][:, :, None], D, axis=2).astype(dtype)
+    v = _rand((N, H, D), seed + 1, dtype)
+    return c, tok_blk, alpha, q, k, v
+
+
+def expected_selection(tok_blk, alpha, topk):
+    N, H = len(tok_blk), alpha.shape[1]
+    mb = alpha.shape[0]
+    sel = np.full((N, H, topk), -1, np.int64)
+    for i in range(N):
+        for h in range(H):
+            own = tok_blk[i]
+            others = sorted((b for b in range(mb) if b != own), key=lambda b: (-alpha[b, h], b))
+            row = [own] + others[:topk - 1]
+            sel[i, h, :len(row)] = row
+    return sel
+
+
+def test_planted_topk_is_exact():
+    c, tok_blk, alpha, q, k, v = planted_case()
+    N, H, D = q.shape
+    topk = 6
+    res = run(c, q, k, v, _gates(N, H, None), np.eye(D, dtype=np.float32), topk, 2)
+    assert np.array_equal(res["sel"], expected_selection(tok_blk, alpha, topk))
+
+
+def test_planted_topk_with_fewer_blocks_than_k():
+    c, tok_blk, alpha, q, k, v = planted_case()
+    N, H, D = q.shape
+    mb = alpha.shape[0]
+    res = run(c, q, k, v, _gates(N, H, None), np.eye(D, dtype=np.float32), mb + 2, 2)
+    assert np.array_equal(res["sel"], expected_selection(tok_blk, alpha, mb + 2))
+
+
+# ---------------------------------------------------------------------------------------------
+# brute-force restatement on a tiny input (no plan, plain loops)
+# ---------------------------------------------------------------------------------------------
+
+def brute_forward(coords, q, k, v, gates, Wc, topk, r):
+    N, H, D = q.shape
+    s = 1.0 / np.sqrt(D)
+    W = Wc.astype(np.float64)
+    key = [tuple(int(t) // 8 for t in xyz) for xyz in coords]
+    blocks = sorted(set(key))
+    members = [[i for i in range(N) if key[i] == b] for b in blocks]
+    out = np.zeros((N, H, D))
+
+    def softmax_mix(qv, kk, vv):
+        z = s * (kk @ qv)
+        e = np.exp(z - z.max())
+        return (e / e.sum()) @ vv
+
+    for h in range(H):
+        Kc = np.array([k[m, h].mean(axis=0) @ W for m in members])
+        Vc = np.array([v[m, h].mean(axis=0) @ W for m in members])
+        for i in range(N):
+            z = s * (Kc @ q[i, h])
+            o_cmp = softmax_mix(q[i, h], Kc, Vc)
+            own = blocks.index(key[i])
+            others = sorted((b for b in range(len(blocks)) if b != own), key=lambda b: (-z[b], b))
+            J = [j for b in [own] + others[:topk - 1] for j in members[b]]
+            o_sel = softmax_mix(q[i, h], k[J, h], v[J, h])
+            Wn = [j for j in range(N) if np.abs(coords[j] - coords[i]).max() <= r]
+            o_win = softmax_mix(q[i, h], k[Wn, h], v[Wn, h])
+            g = gates[i, h].astype(np.float64)
+            out[i, h] = g[0] * o_cmp + g[1] * o_sel + g[2] * o_win
+    return out
+
+
+def test_brute_force_agrees_on_tiny_input():
+    c, _ = _tiny_coords()
+    c = c[:260]
+    N, H, D = len(c), 2, 8
+    q, k, v = (_rand((N, H, D), 100 + t) for t in range(3))
+    Wc = (_rand((D, D), 104) / np.sqrt(D)).astype(np.float32)
+    g = _gates(N, H, None, seed=5)
+    res = run(c, q, k, v, g, Wc, 3, 2, round_compressed=False)
+    np.testing.assert_allclose(res["out"], brute_forward(c, q, k, v, g, Wc, 3, 2), atol=1e-12)
+
+
+def test_fp16_inputs_are_decoded_exactly():
+    c, q, k, v, Wc = _tiny_inputs(seed=110)
+    qh, kh, vh = (x.astype(np.float16) for x in (q, k, v))
+    g = _gates(len(c), 2, None)
+    a = run(c, qh, kh, vh, g, Wc, 4, 2, round_compressed=False)
+    b = run(c, qh.astype(np.float64), kh.astype(np.float64), vh.astype(np.float64), g, Wc, 4, 2,
+            round_compressed=False)
+    np.testing.assert_array_equal(a["out"], b["out"])
+
+
+# ---------------------------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------------------------
+
+def test_backward_selection_branch_is_dense_attention_backward():
+    c, _ = _tiny_coords()
+    c = c[:400]
+    N, H, D = len(c), 2, 16
+    q, k, v, dO = (_rand((N, H, D), 120 + t) for t in range(4))
+    mb = len(oracle.partition(c)[3])
+    g = _gates(N, H, (0, 1, 0))
+    cu = np.array([0, N])
+    dQ, dK, dV = oracle.backward(c, cu, q, k, v, g, np.eye(D, dtype=np.float32), dO, mb + 1, 1,
+                                 round_compressed=False)
+    qt, kt, vt = (torch.from_numpy(x).permute(1, 0, 2).requires_grad_() for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt)
+    (o * torch.from_numpy(dO).permute(1, 0, 2)).sum().backward()
+    for ours, ref in ((dQ, qt.grad), (dK, kt.grad), (dV, vt.grad)):
+        np.testing.assert_allclose(ours, ref.permute(1, 0, 2).numpy(), atol=1e-12)
+
+
+def test_backward_matches_finite_differences():
+    c, _ = _tiny_coords()
+    c = c[:150]
+    N, H, D = len(c), 1, 8
+    rng = np.random.default_rng(130)
+    q, k, v, dO = (rng.standard_normal((N, H, D)) for _ in range(4))
+    Wc = (rng.standard_normal((D, D)) / np.sqrt(D)).astype(np.float32)
+    g = _gates(N, H, None, seed=7)
+    topk, r = 2, 1
+    cu = np.array([0, N])
+    dQ, dK, dV = oracle.backward(c, cu, q, k, v, g, Wc, dO, topk, r, round_compressed=False)
+    base_sel = run(c, q, k, v, g, Wc, topk, r, round_compressed=False)["sel"]
+
+    def loss(qq, kk, vv):
+        res = run(c, qq, kk, vv, g, Wc, topk, r, round_compressed=False)
+        assert np.array_equal(res["sel"], base_sel)   # the selection must not move
+        return float((res["out"] * dO).sum())
+
+    eps = 1e-6
+    for name, x, grad in (("q", q, dQ), ("k", k, dK), ("v", v, dV)):
+        for t in rng.choice(x.size, 12, replace=False):
+            xp, xm = x.copy(), x.copy()
+            xp.flat[t] += eps
+            xm.flat[t] -= eps
+            args_p = [xp if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            args_m = [xm if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad.flat[t]) <= 1e-6 * max(1.0, abs(fd)), (name, t, fd, grad.flat[t])
+
+
+def test_backward_dq_rows_matches_full_backward():
+    c, _ = _tiny_coords()
+    N, H, D = len(c), 2, 8
+    q, k, v, dO = (_rand((N, H, D), 140 + t) for t in range(4))
+    Wc = (_rand((D, D), 145) / np.sqrt(D)).astype(np.float32)
+    g = _gates(N, H, None, seed=9)
+    cu = np.array([0, N])
+    dQ, _, _ = oracle.backward(c, cu, q, k, v, g, Wc, dO, 4, 2)
+    rows = np.array([0, 5, 77, 1000, N - 1])
+    dq = oracle.backward_dq_rows(c, cu, q, k, v, g, Wc, dO, 4, 2, rows)
+    np.testing.assert_allclose(dq, dQ[rows], atol=1e-13)
+
+
+def test_backward_gradient_sums():
+    # sum_j dK_j = 0 for every head (each branch's dz rows sum to zero, and the compression
+    # map spreads dKc_b evenly over the block); sum_j dV_j = sum_i (g0 dO_i Wc^T + g1 dO_i + g2 dO_i)
+    c, _ = _tiny_coords()
+    N, H, D = len(c), 2, 8
+    q, k, v, dO = (_rand((N, H, D), 150 + t) for t in range(4))
+    Wc = (_rand((D, D), 155) / np.sqrt(D)).astype(np.float32)
+    g = _gates(N, H, None, seed=11)
+    cu = np.array([0, N])
+    dQ, dK, dV = oracle.backward(c, cu, q, k, v, g, Wc, dO, 4, 2)
+    np.testing.assert_allclose(dK.sum(axis=0), 0.0, atol=1e-10)
+    gd = g.astype(np.float64)
+    ref = (np.einsum("nh,nhd->hd", gd[:, :, 0], dO) @ Wc.astype(np.float64).T
+           + np.einsum("nh,nhd->hd", gd[:, :, 1] + gd[:, :, 2], dO))
+    np.testing.assert_allclose(dV.sum(axis=0), ref, atol=1e-10)

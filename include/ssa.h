@@ -1,0 +1,188 @@
+/*
+ * ssa.h -- C ABI of libssa.so: Spatial Sparse Attention (SSA) forward on B200 (sm_100a).
+ *
+ * The operation (Direct3D-S2 summary page, "Technical principles of Direct3D-S2", SSA item;
+ * Direct3D-S2 model page, "What is Direct3D-S2?"): sparse voxel tokens are partitioned by their
+ * 3D coordinates into aligned 8^3 blocks; each query combines
+ *   (a) attention over compressed block tokens (block mean of K/V times a D x D map Wc),
+ *   (b) exact attention over the tokens of its own block plus the top (k-1) other blocks ranked
+ *       by (a)'s attention scores,
+ *   (c) attention over the tokens within Chebyshev radius r of it,
+ * summed with per-(token, head) gates: out = g0*o_cmp + g1*o_sel + g2*o_win. Softmax scale is
+ * 1/sqrt(D). Blocks are indexed in lexicographic (bx, by, bz) order inside each sequence and
+ * sequences are independent.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are CUDA device pointers owned by the caller; they must stay valid
+ *     until the work queued on `stream` has finished. Pointers marked "host" are read before the
+ *     call returns unless stated otherwise.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All device work is queued on
+ *     it; only ssa_plan*, ssa_plan_export, ssa_forward_host and ssa_last_device_status wait for
+ *     the device.
+ *   - Tensors are contiguous, row-major. Q, K, V, out: [N, H, D] elements of `dtype` (token-major,
+ *     one row of H*D values per token). gates: [N, H, 3] fp32 in order (cmp, sel, win). Wc: [D, D]
+ *     fp32, applied as a row vector times Wc (Kc[e] = sum_d mean(K)[d] * Wc[d][e]).
+ *   - Errors: every function returns SSA_OK or an ssa_status_t code and leaves outputs
+ *     unspecified on error. Argument errors are reported before any work is queued. Errors found
+ *     by kernels (bad coordinates, bounded waits that ran out) are recorded in the plan's device
+ *     status word, returned by the next call that waits for the device, and readable with
+ *     ssa_last_device_status. No kernel traps or asserts.
+ *   - Device memory is obtained through the allocator hook (ssa_set_allocator; default
+ *     cudaMallocAsync/cudaFreeAsync on the call's stream). A plan owns its buffers until
+ *     ssa_plan_destroy; the forward workspace is cached in the plan and allocated on the first
+ *     forward call for a given (H, D, dtype, k), so later calls of that shape allocate nothing.
+ *   - Supported: block = 8; 0 <= r <= 8; 1 <= k <= 32; D in {32, 64, 96, 128};
+ *     fp32 (CUDA-core path), bf16 and fp16 (tensor-core path, fp32 accumulation);
+ *     grid extents 1..65535 per axis; N < 2^31 / H tokens.
+ *   - There is no CPU fallback.
+ */
+#ifndef SSA_H
+#define SSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSA_API __attribute__((visibility("default")))
+#else
+#define SSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ssa_plan_s* ssa_plan_t;
+
+typedef enum { SSA_F32 = 0, SSA_BF16 = 1, SSA_F16 = 2 } ssa_dtype_t;
+
+typedef enum {
+    SSA_OK = 0,
+    SSA_ERR_INVALID_ARG = 1,      /* bad pointer, size, or unsupported combination of sizes */
+    SSA_ERR_COORD_RANGE = 2,      /* a coordinate outside [0, grid) of its sequence */
+    SSA_ERR_DUPLICATE_COORD = 3,  /* two tokens of one sequence share a voxel */
+    SSA_ERR_ALLOC = 4,            /* the allocator hook returned NULL */
+    SSA_ERR_CUDA = 5,             /* a CUDA runtime call failed */
+    SSA_ERR_UNSUPPORTED = 6,      /* block != 8, D/k/r outside the supported set, no sm_100 GPU */
+    SSA_ERR_DEVICE_TIMEOUT = 7    /* a kernel's bounded wait ran out; its outputs are invalid */
+} ssa_status_t;
+
+/* Device allocator hook: return `bytes` of device memory usable on `stream` (a cudaStream_t),
+ * or NULL on failure. `ctx` is passed through. */
+typedef void* (*ssa_alloc_fn)(size_t bytes, void* stream, void* ctx);
+typedef void (*ssa_free_fn)(void* ptr, void* stream, void* ctx);
+
+/* Replace the process-wide allocator (NULL, NULL restores cudaMallocAsync/cudaFreeAsync).
+ * Plans keep the hook they were created with. Not thread-safe against concurrent plan calls. */
+SSA_API ssa_status_t ssa_set_allocator(ssa_alloc_fn alloc, ssa_free_fn release, void* ctx);
+
+/*
+ * Build the plan of one sequence: rows a1 (block partition) and a2 (coordinate hash and window
+ * neighbour lists) of the method (Direct3D-S2 model page, "What is Direct3D-S2?": tokens are
+ * partitioned by 3D coordinates; summary page, SSA item: local window operations).
+ *   coords: device int32 [n, 3] voxel coordinates (x, y, z), each in [0, grid[axis]).
+ *   n:      number of tokens (>= 1).
+ *   grid:   host int32[3] grid extent.
+ *   block:  block edge, must be 8.
+ *   r:      window radius (Chebyshev), 0..8.
+ *   out:    receives the plan handle (owned by the caller; release with ssa_plan_destroy).
+ * Waits for the device twice (to size the neighbour lists and to report coordinate errors).
+ * Errors: SSA_ERR_COORD_RANGE, SSA_ERR_DUPLICATE_COORD, SSA_ERR_INVALID_ARG, SSA_ERR_ALLOC,
+ * SSA_ERR_CUDA, SSA_ERR_UNSUPPORTED. The coords buffer is not retained.
+ */
+SSA_API ssa_status_t ssa_plan(const int32_t* coords, int64_t n, const int32_t grid[3], int32_t block,
+                      int32_t r, void* stream, ssa_plan_t* out);
+
+/*
+ * Plan of a packed batch of `batch` independent sequences.
+ *   coords:     device int32 [N, 3], sequence s occupying rows cu_seqlens[s]..cu_seqlens[s+1]-1.
+ *   cu_seqlens: host int64 [batch + 1], cu_seqlens[0] = 0, non-decreasing, last = N.
+ *   grids:      host int32 [batch, 3], per-sequence grid extent.
+ * Blocks are numbered sequence by sequence (all blocks of sequence 0 first). Same errors as
+ * ssa_plan.
+ */
+SSA_API ssa_status_t ssa_plan_varlen(const int32_t* coords, const int64_t* cu_seqlens, int32_t batch,
+                             const int32_t* grids, int32_t block, int32_t r, void* stream,
+                             ssa_plan_t* out);
+
+/* Sizes of a plan (host outputs; any may be NULL): tokens, occupied blocks, total neighbour
+ * list length, number of sequences. */
+SSA_API ssa_status_t ssa_plan_info(ssa_plan_t plan, int64_t* n, int64_t* num_blocks, int64_t* nnz,
+                           int32_t* batch);
+
+/*
+ * Copy the plan's canonical arrays into caller buffers (device pointers, any may be NULL):
+ *   perm      int32 [N]       tokens in block order (ascending token index inside a block)
+ *   tok_blk   int32 [N]       block index of every token
+ *   blk_off   int32 [Mb + 1]  first position in perm of every block
+ *   blk_coord int32 [Mb, 3]   block coordinates (bx, by, bz)
+ *   blk_seq   int32 [Mb]      sequence of every block
+ *   nbr_off   int64 [N + 1]   window CSR offsets
+ *   nbr_idx   int32 [nnz]     window neighbours (global token indices), ascending per row
+ * Waits for the device.
+ */
+SSA_API ssa_status_t ssa_plan_export(ssa_plan_t plan, int32_t* perm, int32_t* tok_blk, int32_t* blk_off,
+                             int32_t* blk_coord, int32_t* blk_seq, int64_t* nbr_off,
+                             int32_t* nbr_idx, void* stream);
+
+/*
+ * Forward pass (rows a3-a8): out = g0*o_cmp + g1*o_sel + g2*o_win for every token and head.
+ *   q, k, v:  device [N, H, D] of dtype.
+ *   gates:    device fp32 [N, H, 3].
+ *   wc:       device fp32 [D, D].
+ *   heads, head_dim: H and D.
+ *   topk:     k, number of selected blocks including the own block (1..32).
+ *   out:      device [N, H, D] of dtype (written in token order).
+ * Queues work on `stream` and returns without waiting. The first call for a given
+ * (H, D, dtype, k) allocates the plan's workspace; later calls allocate nothing.
+ * Not reentrant on one plan: calls that share a plan must be ordered on one stream.
+ */
+SSA_API ssa_status_t ssa_forward(ssa_plan_t plan, const void* q, const void* k, const void* v,
+                         const float* gates, const float* wc, int32_t heads, int32_t head_dim,
+                         ssa_dtype_t dtype, int32_t topk, void* out, void* stream);
+
+/* As ssa_forward, and also writes the selected blocks: sel_out device int32 [N, H, k] (global
+ * block indices; slot 0 = own block; -1 = empty slot). */
+SSA_API ssa_status_t ssa_forward_debug(ssa_plan_t plan, const void* q, const void* k, const void* v,
+                               const float* gates, const float* wc, int32_t heads,
+                               int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
+                               int32_t* sel_out, void* stream);
+
+/*
+ * ssa_forward on HOST buffers: copies q, k, v, gates, wc (host) to plan-owned device buffers,
+ * runs the forward and copies the result into out (host). Pinned host memory gives overlapped,
+ * full-speed copies; pageable memory works but is slower. Waits for the device before returning.
+ */
+SSA_API ssa_status_t ssa_forward_host(ssa_plan_t plan, const void* q, const void* k, const void* v,
+                              const float* gates, const float* wc, int32_t heads,
+                              int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
+                              void* stream);
+
+/*
+ * Backward pass (row a9): gradients of sum(dO * out) with respect to q, k, v, with the block
+ * selection held fixed (it is not differentiable) and the compressed tokens' rounding treated as
+ * identity. dq, dk, dv: device [N, H, D] of dtype. Accumulates in fp32 (CUDA cores); intended for
+ * correctness, not speed. Queues work and returns without waiting.
+ */
+SSA_API ssa_status_t ssa_backward(ssa_plan_t plan, const void* q, const void* k, const void* v,
+                          const float* gates, const float* wc, const void* dout, int32_t heads,
+                          int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* dq, void* dk,
+                          void* dv, void* stream);
+
+/* Wait for `stream`, then read and clear the plan's device status word. */
+SSA_API ssa_status_t ssa_last_device_status(ssa_plan_t plan, void* stream);
+
+/* Release a plan and every buffer it owns (queued on the stream it was created on). */
+SSA_API ssa_status_t ssa_plan_destroy(ssa_plan_t plan);
+
+/* Static description of a status code. */
+SSA_API const char* ssa_status_string(ssa_status_t status);
+
+/* Number of kernels this library has launched in the process so far. */
+SSA_API int64_t ssa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H */

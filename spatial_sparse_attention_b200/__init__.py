@@ -1,0 +1,209 @@
+"""Python binding of libssa.so: Spatial Sparse Attention forward on B200 (sm_100a).
+
+Argument marshalling only. Every step of the method runs in the library's CUDA kernels; PyTorch
+provides device memory and the current stream. There is no CPU fallback: importing this package
+without the built library raises.
+
+    plan = ssa.Plan(coords, grid=(192, 192, 192), r=3)          # rows a1, a2
+    out = plan.forward(q, k, v, gates, wc, topk=16)             # rows a3-a8
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssa.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "ssa.h")
+
+STATUS = {
+    0: "SSA_OK", 1: "SSA_ERR_INVALID_ARG", 2: "SSA_ERR_COORD_RANGE", 3: "SSA_ERR_DUPLICATE_COORD",
+    4: "SSA_ERR_ALLOC", 5: "SSA_ERR_CUDA", 6: "SSA_ERR_UNSUPPORTED", 7: "SSA_ERR_DEVICE_TIMEOUT",
+}
+_DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+
+
+class SSAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        self.name = STATUS.get(code, str(code))
+        super().__init__(f"{where}: {self.name}")
+
+
+_vp = ctypes.c_void_p
+_i32, _i64 = ctypes.c_int32, ctypes.c_int64
+_SIGS = {
+    "ssa_set_allocator": [_vp, _vp, _vp],
+    "ssa_plan": [_vp, _i64, _vp, _i32, _i32, _vp, _vp],
+    "ssa_plan_varlen": [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp],
+    "ssa_plan_info": [_vp, _vp, _vp, _vp, _vp],
+    "ssa_plan_export": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "ssa_forward": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp],
+    "ssa_forward_debug": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "ssa_forward_host": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp],
+    "ssa_backward": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
+    "ssa_last_device_status": [_vp, _vp],
+    "ssa_plan_destroy": [_vp],
+    "ssa_status_string": [_i32],
+    "ssa_launch_count": [],
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built (run spatial_sparse_attention_b200/build.py); "
+                          "there is no CPU fallback")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, args in _SIGS.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.ssa_status_string.restype = ctypes.c_char_p
+    lib.ssa_launch_count.restype = ctypes.c_int64
+    return lib
+
+
+lib = _load()
+
+
+def declared_symbols() -> Sequence[str]:
+    """Entry points declared in include/ssa.h."""
+    return re.findall(r"SSA_API\s+[\w\s\*]+?\b(ssa_\w+)\s*\(", open(HEADER).read())
+
+
+def launch_count() -> int:
+    return int(lib.ssa_launch_count())
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise SSAError(code, where)
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, dtype=None) -> torch.Tensor:
+    if not t.is_cuda or not t.is_contiguous() or (dtype is not None and t.dtype != dtype):
+        raise ValueError("expected a contiguous CUDA tensor" + (f" of {dtype}" if dtype else ""))
+    return t
+
+
+class Plan:
+    """Block partition and window lists of a packed batch of voxel token sequences.
+
+    coords: int32 CUDA tensor [N, 3]. Either `grid` (one sequence) or `cu_seqlens` + `grids`.
+    """
+
+    def __init__(self, coords: torch.Tensor, grid=None, r: int = 2, block: int = 8,
+                 cu_seqlens: Optional[Sequence[int]] = None, grids=None, stream=None):
+        _dev(coords, torch.int32)
+        self._h = _vp()
+        self.stream = stream
+        st = _stream(stream)
+        if cu_seqlens is None:
+            g = (ctypes.c_int32 * 3)(*[int(x) for x in grid])
+            _check(lib.ssa_plan(coords.data_ptr(), coords.shape[0], ctypes.addressof(g), block, r,
+                                st, ctypes.byref(self._h)), "ssa_plan")
+        else:
+            B = len(cu_seqlens) - 1
+            cu = (ctypes.c_int64 * (B + 1))(*[int(x) for x in cu_seqlens])
+            flat = [int(x) for row in grids for x in row]
+            gr = (ctypes.c_int32 * len(flat))(*flat)
+            _check(lib.ssa_plan_varlen(coords.data_ptr(), ctypes.addressof(cu), B,
+                                       ctypes.addressof(gr), block, r, st, ctypes.byref(self._h)),
+                   "ssa_plan_varlen")
+        n, mb, nnz, b = _i64(), _i64(), _i64(), _i32()
+        _check(lib.ssa_plan_info(self._h, ctypes.byref(n), ctypes.byref(mb), ctypes.byref(nnz),
+                                 ctypes.byref(b)), "ssa_plan_info")
+        self.N, self.num_blocks, self.nnz, self.batch = n.value, mb.value, nnz.value, b.value
+        self.r = r
+
+    def close(self):
+        if self._h:
+            lib.ssa_plan_destroy(self._h)
+            self._h = _vp()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def export(self):
+        """The canonical plan arrays as CUDA tensors (see ssa_plan_export)."""
+        dev = torch.device("cuda")
+        i32 = dict(dtype=torch.int32, device=dev)
+        out = dict(perm=torch.empty(self.N, **i32), tok_blk=torch.empty(self.N, **i32),
+                   blk_off=torch.empty(self.num_blocks + 1, **i32),
+                   blk_coord=torch.empty(self.num_blocks, 3, **i32),
+                   blk_seq=torch.empty(self.num_blocks, **i32),
+                   nbr_off=torch.empty(self.N + 1, dtype=torch.int64, device=dev),
+                   nbr_idx=torch.empty(max(self.nnz, 1), **i32))
+        _check(lib.ssa_plan_export(self._h, *[_ptr(out[k]) for k in
+                                              ("perm", "tok_blk", "blk_off", "blk_coord", "blk_seq",
+                                               "nbr_off", "nbr_idx")], _stream(self.stream)),
+               "ssa_plan_export")
+        out["nbr_idx"] = out["nbr_idx"][:self.nnz]
+        return out
+
+    def _args(self, q, k, v, gates, wc):
+        dt = q.dtype
+        for t in (q, k, v):
+            _dev(t, dt)
+            if t.dim() != 3 or t.shape[0] != self.N:
+                raise ValueError("q, k, v must be [N, H, D]")
+        _dev(gates, torch.float32)
+        _dev(wc, torch.float32)
+        return dt, q.shape[1], q.shape[2]
+
+    def forward(self, q, k, v, gates, wc, topk: int, out: Optional[torch.Tensor] = None,
+                return_sel: bool = False):
+        dt, H, D = self._args(q, k, v, gates, wc)
+        out = torch.empty_like(q) if out is None else _dev(out, dt)
+        st = _stream(self.stream)
+        if return_sel:
+            sel = torch.empty(self.N, H, topk, dtype=torch.int32, device=q.device)
+            _check(lib.ssa_forward_debug(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         gates.data_ptr(), wc.data_ptr(), H, D, _DTYPE[dt], topk,
+                                         out.data_ptr(), sel.data_ptr(), st), "ssa_forward_debug")
+            return out, sel
+        _check(lib.ssa_forward(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), gates.data_ptr(),
+                               wc.data_ptr(), H, D, _DTYPE[dt], topk, out.data_ptr(), st),
+               "ssa_forward")
+        return out
+
+    def forward_host(self, q, k, v, gates, wc, topk: int, out: torch.Tensor):
+        """Forward on host (preferably pinned) CPU tensors; copies run inside the library."""
+        for t in (q, k, v, gates, wc, out):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("forward_host takes contiguous CPU tensors")
+        H, D = q.shape[1], q.shape[2]
+        _check(lib.ssa_forward_host(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                    gates.data_ptr(), wc.data_ptr(), H, D, _DTYPE[q.dtype], topk,
+                                    out.data_ptr(), _stream(self.stream)), "ssa_forward_host")
+        return out
+
+    def backward(self, q, k, v, gates, wc, dout, topk: int):
+        dt, H, D = self._args(q, k, v, gates, wc)
+        _dev(dout, dt)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        _check(lib.ssa_backward(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                gates.data_ptr(), wc.data_ptr(), dout.data_ptr(), H, D,
+                                _DTYPE[dt], topk, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                _stream(self.stream)), "ssa_backward")
+        return dq, dk, dv
+
+    def status(self):
+        """Waits for the stream, returns and clears the device status (0 = ok)."""
+        return lib.ssa_last_device_status(self._h, _stream(self.stream))

@@ -1,0 +1,393 @@
+// C ABI of libssa.so (declared in include/ssa.h): argument validation, the plan object and its
+// device buffers, the cached forward workspace, and dispatch to the kernels.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "common.cuh"
+
+namespace ssa {
+
+std::atomic<int64_t> g_launches{0};
+
+namespace {
+
+void* default_alloc(size_t bytes, void* stream, void*) {
+    void* p = nullptr;
+    if (cudaMallocAsync(&p, bytes, (cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return p;
+}
+void default_free(void* p, void* stream, void*) { cudaFreeAsync(p, (cudaStream_t)stream); }
+
+std::mutex g_alloc_mu;
+ssa_alloc_fn g_alloc = default_alloc;
+ssa_free_fn g_free = default_free;
+void* g_alloc_ctx = nullptr;
+
+bool check_device(ssa_status_t* st) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        *st = SSA_ERR_CUDA;
+        return false;
+    }
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (major != 10) {
+        *st = SSA_ERR_UNSUPPORTED;
+        return false;
+    }
+    return true;
+}
+
+size_t elem_size(ssa_dtype_t t) { return t == SSA_F32 ? 4 : 2; }
+
+void destroy(Plan* p) {
+    ssa_plan_s* h = static_cast<ssa_plan_s*>(p);
+    if (!p) return;
+    plan_free_all(p, p->ws.owned);
+    plan_free_all(p, p->owned);
+    if (p->ws.h_q) cudaStreamSynchronize(p->stream);
+    delete h;
+}
+
+ssa_status_t map_device_status(int32_t s) {
+    if (!s) return SSA_OK;
+    if (s & DEV_TIMEOUT) return SSA_ERR_DEVICE_TIMEOUT;
+    if (s & DEV_COORD_RANGE) return SSA_ERR_COORD_RANGE;
+    if (s & DEV_DUPLICATE) return SSA_ERR_DUPLICATE_COORD;
+    if (s & DEV_TOO_LARGE) return SSA_ERR_UNSUPPORTED;
+    return SSA_ERR_CUDA;
+}
+
+ssa_status_t make_plan(const int32_t* coords, const int64_t* cu, int32_t B, const int32_t* grids,
+                       int32_t block, int32_t r, void* stream, ssa_plan_t* out) {
+    if (!out) return SSA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!coords || !cu || !grids || B < 1 || B > 65535) return SSA_ERR_INVALID_ARG;
+    if (block != kBlockEdge || r < 0 || r > kBlockEdge) return SSA_ERR_UNSUPPORTED;
+    if (cu[0] != 0) return SSA_ERR_INVALID_ARG;
+    for (int s = 0; s < B; ++s) {
+        if (cu[s + 1] < cu[s]) return SSA_ERR_INVALID_ARG;
+        for (int a = 0; a < 3; ++a)
+            if (grids[3 * s + a] < 1 || grids[3 * s + a] > 65535) return SSA_ERR_INVALID_ARG;
+    }
+    const int64_t N = cu[B];
+    if (N < 1 || N >= (int64_t)1 << 26) return SSA_ERR_INVALID_ARG;
+    ssa_status_t st = SSA_OK;
+    if (!check_device(&st)) return st;
+
+    ssa_plan_s* p = new (std::nothrow) ssa_plan_s();
+    if (!p) return SSA_ERR_ALLOC;
+    {
+        std::lock_guard<std::mutex> lk(g_alloc_mu);
+        p->alloc = g_alloc;
+        p->release = g_free;
+        p->alloc_ctx = g_alloc_ctx;
+    }
+    cudaGetDevice(&p->device);
+    p->stream = (cudaStream_t)stream;
+    p->N = N;
+    p->B = B;
+    p->r = r;
+    int64_t dense = 0;
+    for (int s = 0; s < B; ++s) {
+        SeqInfo q;
+        q.lo = cu[s];
+        q.hi = cu[s + 1];
+        q.gx = grids[3 * s];
+        q.gy = grids[3 * s + 1];
+        q.gz = grids[3 * s + 2];
+        q.gbx = (int32_t)cdiv(q.gx, kBlockEdge);
+        q.gby = (int32_t)cdiv(q.gy, kBlockEdge);
+        q.gbz = (int32_t)cdiv(q.gz, kBlockEdge);
+        q.dense_base = dense;
+        dense += (int64_t)q.gbx * q.gby * q.gbz;
+        p->seqs.push_back(q);
+    }
+    p->G = dense;
+    if (p->G >= ((int64_t)1 << 30)) {
+        delete p;
+        return SSA_ERR_UNSUPPORTED;
+    }
+    st = build_plan(p, coords, (cudaStream_t)stream);
+    if (st != SSA_OK) {
+        cudaStreamSynchronize((cudaStream_t)stream);
+        cudaGetLastError();
+        destroy(p);
+        return st;
+    }
+    *out = p;
+    return SSA_OK;
+}
+
+// (Re)allocates the forward workspace for (H, D, dtype, k) if the cached one does not match.
+ssa_status_t ensure_workspace(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int32_t k,
+                              cudaStream_t st) {
+    Workspace& w = p->ws;
+    if (w.H == H && w.D == D && w.dtype == dt && w.k == k && w.kc) return SSA_OK;
+    plan_free_all(p, w.owned);
+    w = Workspace();
+    const size_t es = elem_size(dt);
+    const int64_t N = p->N, Mb = p->Mb;
+    auto A = [&](size_t bytes) -> void* {
+        void* ptr = p->alloc(std::max<size_t>(bytes, 16), st, p->alloc_ctx);
+        if (ptr) w.owned.push_back(ptr);
+        return ptr;
+    };
+    w.kc = A(es * H * Mb * D);
+    w.vc = A(es * H * Mb * D);
+    w.sel = (int32_t*)A(sizeof(int32_t) * N * H * k);
+    if (!w.kc || !w.vc || !w.sel) return SSA_ERR_ALLOC;
+    if (dt != SSA_F32) {
+        const int64_t HMb = (int64_t)H * Mb;
+        w.ks = A(es * H * p->Npad * D);
+        w.vs = A(es * H * p->Npad * D);
+        w.base = (float*)A(sizeof(float) * N * H * D);
+        w.part_o = A(es * N * H * k * D);
+        w.part_lse = (float*)A(sizeof(float) * N * H * k);
+        w.inv_cnt = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
+        w.inv_off = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
+        w.inv_fill = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
+        w.inv_list = (int32_t*)A(sizeof(int32_t) * std::max<int64_t>(1, N * H * (k - 1)));
+        w.item_cnt = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
+        w.item_off = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
+        w.scan_tmp_len = scan_tmp_len(HMb + 1);
+        w.scan_tmp = (int32_t*)A(sizeof(int32_t) * w.scan_tmp_len);
+        if (!w.ks || !w.vs || !w.base || !w.part_o || !w.part_lse || !w.inv_cnt || !w.inv_off ||
+            !w.inv_fill || !w.inv_list || !w.item_cnt || !w.item_off || !w.scan_tmp)
+            return SSA_ERR_ALLOC;
+        // padding rows of the block-ordered copies stay zero for the life of the workspace
+        if (cudaMemsetAsync(w.ks, 0, es * H * p->Npad * D, st) ||
+            cudaMemsetAsync(w.vs, 0, es * H * p->Npad * D, st))
+            return SSA_ERR_CUDA;
+    }
+    w.H = H;
+    w.D = D;
+    w.dtype = dt;
+    w.k = k;
+    return SSA_OK;
+}
+
+ssa_status_t check_forward_args(Plan* p, const void* q, const void* k, const void* v,
+                                const float* gates, const float* wc, int32_t H, int32_t D,
+                                ssa_dtype_t dt, int32_t topk, const void* out) {
+    if (!p || !q || !k || !v || !gates || !wc || !out) return SSA_ERR_INVALID_ARG;
+    if (dt != SSA_F32 && dt != SSA_BF16 && dt != SSA_F16) return SSA_ERR_INVALID_ARG;
+    if (H < 1 || topk < 1) return SSA_ERR_INVALID_ARG;
+    if (topk > kMaxTopk) return SSA_ERR_UNSUPPORTED;
+    if (D != 32 && D != 64 && D != 96 && D != 128) return SSA_ERR_UNSUPPORTED;
+    const int64_t hd = (int64_t)H * D;
+    if (hd > (dt == SSA_F32 ? 8192 : 16384)) return SSA_ERR_UNSUPPORTED;
+    if (p->N * H >= ((int64_t)1 << 31) / std::max(topk, 1)) return SSA_ERR_UNSUPPORTED;
+    return SSA_OK;
+}
+
+ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, const float* gates,
+                         const float* wc, int32_t H, int32_t D, ssa_dtype_t dt, int32_t topk,
+                         void* out, int32_t* sel_out, cudaStream_t st) {
+    ssa_status_t rc = ensure_workspace(p, H, D, dt, topk, st);
+    if (rc != SSA_OK) return rc;
+    const Workspace& w = p->ws;
+    launch_pool(p, w, k, v, wc, st);
+    if (dt == SSA_F32) launch_forward_simt(p, w, q, k, v, gates, out, st);
+    else launch_forward_tc(p, w, q, gates, out, st);
+    if (sel_out) launch_export_sel(p, w, sel_out, st);
+    return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+}  // namespace
+
+void* plan_alloc(Plan* p, size_t bytes) {
+    void* ptr = p->alloc(std::max<size_t>(bytes, 16), p->stream, p->alloc_ctx);
+    if (ptr) p->owned.push_back(ptr);
+    return ptr;
+}
+
+void plan_free_all(Plan* p, std::vector<void*>& list) {
+    for (void* ptr : list) p->release(ptr, p->stream, p->alloc_ctx);
+    list.clear();
+}
+
+}  // namespace ssa
+
+using namespace ssa;
+
+extern "C" {
+
+ssa_status_t ssa_set_allocator(ssa_alloc_fn alloc, ssa_free_fn release, void* ctx) {
+    if ((alloc == nullptr) != (release == nullptr)) return SSA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_alloc_mu);
+    g_alloc = alloc ? alloc : default_alloc;
+    g_free = release ? release : default_free;
+    g_alloc_ctx = alloc ? ctx : nullptr;
+    return SSA_OK;
+}
+
+ssa_status_t ssa_plan(const int32_t* coords, int64_t n, const int32_t grid[3], int32_t block,
+                      int32_t r, void* stream, ssa_plan_t* out) {
+    if (!grid || n < 1) return SSA_ERR_INVALID_ARG;
+    int64_t cu[2] = {0, n};
+    return make_plan(coords, cu, 1, grid, block, r, stream, out);
+}
+
+ssa_status_t ssa_plan_varlen(const int32_t* coords, const int64_t* cu_seqlens, int32_t batch,
+                             const int32_t* grids, int32_t block, int32_t r, void* stream,
+                             ssa_plan_t* out) {
+    return make_plan(coords, cu_seqlens, batch, grids, block, r, stream, out);
+}
+
+ssa_status_t ssa_plan_info(ssa_plan_t plan, int64_t* n, int64_t* num_blocks, int64_t* nnz,
+                           int32_t* batch) {
+    if (!plan) return SSA_ERR_INVALID_ARG;
+    if (n) *n = plan->N;
+    if (num_blocks) *num_blocks = plan->Mb;
+    if (nnz) *nnz = plan->nnz;
+    if (batch) *batch = plan->B;
+    return SSA_OK;
+}
+
+ssa_status_t ssa_plan_export(ssa_plan_t p, int32_t* perm, int32_t* tok_blk, int32_t* blk_off,
+                             int32_t* blk_coord, int32_t* blk_seq, int64_t* nbr_off,
+                             int32_t* nbr_idx, void* stream) {
+    if (!p) return SSA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const auto D2D = cudaMemcpyDeviceToDevice;
+    cudaError_t e = cudaSuccess;
+    if (perm && !e) e = cudaMemcpyAsync(perm, p->perm, sizeof(int32_t) * p->N, D2D, st);
+    if (tok_blk && !e) e = cudaMemcpyAsync(tok_blk, p->tok_blk, sizeof(int32_t) * p->N, D2D, st);
+    if (blk_off && !e) e = cudaMemcpyAsync(blk_off, p->blk_off, sizeof(int32_t) * (p->Mb + 1), D2D, st);
+    if (blk_coord && !e) e = cudaMemcpyAsync(blk_coord, p->blk_coord, sizeof(int32_t) * 3 * p->Mb, D2D, st);
+    if (blk_seq && !e) e = cudaMemcpyAsync(blk_seq, p->blk_seq, sizeof(int32_t) * p->Mb, D2D, st);
+    if (nbr_idx && !e && p->nnz) e = cudaMemcpyAsync(nbr_idx, p->nbr_idx, sizeof(int32_t) * p->nnz, D2D, st);
+    if (nbr_off && !e) {
+        std::vector<int32_t> h32(p->N + 1);
+        std::vector<int64_t> h64(p->N + 1);
+        e = cudaMemcpyAsync(h32.data(), p->nbr_off32, sizeof(int32_t) * (p->N + 1), cudaMemcpyDeviceToHost, st);
+        if (!e) e = cudaStreamSynchronize(st);
+        for (int64_t i = 0; i <= p->N && !e; ++i) h64[i] = h32[i];
+        if (!e) e = cudaMemcpyAsync(nbr_off, h64.data(), sizeof(int64_t) * (p->N + 1), cudaMemcpyHostToDevice, st);
+    }
+    if (!e) e = cudaStreamSynchronize(st);
+    return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+ssa_status_t ssa_forward(ssa_plan_t p, const void* q, const void* k, const void* v,
+                         const float* gates, const float* wc, int32_t heads, int32_t head_dim,
+                         ssa_dtype_t dtype, int32_t topk, void* out, void* stream) {
+    ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out);
+    if (rc != SSA_OK) return rc;
+    return run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, nullptr,
+                       (cudaStream_t)stream);
+}
+
+ssa_status_t ssa_forward_debug(ssa_plan_t p, const void* q, const void* k, const void* v,
+                               const float* gates, const float* wc, int32_t heads,
+                               int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
+                               int32_t* sel_out, void* stream) {
+    ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out);
+    if (rc != SSA_OK) return rc;
+    if (!sel_out) return SSA_ERR_INVALID_ARG;
+    return run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, sel_out,
+                       (cudaStream_t)stream);
+}
+
+ssa_status_t ssa_forward_host(ssa_plan_t p, const void* q, const void* k, const void* v,
+                              const float* gates, const float* wc, int32_t heads,
+                              int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
+                              void* stream) {
+    ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out);
+    if (rc != SSA_OK) return rc;
+    cudaStream_t st = (cudaStream_t)stream;
+    Workspace& w = p->ws;
+    const size_t tb = elem_size(dtype) * (size_t)p->N * heads * head_dim;
+    const size_t gb = sizeof(float) * (size_t)p->N * heads * 3;
+    const size_t wb = sizeof(float) * (size_t)head_dim * head_dim;
+    rc = ensure_workspace(p, heads, head_dim, dtype, topk, st);
+    if (rc != SSA_OK) return rc;
+    if (!w.h_q) {
+        void* bufs[6];
+        const size_t sizes[6] = {tb, tb, tb, tb, gb, wb};
+        for (int i = 0; i < 6; ++i) {
+            bufs[i] = p->alloc(sizes[i], st, p->alloc_ctx);
+            if (!bufs[i]) return SSA_ERR_ALLOC;
+            w.owned.push_back(bufs[i]);
+        }
+        w.h_q = bufs[0];
+        w.h_k = bufs[1];
+        w.h_v = bufs[2];
+        w.h_out = bufs[3];
+        w.h_gates = (float*)bufs[4];
+        w.h_wc = (float*)bufs[5];
+    }
+    const auto H2D = cudaMemcpyHostToDevice;
+    if (cudaMemcpyAsync(w.h_q, q, tb, H2D, st) || cudaMemcpyAsync(w.h_k, k, tb, H2D, st) ||
+        cudaMemcpyAsync(w.h_v, v, tb, H2D, st) || cudaMemcpyAsync(w.h_gates, gates, gb, H2D, st) ||
+        cudaMemcpyAsync(w.h_wc, wc, wb, H2D, st))
+        return SSA_ERR_CUDA;
+    rc = run_forward(p, w.h_q, w.h_k, w.h_v, w.h_gates, w.h_wc, heads, head_dim, dtype, topk,
+                     w.h_out, nullptr, st);
+    if (rc != SSA_OK) return rc;
+    if (cudaMemcpyAsync(out, w.h_out, tb, cudaMemcpyDeviceToHost, st) || cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    int32_t s = 0;
+    if (cudaMemcpy(&s, p->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost)) return SSA_ERR_CUDA;
+    return map_device_status(s);
+}
+
+ssa_status_t ssa_backward(ssa_plan_t p, const void* q, const void* k, const void* v,
+                          const float* gates, const float* wc, const void* dout, int32_t heads,
+                          int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* dq, void* dk,
+                          void* dv, void* stream) {
+    ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, dq);
+    if (rc != SSA_OK) return rc;
+    if (!dout || !dk || !dv) return SSA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    rc = ensure_workspace(p, heads, head_dim, dtype, topk, st);
+    if (rc != SSA_OK) return rc;
+    // the selection is the forward's: run the forward path to produce it (output goes to dq,
+    // which the backward overwrites)
+    rc = run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, dq, nullptr, st);
+    if (rc != SSA_OK) return rc;
+    return launch_backward(p, p->ws, q, k, v, gates, wc, dout, dq, dk, dv, st);
+}
+
+ssa_status_t ssa_last_device_status(ssa_plan_t p, void* stream) {
+    if (!p) return SSA_ERR_INVALID_ARG;
+    int32_t s = 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(st) ||
+        cudaMemcpyAsync(&s, p->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaMemsetAsync(p->d_status, 0, sizeof(int32_t), st) || cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    return map_device_status(s);
+}
+
+ssa_status_t ssa_plan_destroy(ssa_plan_t p) {
+    if (!p) return SSA_ERR_INVALID_ARG;
+    destroy(p);
+    return SSA_OK;
+}
+
+const char* ssa_status_string(ssa_status_t s) {
+    switch (s) {
+    case SSA_OK: return "ok";
+    case SSA_ERR_INVALID_ARG: return "invalid argument";
+    case SSA_ERR_COORD_RANGE: return "coordinate outside the grid";
+    case SSA_ERR_DUPLICATE_COORD: return "duplicate coordinate";
+    case SSA_ERR_ALLOC: return "device allocation failed";
+    case SSA_ERR_CUDA: return "CUDA error";
+    case SSA_ERR_UNSUPPORTED: return "unsupported size or device";
+    case SSA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int64_t ssa_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

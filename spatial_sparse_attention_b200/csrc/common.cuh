@@ -1,0 +1,189 @@
+// Internal definitions shared by the translation units of libssa.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <vector>
+
+#include "../../include/ssa.h"
+
+namespace ssa {
+
+// Bits of the device status word (one int32 per plan). Kernels OR these in; the host maps them to
+// ssa_status_t when it next waits for the device.
+enum : int32_t {
+    DEV_COORD_RANGE = 1,
+    DEV_DUPLICATE = 2,
+    DEV_TIMEOUT = 4,
+    DEV_BAD_INDEX = 8,
+    DEV_TOO_LARGE = 16,
+};
+
+constexpr int kBlockEdge = 8;      // block edge in voxels (the only supported value)
+constexpr int kPad = 16;           // blocks start on multiples of 16 rows in the sorted K/V copies
+constexpr int kQTile = 128;        // query rows per tensor-core tile
+constexpr int kMaxTopk = 32;
+
+// Per-sequence constants, mirrored on the device.
+struct SeqInfo {
+    int64_t lo, hi;          // token range [lo, hi)
+    int64_t dense_base;      // first dense block key of this sequence
+    int32_t gx, gy, gz;      // grid extent
+    int32_t gbx, gby, gbz;   // blocks per axis (ceil(g / 8))
+};
+
+// Forward workspace, cached in the plan for one (H, D, dtype, k).
+struct Workspace {
+    int32_t H = 0, D = 0, k = 0;
+    ssa_dtype_t dtype = SSA_F32;
+    void* ks = nullptr;        // [H, Npad, D] T   K rows in padded block order
+    void* vs = nullptr;        // [H, Npad, D] T
+    void* kc = nullptr;        // [H, Mb, D]   T (fp32 for the fp32 path)
+    void* vc = nullptr;        // [H, Mb, D]
+    float* base = nullptr;     // [N, H, D]    g0*o_cmp + g2*o_win, sorted token order
+    void* part_o = nullptr;    // [N, H, k, D] T   per-(query, head, slot) normalised partial output
+    float* part_lse = nullptr; // [N, H, k]        log2-sum-exp of each partial
+    int32_t* sel = nullptr;    // [N, H, k]        selected blocks, sorted token order
+    int32_t* inv_cnt = nullptr;  // [H*Mb + 1]
+    int32_t* inv_off = nullptr;  // [H*Mb + 1]
+    int32_t* inv_fill = nullptr; // [H*Mb]
+    int32_t* inv_list = nullptr; // [N*H*(k-1)]  (sorted query position << 5 | slot)
+    int32_t* item_cnt = nullptr; // [H*Mb + 1]   tiles per (head, block)
+    int32_t* item_off = nullptr; // [H*Mb + 1]
+    int32_t* scan_tmp = nullptr;
+    int64_t scan_tmp_len = 0;
+    // host-buffer entry point staging (allocated on first use)
+    void* h_q = nullptr; void* h_k = nullptr; void* h_v = nullptr; void* h_out = nullptr;
+    float* h_gates = nullptr; float* h_wc = nullptr;
+    std::vector<void*> owned;
+};
+
+struct Plan {
+    int device = 0;
+    cudaStream_t stream = nullptr;  // creation stream (frees are queued here)
+    ssa_alloc_fn alloc = nullptr;
+    ssa_free_fn release = nullptr;
+    void* alloc_ctx = nullptr;
+
+    int64_t N = 0;
+    int32_t B = 0;
+    int32_t r = 0;
+    int64_t G = 0;       // dense block keys over all sequences
+    int64_t Mb = 0;      // occupied blocks
+    int64_t Npad = 0;    // padded sorted rows
+    int64_t nnz = 0;     // window neighbour pairs
+    int64_t n_qtiles = 0;
+    std::vector<SeqInfo> seqs;
+    std::vector<int64_t> seq_blk;   // [B+1] block range of each sequence (host copy)
+
+    SeqInfo* d_seqs = nullptr;
+    int32_t* d_status = nullptr;
+    int32_t* coords = nullptr;   // [N,3] copy of the input coordinates
+    int32_t* perm = nullptr;     // [N]
+    int32_t* tok_blk = nullptr;  // [N]
+    int32_t* tok_pos = nullptr;  // [N]  position in perm
+    int32_t* blk_off = nullptr;  // [Mb+1]
+    int32_t* blk_poff = nullptr; // [Mb+1] padded row offsets
+    int32_t* blk_coord = nullptr;// [Mb,3]
+    int32_t* blk_seq = nullptr;  // [Mb]
+    int32_t* seq_blk_d = nullptr;// [B+1]
+    int32_t* spos_tok = nullptr; // [Npad] token of each padded row, -1 for padding
+    int4* scoord = nullptr;      // [Npad] (x, y, z, block) of each padded row; padding far away
+    int32_t* nbr_off32 = nullptr;// [N+1]
+    int32_t* nbr_idx = nullptr;  // [nnz]
+    int32_t* qt_pos = nullptr;   // [n_qtiles] first sorted position of each query tile
+    int32_t* qt_len = nullptr;   // [n_qtiles]
+    int32_t* qt_seq = nullptr;   // [n_qtiles]
+    int32_t* wt_off = nullptr;   // [n_qtiles+1] window key union per query tile (CSR)
+    int32_t* wt_keys = nullptr;  // padded rows, ascending
+    std::vector<void*> owned;
+    Workspace ws;
+};
+
+extern std::atomic<int64_t> g_launches;
+inline void note_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// ---- allocation through the plan's hook -------------------------------------------------------
+void* plan_alloc(Plan* p, size_t bytes);
+void plan_free_all(Plan* p, std::vector<void*>& list);
+
+// ---- launchers implemented in the .cu files ---------------------------------------------------
+// scan.cu: out[i] = sum_{t<i} in[t] for i in [0, n], out[n] = total. `tmp` holds scan_tmp_len(n)
+// ints. In-place (out == in) is allowed.
+int64_t scan_tmp_len(int64_t n);
+void scan_exclusive(const int32_t* in, int32_t* out, int64_t n, int32_t* tmp, cudaStream_t s);
+
+// plan.cu
+ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t s);
+
+// pool.cu
+void launch_pool(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,
+                 cudaStream_t s);
+
+// attn_simt.cu (fp32 path)
+void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const void* k,
+                         const void* v, const float* gates, void* out, cudaStream_t s);
+
+// attn_tc.cu (bf16 / fp16 path)
+void launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
+                       void* out, cudaStream_t s);
+
+// backward.cu
+ssa_status_t launch_backward(Plan* p, const Workspace& w, const void* q, const void* k,
+                             const void* v, const float* gates, const float* wc, const void* dout,
+                             void* dq, void* dk, void* dv, cudaStream_t s);
+
+// selection export (attn_tc.cu): sel_out [N,H,k] in token order from the sorted-order buffer.
+void launch_export_sel(const Plan* p, const Workspace& w, int32_t* sel_out, cudaStream_t s);
+
+// ---- small device helpers -------------------------------------------------------------------
+__host__ __device__ inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float to_f(float x) { return x; }
+    static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Elem<__half> {
+    static __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+    static __device__ __forceinline__ __half from_f(float x) { return __float2half_rn(x); }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// Packed (sequence, x, y, z) key of the coordinate hash; each field < 2^16.
+__device__ __forceinline__ uint64_t pack_cell(int32_t s, int32_t x, int32_t y, int32_t z) {
+    return ((uint64_t)(uint32_t)s << 48) | ((uint64_t)(uint32_t)x << 32) |
+           ((uint64_t)(uint32_t)y << 16) | (uint64_t)(uint32_t)z;
+}
+// MurmurHash3 64-bit finaliser: spreads packed keys over the table.
+__device__ __forceinline__ uint64_t mix64(uint64_t k) {
+    k ^= k >> 33;
+    k *= 0xff51afd7ed558ccdULL;
+    k ^= k >> 33;
+    k *= 0xc4ceb9fe1a85ec53ULL;
+    k ^= k >> 33;
+    return k;
+}
+constexpr uint64_t kEmptyCell = ~0ULL;
+
+__device__ __forceinline__ int find_seq(const SeqInfo* seqs, int B, int64_t i) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (seqs[mid].lo <= i) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+}  // namespace ssa
+
+// The opaque handle of the C ABI is the plan itself.
+struct ssa_plan_s : public ssa::Plan {};

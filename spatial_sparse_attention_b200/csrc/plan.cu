@@ -1,0 +1,537 @@
+// Plan kernels: coordinate-block partition (row a1) and coordinate hash + window neighbour lists
+// (row a2).
+//
+// Direct3D-S2 model page, "What is Direct3D-S2?": SSA partitions sparse tokens by their 3D
+// coordinates. Direct3D-S2 summary page, "Technical principles", SSA item: compression per
+// block, block selection, local window.
+//
+// Partition: every token gets a dense block key (sequence base + (bx*GBy + by)*GBz + bz); a
+// histogram over the dense key space, an occupancy scan and a block-size scan give the block
+// CSR with blocks in lexicographic (bx, by, bz) order; a counting scatter followed by a per-block
+// sort puts the tokens of each block in ascending index order. Window: tokens are inserted in
+// an open-addressing hash of packed (sequence, x, y, z); each token probes the (2r+1)^3 cells
+// around it (count pass, scan, fill pass with a per-row sort).
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace ssa {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+inline unsigned grid_for(int64_t n, int threads = kThreads) {
+    int64_t g = cdiv(n > 0 ? n : 1, threads);
+    return (unsigned)std::min<int64_t>(g, 1 << 30);
+}
+
+// Sorts buf[0..cap) ascending with one warp (cap a power of two).
+__device__ void warp_bitonic_sort(int32_t* buf, int cap) {
+    const int lane = threadIdx.x & 31;
+    for (int k = 2; k <= cap; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = lane; i < cap; i += 32) {
+                int ixj = i ^ j;
+                if (ixj > i) {
+                    int32_t a = buf[i], b = buf[ixj];
+                    bool up = (i & k) == 0;
+                    if ((a > b) == up) {
+                        buf[i] = b;
+                        buf[ixj] = a;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+__device__ __forceinline__ int32_t hash_find(const uint64_t* __restrict__ hkeys,
+                                             const int32_t* __restrict__ hvals, uint64_t hmask,
+                                             uint64_t key) {
+    uint64_t slot = mix64(key) & hmask;
+    for (uint64_t probe = 0; probe <= hmask; ++probe) {
+        uint64_t k = hkeys[slot];
+        if (k == key) return hvals[slot];
+        if (k == kEmptyCell) return -1;
+        slot = (slot + 1) & hmask;
+    }
+    return -1;
+}
+
+// Validates coordinates, computes dense block keys, counts tokens per key and inserts every token
+// in the coordinate hash (duplicates flagged).
+__global__ void k_keys_and_hash(const int32_t* __restrict__ coords, int64_t N,
+                                const SeqInfo* __restrict__ seqs, int B,
+                                int32_t* __restrict__ tok_key, int32_t* __restrict__ key_cnt,
+                                uint64_t* __restrict__ hkeys, int32_t* __restrict__ hvals,
+                                uint64_t hmask, int32_t* __restrict__ status) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    int s = find_seq(seqs, B, i);
+    const SeqInfo q = seqs[s];
+    int32_t x = coords[3 * i], y = coords[3 * i + 1], z = coords[3 * i + 2];
+    if (x < 0 || y < 0 || z < 0 || x >= q.gx || y >= q.gy || z >= q.gz) {
+        atomicOr(status, DEV_COORD_RANGE);
+        tok_key[i] = -1;
+        return;
+    }
+    int64_t key = q.dense_base + ((int64_t)(x / kBlockEdge) * q.gby + (y / kBlockEdge)) * q.gbz +
+                  (z / kBlockEdge);
+    tok_key[i] = (int32_t)key;
+    atomicAdd(&key_cnt[key], 1);
+    uint64_t cell = pack_cell(s, x, y, z);
+    uint64_t slot = mix64(cell) & hmask;
+    for (uint64_t probe = 0; probe <= hmask; ++probe) {
+        unsigned long long prev = atomicCAS((unsigned long long*)&hkeys[slot],
+                                            (unsigned long long)kEmptyCell,
+                                            (unsigned long long)cell);
+        if (prev == kEmptyCell) {
+            hvals[slot] = (int32_t)i;
+            return;
+        }
+        if (prev == cell) {
+            atomicOr(status, DEV_DUPLICATE);
+            return;
+        }
+        slot = (slot + 1) & hmask;
+    }
+    atomicOr(status, DEV_TOO_LARGE);  // table full: cannot happen with 2N slots
+}
+
+__global__ void k_occupied(const int32_t* __restrict__ key_cnt, int64_t G, int32_t* __restrict__ flag) {
+    int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (k < G) flag[k] = key_cnt[k] > 0;
+}
+
+// For every occupied dense key: its block index, size, padded size, coordinates and sequence.
+__global__ void k_blocks(const int32_t* __restrict__ key_cnt, const int32_t* __restrict__ bidx,
+                         int64_t G, const SeqInfo* __restrict__ seqs, int B,
+                         int32_t* __restrict__ key2blk, int32_t* __restrict__ blk_cnt,
+                         int32_t* __restrict__ blk_pcnt, int32_t* __restrict__ blk_coord,
+                         int32_t* __restrict__ blk_seq) {
+    int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= G) return;
+    int32_t c = key_cnt[k];
+    if (c == 0) {
+        key2blk[k] = -1;
+        return;
+    }
+    int32_t b = bidx[k];
+    key2blk[k] = b;
+    blk_cnt[b] = c;
+    blk_pcnt[b] = (int32_t)round_up(c, kPad);
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (seqs[mid].dense_base <= k) lo = mid; else hi = mid - 1;
+    }
+    const SeqInfo q = seqs[lo];
+    int64_t local = k - q.dense_base;
+    blk_coord[3 * b + 2] = (int32_t)(local % q.gbz);
+    blk_coord[3 * b + 1] = (int32_t)((local / q.gbz) % q.gby);
+    blk_coord[3 * b + 0] = (int32_t)(local / ((int64_t)q.gbz * q.gby));
+    blk_seq[b] = lo;
+}
+
+// One warp per token: probe every cell of the (2r+1)^3 cube, count (fill == false) or write the
+// found neighbours sorted ascending (fill == true).
+template <bool kFill>
+__global__ void k_neighbours(const int32_t* __restrict__ coords, int64_t N,
+                             const SeqInfo* __restrict__ seqs, int B, int r,
+                             const uint64_t* __restrict__ hkeys, const int32_t* __restrict__ hvals,
+                             uint64_t hmask, int32_t* __restrict__ nbr_cnt,
+                             const int32_t* __restrict__ nbr_off, int32_t* __restrict__ nbr_idx,
+                             int cap, int32_t* __restrict__ status) {
+    extern __shared__ int32_t sbuf[];
+    const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
+    int64_t i = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib;
+    if (i >= N) return;
+    int32_t* buf = sbuf + (int64_t)wib * cap;
+    int s = find_seq(seqs, B, i);
+    const SeqInfo q = seqs[s];
+    int32_t x = coords[3 * i], y = coords[3 * i + 1], z = coords[3 * i + 2];
+    const int w = 2 * r + 1;
+    const int cube = w * w * w;
+    int count = 0;
+    for (int o0 = 0; o0 < cube; o0 += 32) {
+        int o = o0 + lane;
+        int32_t j = -1;
+        if (o < cube) {
+            int dz = o % w - r, dy = (o / w) % w - r, dx = o / (w * w) - r;
+            int32_t xx = x + dx, yy = y + dy, zz = z + dz;
+            if (xx >= 0 && yy >= 0 && zz >= 0 && xx < q.gx && yy < q.gy && zz < q.gz)
+                j = hash_find(hkeys, hvals, hmask, pack_cell(s, xx, yy, zz));
+        }
+        unsigned found = __ballot_sync(0xffffffffu, j >= 0);
+        if (kFill && j >= 0) buf[count + __popc(found & ((1u << lane) - 1))] = j;
+        count += __popc(found);
+    }
+    if (!kFill) {
+        if (lane == 0) nbr_cnt[i] = count;
+        return;
+    }
+    __syncwarp();
+    if (count != nbr_off[i + 1] - nbr_off[i]) {
+        if (lane == 0) atomicOr(status, DEV_BAD_INDEX);
+        return;
+    }
+    for (int t = count + lane; t < cap; t += 32) buf[t] = 0x7fffffff;
+    __syncwarp();
+    warp_bitonic_sort(buf, cap);
+    for (int t = lane; t < count; t += 32) nbr_idx[nbr_off[i] + t] = buf[t];
+}
+
+// Counting scatter of tokens into their blocks (order inside a block fixed by k_sort_blocks).
+__global__ void k_scatter(const int32_t* __restrict__ tok_key, const int32_t* __restrict__ key2blk,
+                          int64_t N, const int32_t* __restrict__ blk_off,
+                          int32_t* __restrict__ blk_fill, int32_t* __restrict__ perm,
+                          int32_t* __restrict__ tok_blk) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    int32_t b = key2blk[tok_key[i]];
+    tok_blk[i] = b;
+    int32_t pos = blk_off[b] + atomicAdd(&blk_fill[b], 1);
+    perm[pos] = (int32_t)i;
+}
+
+// One warp per block: sort the block's slice of perm ascending (a block holds at most 512 cells).
+__global__ void k_sort_blocks(int32_t* __restrict__ perm, const int32_t* __restrict__ blk_off,
+                              int64_t Mb) {
+    __shared__ int32_t sbuf[8][512];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    int64_t b = (int64_t)blockIdx.x * 8 + wib;
+    if (b >= Mb) return;
+    int32_t lo = blk_off[b], n = blk_off[b + 1] - lo;
+    int cap = 32;
+    while (cap < n) cap <<= 1;
+    int32_t* buf = sbuf[wib];
+    for (int t = lane; t < cap; t += 32) buf[t] = t < n ? perm[lo + t] : 0x7fffffff;
+    __syncwarp();
+    warp_bitonic_sort(buf, cap);
+    for (int t = lane; t < n; t += 32) perm[lo + t] = buf[t];
+}
+
+// Sorted and padded positions of every token, and the per-row tables of the padded layout.
+__global__ void k_positions(const int32_t* __restrict__ perm, const int32_t* __restrict__ tok_blk,
+                            const int32_t* __restrict__ blk_off, const int32_t* __restrict__ blk_poff,
+                            const int32_t* __restrict__ coords, int64_t N,
+                            int32_t* __restrict__ tok_pos, int32_t* __restrict__ spos_tok,
+                            int4* __restrict__ scoord) {
+    int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= N) return;
+    int32_t i = perm[p];
+    int32_t b = tok_blk[i];
+    int32_t sp = blk_poff[b] + ((int32_t)p - blk_off[b]);
+    tok_pos[i] = (int32_t)p;
+    spos_tok[sp] = i;
+    scoord[sp] = make_int4(coords[3 * i], coords[3 * i + 1], coords[3 * i + 2], b);
+}
+
+__global__ void k_fill_i32(int32_t* __restrict__ a, int64_t n, int32_t v) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) a[i] = v;
+}
+
+__global__ void k_fill_int4(int4* __restrict__ a, int64_t n, int4 v) {
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) a[i] = v;
+}
+
+// Per query tile (<= 128 consecutive sorted tokens of one sequence): the union of the window
+// neighbourhoods of its tokens, as ascending padded rows. Candidates are the tokens of the blocks
+// in the 3x3x3 block neighbourhood of every block the tile touches (r <= 8 keeps every window
+// inside it); a candidate is kept if it lies within Chebyshev distance r of some tile token.
+// kFill == false writes counts, kFill == true writes the rows at wt_off.
+template <bool kFill>
+__global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t* __restrict__ qt_len,
+                               const int32_t* __restrict__ qt_seq, const int32_t* __restrict__ perm,
+                               const int32_t* __restrict__ tok_blk, const int32_t* __restrict__ coords,
+                               const int32_t* __restrict__ blk_coord, const int32_t* __restrict__ blk_poff,
+                               const int32_t* __restrict__ blk_off,
+                               const int32_t* __restrict__ key2blk, const SeqInfo* __restrict__ seqs,
+                               const int4* __restrict__ scoord, int r,
+                               int32_t* __restrict__ wt_cnt, const int32_t* __restrict__ wt_off,
+                               int32_t* __restrict__ wt_keys) {
+    constexpr int kCandCap = 4096;     // 27 neighbours x up to 128 distinct tile blocks, padded
+    __shared__ int4 qc[kQTile];
+    __shared__ int32_t cand[kCandCap];
+    __shared__ int32_t tile_blocks[kQTile];
+    __shared__ int32_t ncand_s, ntb_s;
+    const int t = blockIdx.x;
+    const int32_t p0 = qt_pos[t], len = qt_len[t];
+    const SeqInfo q = seqs[qt_seq[t]];
+    if (threadIdx.x == 0) { ncand_s = 0; ntb_s = 0; }
+    __syncthreads();
+    for (int a = threadIdx.x; a < len; a += blockDim.x) {
+        int32_t i = perm[p0 + a];
+        qc[a] = make_int4(coords[3 * i], coords[3 * i + 1], coords[3 * i + 2], 0);
+    }
+    // distinct blocks of the tile (the tile is a run of consecutive sorted tokens)
+    if (threadIdx.x == 0) {
+        int32_t prev = -1;
+        for (int a = 0; a < len; ++a) {
+            int32_t b = tok_blk[perm[p0 + a]];
+            if (b != prev) tile_blocks[ntb_s++] = b;
+            prev = b;
+        }
+    }
+    __syncthreads();
+    // candidate blocks: 27-neighbourhoods of the tile blocks
+    for (int e = threadIdx.x; e < ntb_s * 27; e += blockDim.x) {
+        int32_t tb = tile_blocks[e / 27];
+        int o = e % 27;
+        int bx = blk_coord[3 * tb] + o / 9 - 1, by = blk_coord[3 * tb + 1] + (o / 3) % 3 - 1,
+            bz = blk_coord[3 * tb + 2] + o % 3 - 1;
+        if (bx < 0 || by < 0 || bz < 0 || bx >= q.gbx || by >= q.gby || bz >= q.gbz) continue;
+        int32_t nb = key2blk[q.dense_base + ((int64_t)bx * q.gby + by) * q.gbz + bz];
+        if (nb < 0) continue;
+        cand[atomicAdd(&ncand_s, 1)] = nb;
+    }
+    __syncthreads();
+    // sort (bitonic over the CTA) and deduplicate the candidates
+    {
+        const int n = ncand_s;
+        int capn = 1;
+        while (capn < n) capn <<= 1;
+        for (int a = n + threadIdx.x; a < capn; a += blockDim.x) cand[a] = 0x7fffffff;
+        __syncthreads();
+        for (int k = 2; k <= capn; k <<= 1)
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                for (int i = threadIdx.x; i < capn; i += blockDim.x) {
+                    int ixj = i ^ j;
+                    if (ixj > i) {
+                        int32_t a = cand[i], b = cand[ixj];
+                        if ((a > b) == ((i & k) == 0)) { cand[i] = b; cand[ixj] = a; }
+                    }
+                }
+                __syncthreads();
+            }
+        if (threadIdx.x == 0) {
+            int m = 0;
+            for (int a = 0; a < n; ++a)
+                if (m == 0 || cand[m - 1] != cand[a]) cand[m++] = cand[a];
+            ncand_s = m;
+        }
+        __syncthreads();
+    }
+    const int ncand = ncand_s;
+    int32_t out_base = kFill ? wt_off[t] : 0;
+    int total = 0;
+    for (int cb = 0; cb < ncand; ++cb) {
+        int32_t b = cand[cb];
+        int32_t r0 = blk_poff[b], nrow = blk_off[b + 1] - blk_off[b];
+        for (int a0 = 0; a0 < nrow; a0 += blockDim.x) {
+            int a = a0 + threadIdx.x;
+            bool keep = false;
+            if (a < nrow) {
+                int4 kc = scoord[r0 + a];
+                for (int u = 0; u < len && !keep; ++u) {
+                    int4 c = qc[u];
+                    int d = max(abs(kc.x - c.x), max(abs(kc.y - c.y), abs(kc.z - c.z)));
+                    keep = d <= r;
+                }
+            }
+            // CTA-wide ordered compaction of `keep`
+            unsigned m = __ballot_sync(0xffffffffu, keep);
+            __shared__ int wcount[32];
+            const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+            if (lane == 0) wcount[wid] = __popc(m);
+            __syncthreads();
+            int before = 0, all = 0;
+            for (int u = 0; u < (int)(blockDim.x >> 5); ++u) {
+                if (u < wid) before += wcount[u];
+                all += wcount[u];
+            }
+            if (kFill && keep)
+                wt_keys[out_base + total + before + __popc(m & ((1u << lane) - 1))] = r0 + a;
+            total += all;
+            __syncthreads();
+        }
+    }
+    if (!kFill && threadIdx.x == 0) wt_cnt[t] = total;
+}
+
+}  // namespace
+
+#define SSA_ALLOC(ptr, type, count)                                                      \
+    do {                                                                                 \
+        ptr = (type*)plan_alloc(p, sizeof(type) * (size_t)std::max<int64_t>((count), 1)); \
+        if (!ptr) return SSA_ERR_ALLOC;                                                  \
+    } while (0)
+
+ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
+    const int64_t N = p->N;
+    const int B = p->B;
+    const int r = p->r;
+    // ---- constants ---------------------------------------------------------------------------
+    SSA_ALLOC(p->d_seqs, SeqInfo, B);
+    SSA_ALLOC(p->d_status, int32_t, 1);
+    SSA_ALLOC(p->coords, int32_t, 3 * N);
+    if (cudaMemcpyAsync(p->d_seqs, p->seqs.data(), sizeof(SeqInfo) * B, cudaMemcpyHostToDevice, st) ||
+        cudaMemcpyAsync(p->coords, coords, sizeof(int32_t) * 3 * N, cudaMemcpyDeviceToDevice, st) ||
+        cudaMemsetAsync(p->d_status, 0, sizeof(int32_t), st))
+        return SSA_ERR_CUDA;
+
+    const int64_t G = p->G;
+    const int64_t cap_mb = std::min<int64_t>(G, N);
+    uint64_t hsize = 1024;
+    while (hsize < (uint64_t)(2 * N)) hsize <<= 1;
+    int64_t tmp_len = scan_tmp_len(std::max<int64_t>(G, N) + 1);
+
+    int32_t *tok_key, *key_cnt, *bidx, *key2blk, *blk_cnt, *blk_pcnt, *nbr_cnt, *tmp, *blk_fill;
+    uint64_t* hkeys;
+    int32_t* hvals;
+    SSA_ALLOC(tok_key, int32_t, N);
+    SSA_ALLOC(key_cnt, int32_t, G);
+    SSA_ALLOC(bidx, int32_t, G + 1);
+    SSA_ALLOC(key2blk, int32_t, G);
+    SSA_ALLOC(blk_cnt, int32_t, cap_mb + 1);
+    SSA_ALLOC(blk_pcnt, int32_t, cap_mb + 1);
+    SSA_ALLOC(blk_fill, int32_t, cap_mb + 1);
+    SSA_ALLOC(nbr_cnt, int32_t, N + 1);
+    SSA_ALLOC(tmp, int32_t, tmp_len);
+    SSA_ALLOC(hkeys, uint64_t, hsize);
+    SSA_ALLOC(hvals, int32_t, hsize);
+    SSA_ALLOC(p->blk_off, int32_t, cap_mb + 1);
+    SSA_ALLOC(p->blk_poff, int32_t, cap_mb + 1);
+    SSA_ALLOC(p->blk_coord, int32_t, 3 * cap_mb);
+    SSA_ALLOC(p->blk_seq, int32_t, cap_mb);
+    SSA_ALLOC(p->nbr_off32, int32_t, N + 1);
+    if (cudaMemsetAsync(key_cnt, 0, sizeof(int32_t) * G, st) ||
+        cudaMemsetAsync(blk_cnt, 0, sizeof(int32_t) * (cap_mb + 1), st) ||
+        cudaMemsetAsync(blk_pcnt, 0, sizeof(int32_t) * (cap_mb + 1), st) ||
+        cudaMemsetAsync(blk_fill, 0, sizeof(int32_t) * (cap_mb + 1), st) ||
+        cudaMemsetAsync(hkeys, 0xff, sizeof(uint64_t) * hsize, st))
+        return SSA_ERR_CUDA;
+
+    // ---- a1: keys, histogram, hash -------------------------------------------------------------
+    k_keys_and_hash<<<grid_for(N), kThreads, 0, st>>>(coords, N, p->d_seqs, B, tok_key, key_cnt,
+                                                      hkeys, hvals, hsize - 1, p->d_status);
+    k_occupied<<<grid_for(G), kThreads, 0, st>>>(key_cnt, G, bidx);
+    note_launch(2);
+    scan_exclusive(bidx, bidx, G, tmp, st);
+    k_blocks<<<grid_for(G), kThreads, 0, st>>>(key_cnt, bidx, G, p->d_seqs, B, key2blk, blk_cnt,
+                                               blk_pcnt, p->blk_coord, p->blk_seq);
+    note_launch();
+    scan_exclusive(blk_cnt, p->blk_off, cap_mb, tmp, st);
+    scan_exclusive(blk_pcnt, p->blk_poff, cap_mb, tmp, st);
+
+    // ---- a2: neighbour counts --------------------------------------------------------------------
+    const int cube = (2 * r + 1) * (2 * r + 1) * (2 * r + 1);
+    int cap = 32;
+    while (cap < cube) cap <<= 1;
+    const int warps = std::max(1, std::min(8, 8192 / cap));
+    k_neighbours<false><<<grid_for(N, warps), warps * 32, 0, st>>>(
+        coords, N, p->d_seqs, B, r, hkeys, hvals, hsize - 1, nbr_cnt, nullptr, nullptr, cap,
+        p->d_status);
+    note_launch();
+    scan_exclusive(nbr_cnt, p->nbr_off32, N, tmp, st);
+
+    // ---- first wait: sizes and coordinate errors --------------------------------------------------
+    int32_t h_sizes[4];
+    if (cudaMemcpyAsync(&h_sizes[0], bidx + G, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaMemcpyAsync(&h_sizes[1], p->blk_poff + cap_mb, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaMemcpyAsync(&h_sizes[2], p->nbr_off32 + N, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaMemcpyAsync(&h_sizes[3], p->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    if (h_sizes[3] & DEV_COORD_RANGE) return SSA_ERR_COORD_RANGE;
+    if (h_sizes[3] & DEV_DUPLICATE) return SSA_ERR_DUPLICATE_COORD;
+    if (h_sizes[3]) return SSA_ERR_CUDA;
+    p->Mb = h_sizes[0];
+    p->Npad = h_sizes[1];
+    p->nnz = h_sizes[2];
+    if (p->nnz < 0) return SSA_ERR_UNSUPPORTED;  // more than 2^31 neighbour pairs
+
+    // ---- a1: scatter, per-block sort, positions ------------------------------------------------
+    SSA_ALLOC(p->perm, int32_t, N);
+    SSA_ALLOC(p->tok_blk, int32_t, N);
+    SSA_ALLOC(p->tok_pos, int32_t, N);
+    SSA_ALLOC(p->spos_tok, int32_t, p->Npad);
+    SSA_ALLOC(p->scoord, int4, p->Npad);
+    SSA_ALLOC(p->nbr_idx, int32_t, p->nnz);
+    k_scatter<<<grid_for(N), kThreads, 0, st>>>(tok_key, key2blk, N, p->blk_off, blk_fill, p->perm,
+                                                p->tok_blk);
+    k_sort_blocks<<<grid_for(p->Mb, 8), 256, 0, st>>>(p->perm, p->blk_off, p->Mb);
+    k_fill_i32<<<grid_for(p->Npad), kThreads, 0, st>>>(p->spos_tok, p->Npad, -1);
+    // padding rows sit far outside every grid so no window test ever accepts them
+    k_fill_int4<<<grid_for(p->Npad), kThreads, 0, st>>>(p->scoord, p->Npad,
+                                                        make_int4(1 << 28, 1 << 28, 1 << 28, -1));
+    k_positions<<<grid_for(N), kThreads, 0, st>>>(p->perm, p->tok_blk, p->blk_off, p->blk_poff,
+                                                  p->coords, N, p->tok_pos, p->spos_tok, p->scoord);
+    note_launch(5);
+
+    // ---- a2: neighbour lists -----------------------------------------------------------------------
+    k_neighbours<true><<<grid_for(N, warps), warps * 32, (size_t)warps * cap * sizeof(int32_t), st>>>(
+        coords, N, p->d_seqs, B, r, hkeys, hvals, hsize - 1, nullptr, p->nbr_off32, p->nbr_idx,
+        cap, p->d_status);
+    note_launch();
+
+    // ---- query tiles and their window key unions (tensor-core window kernel) ----------------------
+    std::vector<int32_t> qpos, qlen, qseq;
+    for (int s = 0; s < B; ++s) {
+        for (int64_t a = p->seqs[s].lo; a < p->seqs[s].hi; a += kQTile) {
+            qpos.push_back((int32_t)a);
+            qlen.push_back((int32_t)std::min<int64_t>(kQTile, p->seqs[s].hi - a));
+            qseq.push_back(s);
+        }
+    }
+    p->n_qtiles = (int64_t)qpos.size();
+    const int64_t T = p->n_qtiles;
+    SSA_ALLOC(p->qt_pos, int32_t, T);
+    SSA_ALLOC(p->qt_len, int32_t, T);
+    SSA_ALLOC(p->qt_seq, int32_t, T);
+    SSA_ALLOC(p->wt_off, int32_t, T + 1);
+    SSA_ALLOC(p->wt_keys, int32_t, p->nnz);
+    if (cudaMemcpyAsync(p->qt_pos, qpos.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st) ||
+        cudaMemcpyAsync(p->qt_len, qlen.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st) ||
+        cudaMemcpyAsync(p->qt_seq, qseq.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st))
+        return SSA_ERR_CUDA;
+    int32_t* wt_cnt;
+    SSA_ALLOC(wt_cnt, int32_t, T + 1);
+    k_window_union<false><<<(unsigned)T, 128, 0, st>>>(
+        p->qt_pos, p->qt_len, p->qt_seq, p->perm, p->tok_blk, p->coords, p->blk_coord, p->blk_poff,
+        p->blk_off, key2blk, p->d_seqs, p->scoord, r, wt_cnt, nullptr, nullptr);
+    note_launch();
+    scan_exclusive(wt_cnt, p->wt_off, T, tmp, st);
+    k_window_union<true><<<(unsigned)T, 128, 0, st>>>(
+        p->qt_pos, p->qt_len, p->qt_seq, p->perm, p->tok_blk, p->coords, p->blk_coord, p->blk_poff,
+        p->blk_off, key2blk, p->d_seqs, p->scoord, r, nullptr, p->wt_off, p->wt_keys);
+    note_launch();
+
+    // block range of every sequence (host copy for launches)
+    p->seq_blk.assign(B + 1, 0);
+    std::vector<int32_t> sb(B + 1);
+    for (int s = 0; s <= B; ++s) {
+        int64_t key = s < B ? p->seqs[s].dense_base : G;
+        if (cudaMemcpyAsync(&sb[s], bidx + key, sizeof(int32_t), cudaMemcpyDeviceToHost, st))
+            return SSA_ERR_CUDA;
+    }
+    int32_t status = 0;
+    if (cudaMemcpyAsync(&status, p->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    for (int s = 0; s <= B; ++s) p->seq_blk[s] = sb[s];
+    SSA_ALLOC(p->seq_blk_d, int32_t, B + 1);
+    if (cudaMemcpyAsync(p->seq_blk_d, sb.data(), sizeof(int32_t) * (B + 1), cudaMemcpyHostToDevice, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    if (status) return SSA_ERR_CUDA;
+
+    // scratch of the plan build is released now
+    void* scratch[] = {tok_key, key_cnt, bidx, key2blk, blk_cnt, blk_pcnt, blk_fill,
+                       nbr_cnt, tmp, hkeys, hvals, wt_cnt};
+    for (void* ptr : scratch) {
+        auto it = std::find(p->owned.begin(), p->owned.end(), ptr);
+        if (it != p->owned.end()) {
+            p->release(ptr, st, p->alloc_ctx);
+            p->owned.erase(it);
+        }
+    }
+    return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+}  // namespace ssa

@@ -1,0 +1,182 @@
+"""Forward parity (rows a3-a8) of the CUDA path against the fp64 oracle, through the C ABI.
+
+Small configurations are compared on every output element; the full-size configurations
+(80k, 110k and the 340k-token varlen batch, H=22, D=96, fp16) on 512 seeded rows per sequence,
+in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from ssa_testlib import (blk_base_of_rows, check_close, coords_of, make_plan, selection_agreement,
+                         tensors_of, to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_forward(plan, t, topk):
+    g = to_gpu(t)
+    out, sel = plan.forward(g["Q"], g["K"], g["V"], g["gates"], g["Wc"], topk, return_sel=True)
+    torch.cuda.synchronize()
+    assert plan.status() == 0
+    return out.double().cpu().numpy(), sel.cpu().numpy()
+
+
+def compare(name_or_cfg, coords, cu, grids, t, topk, r, dtype, rows=None, max_mismatch=0.01):
+    plan = make_plan(coords, cu, grids, r)
+    out, sel = gpu_forward(plan, t, topk)
+    ref = oracle.forward(coords, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], topk, r,
+                         rows=rows, want_z=True)
+    rows = ref["rows"]
+    bs = plan.export()["blk_seq"].cpu().numpy()
+    mism, rep = selection_agreement(sel[rows], ref["sel"], ref["z"], blk_base_of_rows(cu, rows, bs),
+                                    dtype)
+    assert rep["mismatched"] <= max_mismatch * rep["rows"], rep
+    keep = ~mism
+    check_close(out[rows][keep], ref["out"][keep], dtype, f"{name_or_cfg} out")
+    return plan, out, sel, ref, rep
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_forward_full_output(name):
+    cfg = workloads.CONFIGS[name]
+    c, cu, g = coords_of(name)
+    compare(name, c, cu, g, tensors_of(name), cfg.topk, cfg.radius, cfg.dtype)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["pass1", "pass3", "varlen"])
+def test_forward_full_size_sampled_rows(name):
+    cfg = workloads.CONFIGS[name]
+    c, cu, g = coords_of(name)
+    rows = np.concatenate(workloads.stratified_rows(cu, 512, seed=cfg.index * 1000 + 99))
+    compare(name, c, cu, g, tensors_of(name), cfg.topk, cfg.radius, cfg.dtype, rows=rows)
+
+
+def _branch_inputs(name, dtype):
+    cfg = workloads.CONFIGS[name]
+    c, cu, g = coords_of(name)
+    t = dict(tensors_of(name))
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[dtype]
+    for key in ("Q", "K", "V"):
+        t[key] = t[key].float().to(tdt)
+    return cfg, c, cu, g, t
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("branch", [0, 1, 2])
+def test_each_branch_alone(dtype, branch):
+    """One-hot gates isolate the compressed, selected and window branches."""
+    cfg, c, cu, g, t = _branch_inputs("small", dtype)
+    gates = torch.zeros_like(t["gates"])
+    gates[:, :, branch] = 1.0
+    t["gates"] = gates
+    compare(f"branch{branch}", c, cu, g, t, cfg.topk, cfg.radius, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_planted_topk_is_exact(dtype):
+    """Queries e = 1, keys of block b = alpha_b * 1, Wc = I: the ranking is known exactly."""
+    c, cu, g = coords_of("tiny")
+    N, H, D, topk = len(c), 2, 32, 6
+    perm, tok_blk, blk_off, blk_coord = oracle.partition(c)
+    mb = len(blk_coord)
+    rng = np.random.default_rng(7)
+    alpha = (np.stack([rng.permutation(mb) for _ in range(H)], 1) - mb / 2) / 8.0
+    alpha[7, 0] = alpha[3, 0]   # tie: the lower block index wins
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[dtype]
+    t = dict(Q=torch.ones(N, H, D).to(tdt),
+             K=torch.from_numpy(np.repeat(alpha[tok_blk][:, :, None], D, 2)).float().to(tdt),
+             V=torch.randn(N, H, D, generator=torch.Generator().manual_seed(3)).to(tdt),
+             gates=torch.rand(N, H, 3, generator=torch.Generator().manual_seed(4)),
+             Wc=torch.eye(D))
+    plan = make_plan(c, cu, g, 2)
+    out, sel = gpu_forward(plan, t, topk)
+    exp = np.full((N, H, topk), -1)
+    for i in range(N):
+        for h in range(H):
+            others = sorted((b for b in range(mb) if b != tok_blk[i]), key=lambda b: (-alpha[b, h], b))
+            exp[i, h] = [tok_blk[i]] + others[:topk - 1]
+    assert np.array_equal(sel, exp)
+    ref = oracle.forward(c, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], topk, 2)
+    check_close(out, ref["out"], dtype, "planted")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+def test_fewer_blocks_than_k_and_dense_limit(dtype):
+    """k >= Mb selects every block: with selection-only gates the output is dense attention."""
+    c_all, _, g = coords_of("tiny")
+    c = c_all[:300]                      # the first 300 voxels in (x, y, z) order: a few blocks
+    cu = np.array([0, len(c)])
+    mb = len(oracle.partition(c)[3])
+    assert mb + 2 <= 32
+    cfg = workloads.WorkloadConfig("dense", 7, (), H=2, D=32, dtype=dtype, topk=mb + 2, radius=2)
+    t = workloads.make_tensors(cfg, len(c))
+    gates = torch.zeros_like(t["gates"])
+    gates[:, :, 1] = 1.0
+    t["gates"] = gates
+    plan, out, sel, ref, rep = compare("dense", c, cu, g, t, mb + 2, 2, dtype)
+    assert np.all(sel[:, :, mb:] == -1)
+    # textbook dense attention over all tokens (library routine, fp64)
+    q, k, v = (x.double().permute(1, 0, 2) for x in (t["Q"], t["K"], t["V"]))
+    dense = torch.nn.functional.scaled_dot_product_attention(q, k, v).permute(1, 0, 2).numpy()
+    check_close(out, dense, dtype, "dense limit")
+
+
+@pytest.mark.parametrize("r", [0, 1, 3, 8])
+def test_window_radii(r):
+    cfg, c, cu, g, t = _branch_inputs("small", "f16")
+    compare(f"r={r}", c, cu, g, t, cfg.topk, r, "f16")
+
+
+def test_ragged_tiles_single_token_and_varlen_edge_cases():
+    a, _, _ = coords_of("tiny")
+    b = np.array([[5, 6, 7]], np.int32)
+    c = np.concatenate([a[:700], b, a[700:1333]])
+    cu = np.array([0, 700, 700, 701, len(c)])
+    grids = np.array([[32, 32, 32], [16, 16, 16], [9, 9, 9], [32, 32, 32]], np.int32)
+    cfg = workloads.WorkloadConfig("edge", 9, (), H=3, D=64, dtype="f16", topk=5, radius=2)
+    t = workloads.make_tensors(cfg, len(c))
+    compare("edge", c, cu, grids, t, 5, 2, "f16")
+
+
+def test_head_dims_and_k_values():
+    c, cu, g = coords_of("tiny")
+    for D, topk in ((32, 1), (64, 9), (128, 17), (96, 32)):
+        cfg = workloads.WorkloadConfig("hd", 8, (), H=2, D=D, dtype="bf16", topk=topk, radius=2)
+        t = workloads.make_tensors(cfg, len(c))
+        compare(f"D={D},k={topk}", c, cu, g, t, topk, 2, "bf16")
+
+
+def test_repeat_calls_are_bitwise_identical_and_host_entry_matches():
+    cfg = workloads.CONFIGS["small"]
+    c, cu, g = coords_of("small")
+    t = tensors_of("small")
+    plan = make_plan(c, cu, g, cfg.radius)
+    dev = to_gpu(t)
+    a = plan.forward(dev["Q"], dev["K"], dev["V"], dev["gates"], dev["Wc"], cfg.topk)
+    b = plan.forward(dev["Q"], dev["K"], dev["V"], dev["gates"], dev["Wc"], cfg.topk)
+    host = {k: v.pin_memory() for k, v in t.items()}
+    out_h = torch.empty_like(host["Q"]).pin_memory()
+    plan.forward_host(host["Q"], host["K"], host["V"], host["gates"], host["Wc"], cfg.topk, out_h)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert torch.equal(a.cpu(), out_h)
+
+
+def test_forward_argument_errors():
+    import spatial_sparse_attention_b200 as ssa
+    c, cu, g = coords_of("tiny")
+    plan = make_plan(c, cu, g, 2)
+    N = len(c)
+    q = torch.zeros(N, 2, 48, dtype=torch.float16, device="cuda")
+    gates = torch.zeros(N, 2, 3, device="cuda")
+    with pytest.raises(ssa.SSAError) as e:
+        plan.forward(q, q, q, gates, torch.eye(48, device="cuda"), 4)
+    assert e.value.name == "SSA_ERR_UNSUPPORTED"
+    q = torch.zeros(N, 2, 32, dtype=torch.float16, device="cuda")
+    with pytest.raises(ssa.SSAError) as e:
+        plan.forward(q, q, q, gates, torch.eye(32, device="cuda"), 33)
+    assert e.value.name == "SSA_ERR_UNSUPPORTED"

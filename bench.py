@@ -1,0 +1,364 @@
+"""Benchmark: Spatial Sparse Attention forward on B200 through the C ABI of libssa.so.
+
+One step = the whole hot path on one batch: the plan (block partition, coordinate hash, window
+lists) and the forward (pooling, compressed attention + top-k, window, own block, selected blocks,
+gated combine). Workload: the refinement-pass-3-shaped configuration (110,000 voxel tokens on the
+thickness-3 shell of 5 random ellipsoids/boxes in a 192^3 grid; 22 heads x 96 dims, fp16; top-16
+blocks of 8^3; window radius 3), seeded synthetic inputs resident in HBM.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--config NAME]
+
+Multi-GPU (torchrun): every rank runs its own independent batch (the method shards by sequence or
+head with no exchange), so scaling is weak; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "SSA forward tokens/s and TFLOP/s (% fp16 TC peak) at N=110k, H=22, D=96"
+DEFAULT_CONFIG = "pass3"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def describe(cfg, coords, cu):
+    return {
+        "workload": f"{cfg.name}: {cfg.description}; H={cfg.H}, D={cfg.D}, {cfg.dtype}, "
+                    f"top-{cfg.topk} of 8^3 blocks, window r={cfg.radius}",
+        "tokens": int(len(coords)), "sequences": int(len(cu) - 1), "heads": cfg.H,
+        "head_dim": cfg.D, "topk": cfg.topk, "radius": cfg.radius, "block": 8,
+        "l2": "inputs larger than L2 (Q, K, V are N*H*D*2 bytes each); no flush between steps",
+    }
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def algorithmic_flops(plan, sel, cfg, cu):
+    """Sum over (token, head) of 4*D*(Mb of its sequence + tokens of its selected blocks + window),
+    and the part executed by each kernel (k_qmajor: compressed + window + own block; k_kbmajor:
+    the other selected blocks)."""
+    import torch
+    ex = plan.export()
+    nb = (ex["blk_off"][1:] - ex["blk_off"][:-1]).long()
+    blk_seq = ex["blk_seq"].long()
+    mb_seq = torch.bincount(blk_seq, minlength=len(cu) - 1)
+    seqlens = torch.from_numpy(np.diff(cu)).to(mb_seq.device)
+    cmp_pairs = int((mb_seq * seqlens).sum()) * cfg.H
+    s = sel.long()
+    sizes = torch.where(s >= 0, nb[s.clamp(min=0)], torch.zeros_like(s))
+    own = int(sizes[:, :, 0].sum())
+    other = int(sizes[:, :, 1:].sum())
+    win = int(plan.nnz) * cfg.H
+    f = 4 * cfg.D
+    return {"total": f * (cmp_pairs + own + other + win), "k_qmajor": f * (cmp_pairs + own + win),
+            "k_kbmajor": f * other, "pairs": {"compressed": cmp_pairs, "own": own,
+                                             "selected_other": other, "window": win}}
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    import spatial_sparse_attention_b200 as ssa
+
+    cfg = workloads.CONFIGS[args.config]
+    coords, cu, grids = workloads.make_coords(cfg)
+    t = workloads.make_tensors(cfg, len(coords))
+    dev = {k: v.cuda() for k, v in t.items()}
+    coords_d = torch.from_numpy(coords).cuda()
+    N = len(coords)
+
+    def make_plan():
+        if len(cu) == 2:
+            return ssa.Plan(coords_d, grid=tuple(int(x) for x in grids[0]), r=cfg.radius)
+        return ssa.Plan(coords_d, r=cfg.radius, cu_seqlens=[int(x) for x in cu],
+                        grids=[tuple(int(x) for x in g) for g in grids])
+
+    out = torch.empty_like(dev["Q"])
+    plan = make_plan()
+
+    def step():
+        # the whole path: plan (a1, a2) rebuilt from the coordinates, then the forward (a3-a8)
+        plan.rebuild(coords_d)
+        plan.forward(dev["Q"], dev["K"], dev["V"], dev["gates"], dev["Wc"], cfg.topk, out=out)
+
+    # algorithmic work (outside the timed region)
+    _, sel = plan.forward(dev["Q"], dev["K"], dev["V"], dev["gates"], dev["Wc"], cfg.topk,
+                          return_sel=True)
+    torch.cuda.synchronize()
+    if plan.status() != 0:
+        raise RuntimeError("device status set after the first forward")
+    work = algorithmic_flops(plan, sel, cfg, cu)
+    del sel
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    clocks = Clocks(torch.cuda.current_device())
+    if rank == 0:
+        clocks.start()
+    ssa.profile_reset()
+    ssa.profile_enable(True)
+    launches0 = ssa.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    launches = ssa.launch_count() - launches0
+    ssa.profile_enable(False)
+    prof = ssa.profile_read()
+    if plan.status() != 0:
+        raise RuntimeError("device status set during the timed steps")
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    clk = clocks.stop() if rank == 0 else None
+
+    # end to end through the host-buffer entry point (pinned host memory, copies inside)
+    host = {k: v.pin_memory() for k, v in t.items()}
+    coords_h = torch.from_numpy(coords).pin_memory()
+    out_h = torch.empty_like(host["Q"]).pin_memory()
+    e2e_ms = []
+    cd = torch.empty_like(coords_d)
+    for it in range(args.e2e_steps + 1):
+        torch.cuda.synchronize()
+        a = time.perf_counter()
+        cd.copy_(coords_h, non_blocking=True)
+        plan.rebuild(cd)
+        plan.forward_host(host["Q"], host["K"], host["V"], host["gates"], host["Wc"], cfg.topk,
+                          out_h)
+        b = time.perf_counter()
+        if it > 0:
+            e2e_ms.append((b - a) * 1e3)
+    e2e = statistics.median(e2e_ms)
+    h2d = coords.nbytes + sum(host[k].numel() * host[k].element_size() for k in ("Q", "K", "V", "gates", "Wc"))
+    d2h = out_h.numel() * out_h.element_size()
+
+    pk, src = peaks()
+    dominant = max((k for k in prof if k in ("k_qmajor", "k_kbmajor")), key=lambda k: prof[k][0])
+    dom_ms = prof[dominant][0] / max(prof[dominant][1], 1)
+    achieved = work[dominant] / (dom_ms * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))  # fp16 dense rate = bf16 rate
+    tflops = work["total"] / (ms * 1e-3) / 1e12
+    fwd_ms = sum(prof[k][0] for k in prof if k != "plan") / args.steps
+    res = {
+        "metric": METRIC, "value": N * world / (ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded voxel shells, N(0,1) Q/K/V)",
+        "config": describe(cfg, coords, cu),
+        "tflops": {"value": tflops, "unit": "TFLOP/s (algorithmic attention FLOPs per step / step time)",
+                   "pct_of_peak": 100.0 * tflops / peak, "peak": peak,
+                   "peak_source": f"{src} bf16_tflops_sustained (fp16 dense rate = bf16 rate)",
+                   "algorithmic_tflop_per_step": work["total"] / 1e12, "pairs": work["pairs"]},
+        "breakdown_ms_per_step": {k: v[0] / args.steps for k, v in prof.items()},
+        "forward_only": {"ms": fwd_ms, "tokens_per_s": N / (fwd_ms * 1e-3),
+                         "tflops": work["total"] / (fwd_ms * 1e-3) / 1e12},
+        "roofline": {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_tflop_per_launch": work[dominant] / 1e12,
+                     "avg_launch_ms": dom_ms, "peak_source": src},
+        "e2e": {"value": N / (e2e * 1e-3), "unit": "tokens/s", "ms_per_step": e2e,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "api": "coordinates copied from pinned host memory, ssa_plan_rebuild, "
+                       "ssa_forward_host (pinned host Q/K/V/gates/Wc in, out back to host)"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    return res
+
+
+def cpu_baseline(cfg_name, target_s=15.0):
+    """The oracle (plain C, fp64, OpenMP) on the host: the full plan of the workload plus the
+    forward of a seeded sample of query rows, extrapolated to all tokens."""
+    import oracle
+    cfg = workloads.CONFIGS[cfg_name]
+    coords, cu, grids = workloads.make_coords(cfg)
+    t = workloads.make_tensors(cfg, len(coords))
+    N = len(coords)
+    a = time.perf_counter()
+    oracle.plan(coords, cu, 8, cfg.radius)
+    t_plan = time.perf_counter() - a
+    rows = np.concatenate(workloads.stratified_rows(cu, 16, seed=4242))
+    a = time.perf_counter()
+    oracle.forward(coords, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], cfg.topk, cfg.radius,
+                   rows=rows)
+    t_probe = time.perf_counter() - a
+    per_row = t_probe / len(rows)
+    n_rows = int(min(N, max(len(rows), (target_s - t_plan) / max(per_row, 1e-9))))
+    rows = np.sort(np.random.default_rng(4243).choice(N, n_rows, replace=False))
+    a = time.perf_counter()
+    oracle.forward(coords, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], cfg.topk, cfg.radius,
+                   rows=rows)
+    t_rows = time.perf_counter() - a
+    step_s = t_plan + t_rows * N / n_rows
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": N / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"full plan ({t_plan:.2f} s) + forward of {n_rows} seeded query rows x "
+                      f"{cfg.H} heads ({t_rows:.2f} s), extrapolated to {N} rows"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    cfg = workloads.CONFIGS[args.config]
+    coords, cu, grids = workloads.make_coords(cfg)
+    t = workloads.make_tensors(cfg, len(coords))
+    N = len(coords)
+    rows = np.concatenate(workloads.stratified_rows(cu, 8, seed=777))
+    oracle.lib()
+
+    def step():
+        oracle.plan(coords, cu, 8, cfg.radius)
+        oracle.forward(coords, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], cfg.topk,
+                       cfg.radius, rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    a = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    per_step = (time.perf_counter() - a) / args.steps
+    # time of one full step: plan + forward of all rows, extrapolated from the sampled rows
+    a = time.perf_counter()
+    oracle.plan(coords, cu, 8, cfg.radius)
+    t_plan = time.perf_counter() - a
+    t_rows = max(per_step - t_plan, 1e-9)
+    full = t_plan + t_rows * N / len(rows)
+    value = N / full
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": full * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": describe(cfg, coords, cu), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: full plan + forward of {len(rows)} seeded rows x "
+                                   f"{cfg.H} heads; extrapolated to {N} rows"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as td
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = td
+    res = run_ours(args, rank, world, dist)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args.config)
+        print(json.dumps(res), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -105,6 +105,15 @@ SSA_API ssa_status_t ssa_plan_varlen(const int32_t* coords, const int64_t* cu_se
                              const int32_t* grids, int32_t block, int32_t r, void* stream,
                              ssa_plan_t* out);
 
+/*
+ * Recompute a plan in place for new coordinates with the same token count, sequence layout,
+ * grids and radius (e.g. the next refinement pass over a re-voxelised support of equal size).
+ * coords: device int32 [N, 3]. The forward workspace is kept when the block count and padded row
+ * count are unchanged, so a following ssa_forward allocates nothing. Waits for the device like
+ * ssa_plan. On error the plan is left empty (only ssa_plan_destroy is valid).
+ */
+SSA_API ssa_status_t ssa_plan_rebuild(ssa_plan_t plan, const int32_t* coords, void* stream);
+
 /* Sizes of a plan (host outputs; any may be NULL): tokens, occupied blocks, total neighbour
  * list length, number of sequences. */
 SSA_API ssa_status_t ssa_plan_info(ssa_plan_t plan, int64_t* n, int64_t* num_blocks, int64_t* nnz,
@@ -180,6 +189,19 @@ SSA_API const char* ssa_status_string(ssa_status_t status);
 
 /* Number of kernels this library has launched in the process so far. */
 SSA_API int64_t ssa_launch_count(void);
+
+/*
+ * Kernel timing (measurement support, not part of the method). When enabled, each hot step
+ * (plan, pool, k_qmajor, selection_inversion, k_kbmajor, k_combine) is bracketed by two CUDA
+ * events recorded on the stream it is launched on. ssa_profile_read waits for the recorded
+ * events, adds their durations to per-name totals and copies up to max_entries totals out:
+ * names (host char[max_entries][64], NUL-terminated), total_ms and launches (host arrays; any
+ * may be NULL). Returns the number of entries. ssa_profile_reset clears the totals.
+ */
+SSA_API ssa_status_t ssa_profile_enable(int32_t on);
+SSA_API ssa_status_t ssa_profile_reset(void);
+SSA_API int32_t ssa_profile_read(int32_t max_entries, char* names, double* total_ms,
+                                 int64_t* launches);
 
 #ifdef __cplusplus
 }

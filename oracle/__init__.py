@@ -324,8 +324,10 @@ def backward(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, bloc
 
 
 def backward_dq_rows(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, rows,
-                     block: int = 8, round_compressed: bool = True):
-    """dQ [R, H, D] for the given global rows, evaluated row by row (any size)."""
+                     block: int = 8, round_compressed: bool = True, return_sel: bool = False):
+    """dQ [R, H, D] for the given global rows, evaluated row by row (any size).
+
+    With return_sel, also returns the selection used ([R, H, k] global block indices)."""
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     q, dt = _raw(Q)
@@ -337,26 +339,32 @@ def backward_dq_rows(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: i
     N, H, D = q.shape
     rows = np.asarray(rows, dtype=np.int64)
     dQ = np.zeros((len(rows), H, D))
+    sel_all = np.full((len(rows), H, topk), -1, np.int32)
     seq_of = np.searchsorted(cu, rows, side="right") - 1
     L = lib()
+    blk_base = 0
     for s in range(len(cu) - 1):
         pick = np.nonzero(seq_of == s)[0]
-        if not len(pick):
-            continue
         lo, hi = int(cu[s]), int(cu[s + 1])
         perm, tok_blk, blk_off, mb, no, ni = _seq_plan(coords, lo, hi, block, r)
+        if not len(pick):
+            blk_base += mb
+            continue
         local = np.ascontiguousarray(rows[pick] - lo)
         out = np.zeros((len(local), H, D))
+        sel = np.zeros((len(local), H, topk), np.int32)
         rc = L.oracle_backward_dq_rows(
             hi - lo, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data, v[lo:hi].ctypes.data,
             _ptr(np.ascontiguousarray(g[lo:hi]), c_f32p), _ptr(w, c_f32p), go[lo:hi].ctypes.data,
             topk, int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
             _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p), len(local),
-            _ptr(local, c_i64p), _ptr(out, c_f64p), None)
+            _ptr(local, c_i64p), _ptr(out, c_f64p), _ptr(sel, c_i32p))
         if rc != 0:
             raise RuntimeError("oracle_backward_dq_rows failed")
         dQ[pick] = out
-    return dQ
+        sel_all[pick] = np.where(sel >= 0, sel + blk_base, -1)
+        blk_base += mb
+    return (dQ, sel_all) if return_sel else dQ
 
 
 def compress(coords, K, V, Wc, block: int = 8, round_compressed: bool = False):

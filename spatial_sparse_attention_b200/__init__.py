@@ -40,6 +40,7 @@ _SIGS = {
     "ssa_set_allocator": [_vp, _vp, _vp],
     "ssa_plan": [_vp, _i64, _vp, _i32, _i32, _vp, _vp],
     "ssa_plan_varlen": [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp],
+    "ssa_plan_rebuild": [_vp, _vp, _vp],
     "ssa_plan_info": [_vp, _vp, _vp, _vp, _vp],
     "ssa_plan_export": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "ssa_forward": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp],
@@ -50,6 +51,9 @@ _SIGS = {
     "ssa_plan_destroy": [_vp],
     "ssa_status_string": [_i32],
     "ssa_launch_count": [],
+    "ssa_profile_enable": [_i32],
+    "ssa_profile_reset": [],
+    "ssa_profile_read": [_i32, _vp, _vp, _vp],
 }
 
 
@@ -77,6 +81,25 @@ def declared_symbols() -> Sequence[str]:
 
 def launch_count() -> int:
     return int(lib.ssa_launch_count())
+
+
+def profile_enable(on: bool = True):
+    lib.ssa_profile_enable(1 if on else 0)
+
+
+def profile_reset():
+    lib.ssa_profile_reset()
+
+
+def profile_read():
+    """{kernel name: (total ms, launches)} of the CUDA-event timings recorded so far."""
+    n = 32
+    names = ctypes.create_string_buffer(64 * n)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    k = lib.ssa_profile_read(n, names, ms, cnt)
+    return {names.raw[64 * i:64 * (i + 1)].split(b"\0")[0].decode(): (ms[i], cnt[i])
+            for i in range(k)}
 
 
 def _check(code: int, where: str):
@@ -128,6 +151,17 @@ class Plan:
                                  ctypes.byref(b)), "ssa_plan_info")
         self.N, self.num_blocks, self.nnz, self.batch = n.value, mb.value, nnz.value, b.value
         self.r = r
+
+    def rebuild(self, coords: torch.Tensor):
+        """Recompute the plan in place for new coordinates (same count, layout, grids, r)."""
+        _dev(coords, torch.int32)
+        _check(lib.ssa_plan_rebuild(self._h, coords.data_ptr(), _stream(self.stream)),
+               "ssa_plan_rebuild")
+        n, mb, nnz, b = _i64(), _i64(), _i64(), _i32()
+        _check(lib.ssa_plan_info(self._h, ctypes.byref(n), ctypes.byref(mb), ctypes.byref(nnz),
+                                 ctypes.byref(b)), "ssa_plan_info")
+        self.N, self.num_blocks, self.nnz, self.batch = n.value, mb.value, nnz.value, b.value
+        return self
 
     def close(self):
         if self._h:

@@ -1,16 +1,92 @@
 // C ABI of libssa.so (declared in include/ssa.h): argument validation, the plan object and its
 // device buffers, the cached forward workspace, and dispatch to the kernels.
 #include <algorithm>
+#include <chrono>
+#include <cstdio>
+#include <cstdlib>
 #include <cmath>
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <string>
 
 #include "common.cuh"
 
 namespace ssa {
 
 std::atomic<int64_t> g_launches{0};
+
+void trace_step(const char* what, cudaStream_t st) {
+    static const bool on = [] {
+        const char* e = getenv("SSA_TRACE");
+        return e && e[0] == '1';
+    }();
+    if (!on) return;
+    fprintf(stderr, "[ssa] %s: queued\n", what);
+    fflush(stderr);
+    auto t0 = std::chrono::steady_clock::now();
+    cudaError_t e = cudaStreamSynchronize(st);
+    double ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
+    fprintf(stderr, "[ssa] %s: done %.3f ms (%s)\n", what, ms, cudaGetErrorString(e));
+    fflush(stderr);
+}
+
+namespace {
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+struct ProfRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+std::vector<ProfRec> g_prof_pending;
+std::vector<cudaEvent_t> g_prof_free;
+struct ProfSum {
+    std::string name;
+    double ms = 0.0;
+    int64_t launches = 0;
+};
+std::vector<ProfSum> g_prof_sums;
+
+void prof_drain_locked() {
+    for (auto& r : g_prof_pending) {
+        float ms = 0.0f;
+        cudaEventSynchronize(r.b);
+        cudaEventElapsedTime(&ms, r.a, r.b);
+        ProfSum* slot = nullptr;
+        for (auto& x : g_prof_sums)
+            if (x.name == r.name) slot = &x;
+        if (!slot) {
+            g_prof_sums.push_back(ProfSum{r.name, 0.0, 0});
+            slot = &g_prof_sums.back();
+        }
+        slot->ms += ms;
+        slot->launches += 1;
+        g_prof_free.push_back(r.a);
+        g_prof_free.push_back(r.b);
+    }
+    g_prof_pending.clear();
+}
+}  // namespace
+
+bool profiling_on() { return g_prof_on; }
+
+cudaEvent_t profile_event() {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (!g_prof_free.empty()) {
+        cudaEvent_t e = g_prof_free.back();
+        g_prof_free.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+void profile_record(const char* name, cudaEvent_t start, cudaEvent_t stop) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_pending.push_back(ProfRec{name, start, stop});
+    if (g_prof_pending.size() > 4096) prof_drain_locked();
+}
 
 namespace {
 
@@ -115,7 +191,10 @@ ssa_status_t make_plan(const int32_t* coords, const int64_t* cu, int32_t B, cons
         delete p;
         return SSA_ERR_UNSUPPORTED;
     }
-    st = build_plan(p, coords, (cudaStream_t)stream);
+    {
+        ProfScope ps("plan", (cudaStream_t)stream);
+        st = build_plan(p, coords, (cudaStream_t)stream);
+    }
     if (st != SSA_OK) {
         cudaStreamSynchronize((cudaStream_t)stream);
         cudaGetLastError();
@@ -149,7 +228,8 @@ ssa_status_t ensure_workspace(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int
         w.ks = A(es * H * p->Npad * D);
         w.vs = A(es * H * p->Npad * D);
         w.base = (float*)A(sizeof(float) * N * H * D);
-        w.part_o = A(es * N * H * k * D);
+        // partials: fp16 for fp16 inputs, fp32 for bf16 inputs
+        w.part_o = A((dt == SSA_BF16 ? 4 : 2) * N * H * k * D);
         w.part_lse = (float*)A(sizeof(float) * N * H * k);
         w.inv_cnt = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
         w.inv_off = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
@@ -194,9 +274,14 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
     ssa_status_t rc = ensure_workspace(p, H, D, dt, topk, st);
     if (rc != SSA_OK) return rc;
     const Workspace& w = p->ws;
-    launch_pool(p, w, k, v, wc, st);
+    {
+        ProfScope ps("pool", st);
+        launch_pool(p, w, k, v, wc, st);
+    }
+    trace_step("pool", st);
     if (dt == SSA_F32) launch_forward_simt(p, w, q, k, v, gates, out, st);
     else launch_forward_tc(p, w, q, gates, out, st);
+    trace_step("forward", st);
     if (sel_out) launch_export_sel(p, w, sel_out, st);
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
@@ -240,6 +325,32 @@ ssa_status_t ssa_plan_varlen(const int32_t* coords, const int64_t* cu_seqlens, i
                              const int32_t* grids, int32_t block, int32_t r, void* stream,
                              ssa_plan_t* out) {
     return make_plan(coords, cu_seqlens, batch, grids, block, r, stream, out);
+}
+
+ssa_status_t ssa_plan_rebuild(ssa_plan_t p, const int32_t* coords, void* stream) {
+    if (!p || !coords) return SSA_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t old_mb = p->Mb, old_npad = p->Npad;
+    plan_free_all(p, p->owned);
+    p->stream = st;
+    ssa_status_t rc;
+    {
+        ProfScope ps("plan", st);
+        rc = build_plan(p, coords, st);
+    }
+    if (rc != SSA_OK) {
+        cudaStreamSynchronize(st);
+        cudaGetLastError();
+        plan_free_all(p, p->owned);
+        plan_free_all(p, p->ws.owned);
+        p->ws = Workspace();
+        return rc;
+    }
+    if (p->Mb != old_mb || p->Npad != old_npad) {
+        plan_free_all(p, p->ws.owned);
+        p->ws = Workspace();
+    }
+    return SSA_OK;
 }
 
 ssa_status_t ssa_plan_info(ssa_plan_t plan, int64_t* n, int64_t* num_blocks, int64_t* nnz,
@@ -389,5 +500,35 @@ const char* ssa_status_string(ssa_status_t s) {
 }
 
 int64_t ssa_launch_count(void) { return g_launches.load(); }
+
+ssa_status_t ssa_profile_enable(int32_t on) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = on != 0;
+    return SSA_OK;
+}
+
+ssa_status_t ssa_profile_reset(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    prof_drain_locked();
+    g_prof_sums.clear();
+    return SSA_OK;
+}
+
+int32_t ssa_profile_read(int32_t max_entries, char* names, double* total_ms, int64_t* launches) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    prof_drain_locked();
+    int32_t n = 0;
+    for (auto& x : g_prof_sums) {
+        if (n >= max_entries) break;
+        if (names) {
+            std::strncpy(names + 64 * n, x.name.c_str(), 63);
+            names[64 * n + 63] = 0;
+        }
+        if (total_ms) total_ms[n] = x.ms;
+        if (launches) launches[n] = x.launches;
+        ++n;
+    }
+    return n;
+}
 
 }  // extern "C"

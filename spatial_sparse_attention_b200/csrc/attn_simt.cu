@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kWarps * 32) k_forward_simt(const SimtParams P
             int32_t cb = b;
 #pragma unroll
             for (int t = 0; t < KM; ++t) {
-                const bool better = cz > tv[t];
+                const bool better = cz > tv[t] || (cz == tv[t] && (unsigned)cb < (unsigned)ti[t]);
                 const float ov = tv[t];
                 const int32_t oi = ti[t];
                 tv[t] = better ? cz : ov;

@@ -90,6 +90,17 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     }
 }
 
+template <typename T>
+__device__ __forceinline__ float unpack_lo(uint32_t v) {
+    if constexpr (std::is_same<T, __half>::value) return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu)));
+    else return __uint_as_float(v << 16);
+}
+template <typename T>
+__device__ __forceinline__ float unpack_hi(uint32_t v) {
+    if constexpr (std::is_same<T, __half>::value) return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
+    else return __uint_as_float(v & 0xffff0000u);
+}
+
 struct Ctx {
     uint8_t* g;      // generic pointer to the 1024-aligned shared base
     uint32_t sb;     // shared-space address of the same
@@ -149,21 +160,27 @@ __device__ __forceinline__ bool run_tile(Ctx& c, int width, bool first, float& m
         }
     }
     const float tm = tmax * sl;
+    bool rescale = false;
+    float alpha = 1.0f;
     if (tm > m + 8.0f) {
         const bool had = m != -INFINITY;
-        const float alpha = had ? tc::ex2(m - tm) : 0.0f;
-        if (had && !first) {
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float o[16];
-                tc::tmem_ld16(o_tm + c0, o);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) o[e] *= alpha;
-                tc::tmem_st16(o_tm + c0, o);
-            }
-        }
+        alpha = had ? tc::ex2(m - tm) : 0.0f;
+        rescale = had && !first;
         l *= alpha;
         m = tm;
+    }
+    // TMEM loads/stores are warp-collective: the O round trip runs for the whole warp when any
+    // of its rows needs it (factor 1 for the others)
+    if (__any_sync(0xffffffffu, rescale)) {
+        const float f = rescale ? alpha : 1.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float o[16];
+            tc::tmem_ld16(o_tm + c0, o);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] *= f;
+            tc::tmem_st16(o_tm + c0, o);
+        }
     }
     // pass 2: P = exp2(z*sl - m) into shared memory (row tid, K-major, swizzled)
     const bool live = m != -INFINITY;
@@ -175,8 +192,10 @@ __device__ __forceinline__ bool run_tile(Ctx& c, int width, bool first, float& m
         for (int e = 0; e < 8; ++e) {
             float p0 = (live && valid(c0 + 2 * e)) ? tc::ex2(fmaf(s[2 * e], sl, -m)) : 0.0f;
             float p1 = (live && valid(c0 + 2 * e + 1)) ? tc::ex2(fmaf(s[2 * e + 1], sl, -m)) : 0.0f;
-            l += p0 + p1;
             pk[e] = pack2<T>(p0, p1);
+            // the row sum uses the rounded weights the MMA multiplies V with, so that the
+            // normalised output is an exact convex combination of the rounded weights
+            l += unpack_lo<T>(pk[e]) + unpack_hi<T>(pk[e]);
         }
         uint4* dst0 = reinterpret_cast<uint4*>(c.g + L::kP + tc::tile_off(tid, c0 >> 3));
         uint4* dst1 = reinterpret_cast<uint4*>(c.g + L::kP + tc::tile_off(tid, (c0 >> 3) + 1));
@@ -230,7 +249,9 @@ __device__ __forceinline__ void topk_insert(float (&tv)[KM], int32_t (&ti)[KM], 
     int32_t cb = b;
 #pragma unroll
     for (int t = 0; t < KM; ++t) {
-        const bool better = cz > tv[t];   // strict: an equal logit keeps the earlier, lower index
+        // order: logit descending, then block index ascending (an entry displaced by a larger
+        // logit must still pass equal-logit entries with a higher index)
+        const bool better = cz > tv[t] || (cz == tv[t] && (unsigned)cb < (unsigned)ti[t]);
         const float ov = tv[t];
         const int32_t oi = ti[t];
         tv[t] = better ? cz : ov;
@@ -241,7 +262,7 @@ __device__ __forceinline__ void topk_insert(float (&tv)[KM], int32_t (&ti)[KM], 
 }
 
 // Reads this row's O (D columns) scaled by `f` into registers chunk by chunk and hands each
-// chunk of 16 values to `sink(d0, v)`.
+// chunk of 16 values to `sink(d0, v)`. Warp-collective: every thread of the CTA calls it.
 template <int D, class Sink>
 __device__ __forceinline__ void read_o(const Ctx& c, float f, Sink sink) {
     const uint32_t o_tm = c.tmem + ((uint32_t)((threadIdx.x >> 5) * 32) << 16) + 128;
@@ -255,20 +276,36 @@ __device__ __forceinline__ void read_o(const Ctx& c, float f, Sink sink) {
     }
 }
 
+// Storage type of the per-(query, head, slot) partial outputs: fp16 for fp16 inputs (a partial is
+// a convex combination of V rows, so it cannot overflow fp16, and 2^-11 resolution is kept);
+// fp32 for bf16 inputs (bf16's 2^-8 resolution would dominate the error budget).
+template <typename T>
+using PartT = typename std::conditional<std::is_same<T, __nv_bfloat16>::value, float, __half>::type;
+
+// Normalised partial output and its log2-sum-exp for (pos, h, slot). Called by every thread
+// (TMEM reads are warp-collective); only rows with `row_ok` store.
 template <typename T, int D>
 __device__ __forceinline__ void store_partial(const FwdParams& P, int64_t pos, int h, int slot,
-                                              const Ctx& c, float m, float l) {
-    const float inv = 1.0f / l;
-    T* dst = reinterpret_cast<T*>(P.part_o) + (((int64_t)pos * P.H + h) * P.k + slot) * D;
+                                              bool row_ok, const Ctx& c, float m, float l) {
+    using PT = PartT<T>;
+    const float inv = row_ok ? 1.0f / l : 0.0f;
+    PT* dst = reinterpret_cast<PT*>(P.part_o) + (((int64_t)pos * P.H + h) * P.k + slot) * D;
     read_o<D>(c, inv, [&](int d0, float (&o)[16]) {
-        uint4 a = make_uint4(pack2<T>(o[0], o[1]), pack2<T>(o[2], o[3]), pack2<T>(o[4], o[5]),
-                             pack2<T>(o[6], o[7]));
-        uint4 b = make_uint4(pack2<T>(o[8], o[9]), pack2<T>(o[10], o[11]), pack2<T>(o[12], o[13]),
-                             pack2<T>(o[14], o[15]));
-        reinterpret_cast<uint4*>(dst + d0)[0] = a;
-        reinterpret_cast<uint4*>(dst + d0)[1] = b;
+        if (!row_ok) return;
+        if constexpr (std::is_same<PT, float>::value) {
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<float4*>(dst + d0 + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+        } else {
+            uint4 a = make_uint4(pack2<__half>(o[0], o[1]), pack2<__half>(o[2], o[3]),
+                                 pack2<__half>(o[4], o[5]), pack2<__half>(o[6], o[7]));
+            uint4 b = make_uint4(pack2<__half>(o[8], o[9]), pack2<__half>(o[10], o[11]),
+                                 pack2<__half>(o[12], o[13]), pack2<__half>(o[14], o[15]));
+            reinterpret_cast<uint4*>(dst + d0)[0] = a;
+            reinterpret_cast<uint4*>(dst + d0)[1] = b;
+        }
     });
-    P.part_lse[((int64_t)pos * P.H + h) * P.k + slot] = m + __log2f(l);
+    if (row_ok) P.part_lse[((int64_t)pos * P.H + h) * P.k + slot] = m + __log2f(l);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -349,18 +386,21 @@ __global__ void __launch_bounds__(128) k_qmajor(const FwdParams P) {
                     if (b != ob && z > tv[KM - 1]) topk_insert<KM>(tv, ti, z, b);
                 });
         }
-        if (ok && row_ok) {
-            const float g0 = P.gates[((int64_t)tok * H + h) * 3 + 0];
-            read_o<D>(c, g0 / l, [&](int d0, float (&o)[16]) {
+        if (ok) {
+            const float f = row_ok ? P.gates[((int64_t)tok * H + h) * 3 + 0] / l : 0.0f;
+            read_o<D>(c, f, [&](int d0, float (&o)[16]) {
+                if (!row_ok) return;
 #pragma unroll
                 for (int e = 0; e < 16; e += 4)
                     *reinterpret_cast<float4*>(brow + d0 + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
             });
-            int32_t* srow = P.sel + ((int64_t)pos * H + h) * P.k;
-            srow[0] = ob;
+            if (row_ok) {
+                int32_t* srow = P.sel + ((int64_t)pos * H + h) * P.k;
+                srow[0] = ob;
 #pragma unroll
-            for (int t = 0; t < KM; ++t)
-                if (t + 1 < P.k) srow[t + 1] = ti[t];
+                for (int t = 0; t < KM; ++t)
+                    if (t + 1 < P.k) srow[t + 1] = ti[t];
+            }
         }
     }
 
@@ -392,9 +432,10 @@ __global__ void __launch_bounds__(128) k_qmajor(const FwdParams P) {
                 },
                 [](int, float) {});
         }
-        if (ok && row_ok) {
-            const float g2 = P.gates[((int64_t)tok * H + h) * 3 + 2];
-            read_o<D>(c, g2 / l, [&](int d0, float (&o)[16]) {
+        if (ok) {
+            const float f = row_ok ? P.gates[((int64_t)tok * H + h) * 3 + 2] / l : 0.0f;
+            read_o<D>(c, f, [&](int d0, float (&o)[16]) {
+                if (!row_ok) return;
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {
                     float4 b = *reinterpret_cast<float4*>(brow + d0 + e);
@@ -424,7 +465,7 @@ __global__ void __launch_bounds__(128) k_qmajor(const FwdParams P) {
                 c, width, j0 == 0, m, l, P.sl, P.status, [&](int col) { return kmeta[col].w == ob; },
                 [](int, float) {});
         }
-        if (ok && row_ok) store_partial<T, D>(P, pos, h, 0, c, m, l);
+        if (ok) store_partial<T, D>(P, pos, h, 0, row_ok, c, m, l);
     }
 
     tc::fence_before_sync();
@@ -503,7 +544,7 @@ __global__ void __launch_bounds__(128) k_kbmajor(const FwdParams P, int64_t HMb)
             ok = run_tile<T, D>(c, width, j0 == 0, m, l, P.sl, P.status,
                                 [&](int col) { return col < lim; }, [](int, float) {});
         }
-        if (ok && row_ok) store_partial<T, D>(P, pos, h, slot, c, m, l);
+        if (ok) store_partial<T, D>(P, pos, h, slot, row_ok, c, m, l);
     }
 
     tc::fence_before_sync();
@@ -569,7 +610,7 @@ __global__ void k_combine(const FwdParams P) {
     for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
     const int32_t tok = P.perm[pos];
     const float g1 = P.gates[((int64_t)tok * P.H + h) * 3 + 1] / tot;
-    const T* po = reinterpret_cast<const T*>(P.part_o) + w * k * D;
+    const PartT<T>* po = reinterpret_cast<const PartT<T>*>(P.part_o) + w * k * D;
     T* out = reinterpret_cast<T*>(P.out) + ((int64_t)tok * P.H + h) * D;
     const float* brow = P.base + w * D;
 #pragma unroll
@@ -577,7 +618,7 @@ __global__ void k_combine(const FwdParams P) {
         float acc = 0.0f;
         for (int s = 0; s < k; ++s) {
             const float ws = __shfl_sync(0xffffffffu, wgt, s);
-            if (ws != 0.0f) acc += ws * Elem<T>::to_f(po[s * D + d]);
+            if (ws != 0.0f) acc += ws * Elem<PartT<T>>::to_f(po[s * D + d]);
         }
         out[d] = Elem<T>::from_f(brow[d] + g1 * acc);
     }
@@ -604,19 +645,35 @@ void run_forward(const Plan* p, const FwdParams& P, cudaStream_t st, int num_sms
     const Workspace& w = p->ws;
     const int64_t NH = p->N * P.H;
     const int64_t HMb = (int64_t)P.H * p->Mb;
-    k_qmajor<T, D, KM><<<dim3((unsigned)p->n_qtiles, (unsigned)P.H), 128, L::kAlloc, st>>>(P);
-    cudaMemsetAsync(w.inv_cnt, 0, sizeof(int32_t) * (HMb + 1), st);
-    cudaMemsetAsync(w.inv_fill, 0, sizeof(int32_t) * (HMb + 1), st);
-    const unsigned g256 = (unsigned)cdiv(NH, 256);
-    k_inv_count<<<g256, 256, 0, st>>>(w.sel, NH, P.H, P.k, p->Mb, w.inv_cnt);
-    note_launch(2);
-    scan_exclusive(w.inv_cnt, w.inv_off, HMb, w.scan_tmp, st);
-    k_inv_items<<<(unsigned)cdiv(HMb, 256), 256, 0, st>>>(w.inv_cnt, HMb, w.item_cnt);
-    note_launch();
-    scan_exclusive(w.item_cnt, w.item_off, HMb, w.scan_tmp, st);
-    k_inv_fill<<<g256, 256, 0, st>>>(w.sel, NH, P.H, P.k, p->Mb, w.inv_off, w.inv_fill, w.inv_list);
-    k_kbmajor<T, D><<<(unsigned)(2 * num_sms), 128, L::kAlloc, st>>>(P, HMb);
-    k_combine<T, D><<<(unsigned)cdiv(NH * 32, 256), 256, 0, st>>>(P);
+    {
+        ProfScope ps("k_qmajor", st);
+        k_qmajor<T, D, KM><<<dim3((unsigned)p->n_qtiles, (unsigned)P.H), 128, L::kAlloc, st>>>(P);
+    }
+    trace_step("k_qmajor", st);
+    {
+        ProfScope ps("selection_inversion", st);
+        cudaMemsetAsync(w.inv_cnt, 0, sizeof(int32_t) * (HMb + 1), st);
+        cudaMemsetAsync(w.inv_fill, 0, sizeof(int32_t) * (HMb + 1), st);
+        const unsigned g256 = (unsigned)cdiv(NH, 256);
+        k_inv_count<<<g256, 256, 0, st>>>(w.sel, NH, P.H, P.k, p->Mb, w.inv_cnt);
+        note_launch(2);
+        scan_exclusive(w.inv_cnt, w.inv_off, HMb, w.scan_tmp, st);
+        k_inv_items<<<(unsigned)cdiv(HMb, 256), 256, 0, st>>>(w.inv_cnt, HMb, w.item_cnt);
+        note_launch();
+        scan_exclusive(w.item_cnt, w.item_off, HMb, w.scan_tmp, st);
+        k_inv_fill<<<g256, 256, 0, st>>>(w.sel, NH, P.H, P.k, p->Mb, w.inv_off, w.inv_fill, w.inv_list);
+    }
+    trace_step("selection inversion", st);
+    {
+        ProfScope ps("k_kbmajor", st);
+        k_kbmajor<T, D><<<(unsigned)(2 * num_sms), 128, L::kAlloc, st>>>(P, HMb);
+    }
+    trace_step("k_kbmajor", st);
+    {
+        ProfScope ps("k_combine", st);
+        k_combine<T, D><<<(unsigned)cdiv(NH * 32, 256), 256, 0, st>>>(P);
+    }
+    trace_step("k_combine", st);
     note_launch(3);
 }
 

@@ -106,6 +106,33 @@ struct Plan {
 
 extern std::atomic<int64_t> g_launches;
 inline void note_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+// Opt-in launch trace (environment variable SSA_TRACE=1): waits for `st` after the named step
+// and reports it on stderr with its duration. Off by default; used to locate a stuck kernel.
+void trace_step(const char* what, cudaStream_t st);
+
+// Opt-in kernel timing (ssa_profile_enable): a ProfScope brackets one launch with CUDA events on
+// the launch stream; ssa_profile_read accumulates the durations per kernel name.
+bool profiling_on();
+void profile_record(const char* name, cudaEvent_t start, cudaEvent_t stop);
+cudaEvent_t profile_event();
+struct ProfScope {
+    const char* name;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr;
+    ProfScope(const char* n, cudaStream_t s) : name(n), st(s) {
+        if (profiling_on()) {
+            a = profile_event();
+            cudaEventRecord(a, st);
+        }
+    }
+    ~ProfScope() {
+        if (a) {
+            cudaEvent_t b = profile_event();
+            cudaEventRecord(b, st);
+            profile_record(name, a, b);
+        }
+    }
+};
 
 // ---- allocation through the plan's hook -------------------------------------------------------
 void* plan_alloc(Plan* p, size_t bytes);

@@ -411,6 +411,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     k_keys_and_hash<<<grid_for(N), kThreads, 0, st>>>(coords, N, p->d_seqs, B, tok_key, key_cnt,
                                                       hkeys, hvals, hsize - 1, p->d_status);
     k_occupied<<<grid_for(G), kThreads, 0, st>>>(key_cnt, G, bidx);
+    trace_step("plan keys+hash", st);
     note_launch(2);
     scan_exclusive(bidx, bidx, G, tmp, st);
     k_blocks<<<grid_for(G), kThreads, 0, st>>>(key_cnt, bidx, G, p->d_seqs, B, key2blk, blk_cnt,
@@ -418,6 +419,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     note_launch();
     scan_exclusive(blk_cnt, p->blk_off, cap_mb, tmp, st);
     scan_exclusive(blk_pcnt, p->blk_poff, cap_mb, tmp, st);
+    trace_step("plan blocks", st);
 
     // ---- a2: neighbour counts --------------------------------------------------------------------
     const int cube = (2 * r + 1) * (2 * r + 1) * (2 * r + 1);
@@ -429,6 +431,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         p->d_status);
     note_launch();
     scan_exclusive(nbr_cnt, p->nbr_off32, N, tmp, st);
+    trace_step("plan neighbour counts", st);
 
     // ---- first wait: sizes and coordinate errors --------------------------------------------------
     int32_t h_sizes[4];
@@ -462,6 +465,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
                                                         make_int4(1 << 28, 1 << 28, 1 << 28, -1));
     k_positions<<<grid_for(N), kThreads, 0, st>>>(p->perm, p->tok_blk, p->blk_off, p->blk_poff,
                                                   p->coords, N, p->tok_pos, p->spos_tok, p->scoord);
+    trace_step("plan scatter/sort/positions", st);
     note_launch(5);
 
     // ---- a2: neighbour lists -----------------------------------------------------------------------
@@ -496,11 +500,13 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         p->qt_pos, p->qt_len, p->qt_seq, p->perm, p->tok_blk, p->coords, p->blk_coord, p->blk_poff,
         p->blk_off, key2blk, p->d_seqs, p->scoord, r, wt_cnt, nullptr, nullptr);
     note_launch();
+    trace_step("plan neighbour lists + window union counts", st);
     scan_exclusive(wt_cnt, p->wt_off, T, tmp, st);
     k_window_union<true><<<(unsigned)T, 128, 0, st>>>(
         p->qt_pos, p->qt_len, p->qt_seq, p->perm, p->tok_blk, p->coords, p->blk_coord, p->blk_poff,
         p->blk_off, key2blk, p->d_seqs, p->scoord, r, nullptr, p->wt_off, p->wt_keys);
     note_launch();
+    trace_step("plan window unions", st);
 
     // block range of every sequence (host copy for launches)
     p->seq_blk.assign(B + 1, 0);

@@ -62,6 +62,19 @@ def check_close(gpu, ref, dtype, what=""):
     return err, r
 
 
+def check_grad_close(gpu, ref, dtype, what=""):
+    """Gradients: no tolerance is stated for them, so the bound is taken relative to the tensor's
+    scale: max|delta| <= 1e-2 * max|ref| (about 2.5 bf16 ulps at the largest element) and
+    relative L2 <= 5e-3; fp32 inputs: 1e-5 for both."""
+    atol, rtol = TOL[dtype]
+    scale = float(np.abs(ref).max()) if ref.size else 1.0
+    err = float(np.abs(gpu - ref).max()) if gpu.size else 0.0
+    r = rel_l2(gpu, ref)
+    assert err <= atol * scale and r <= rtol, (
+        f"{what}: max|d|={err:.3e} (<= {atol}*{scale:.3e}), relL2={r:.3e} (<= {rtol})")
+    return err, r
+
+
 def selection_agreement(gpu_sel, ora_sel, z_rows, blk_base_of_row, dtype):
     """Compare selections per (row, head). Returns (mismatch mask [R,H], report).
 

@@ -11,17 +11,38 @@ import torch
 
 import oracle
 import workloads
-from ssa_testlib import check_close, coords_of, make_plan, rel_l2, tensors_of, to_gpu
+from ssa_testlib import check_grad_close, coords_of, make_plan, rel_l2, tensors_of, to_gpu
 
 pytestmark = pytest.mark.gpu
 
 
 def gpu_backward(plan, t, topk):
+    """GPU gradients and the GPU's selection ([N, H, k])."""
     g = to_gpu(t)
     dq, dk, dv = plan.backward(g["Q"], g["K"], g["V"], g["gates"], g["Wc"], g["dO"], topk)
+    _, sel = plan.forward(g["Q"], g["K"], g["V"], g["gates"], g["Wc"], topk, return_sel=True)
     torch.cuda.synchronize()
     assert plan.status() == 0
-    return [x.double().cpu().numpy() for x in (dq, dk, dv)]
+    return [x.double().cpu().numpy() for x in (dq, dk, dv)] + [sel.cpu().numpy()]
+
+
+def swapped_keys(gpu_sel, ora_sel, blk_off, perm, H):
+    """[N, H] mask of (key, head) pairs whose gradient receives a contribution that differs between
+    the two selections: the tokens of every block in the symmetric difference of a (query, head)
+    pair's two block sets."""
+    mask = np.zeros((len(perm), H), bool)
+    diff = np.nonzero(~same_selection(gpu_sel, ora_sel))
+    for i, h in zip(*diff):
+        for b in set(gpu_sel[i, h].tolist()) ^ set(ora_sel[i, h].tolist()):
+            if b >= 0:
+                mask[perm[blk_off[b]:blk_off[b + 1]], h] = True
+    return mask
+
+
+def same_selection(gpu_sel, ora_sel):
+    """[R, H] mask of (row, head) pairs whose selected block sets agree. Rows that differ (near
+    ties, validated by the forward tests) attend to different keys, so their dQ is not comparable."""
+    return np.all(np.sort(gpu_sel, axis=2) == np.sort(ora_sel, axis=2), axis=2)
 
 
 @pytest.mark.parametrize("name", ["tiny", "small"])
@@ -30,11 +51,19 @@ def test_backward_full(name):
     c, cu, g = coords_of(name)
     t = tensors_of(name, with_grad_out=True)
     plan = make_plan(c, cu, g, cfg.radius)
-    got = gpu_backward(plan, t, cfg.topk)
+    dq, dk, dv, sel = gpu_backward(plan, t, cfg.topk)
     ref = oracle.backward(c, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], t["dO"], cfg.topk,
                           cfg.radius)
-    for a, b, what in zip(got, ref, ("dQ", "dK", "dV")):
-        check_close(a, b, cfg.dtype, what)
+    ora_sel = oracle.forward(c, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], cfg.topk,
+                             cfg.radius)["sel"]
+    keep = same_selection(sel, ora_sel)
+    assert keep.mean() >= 0.99
+    check_grad_close(dq[keep], ref[0][keep], cfg.dtype, "dQ")
+    pl = oracle.plan(c, cu, 8, cfg.radius)
+    kk = ~swapped_keys(sel, ora_sel, pl["blk_off"], pl["perm"], cfg.H)
+    assert kk.mean() >= 0.9, kk.mean()
+    check_grad_close(dk[kk], ref[1][kk], cfg.dtype, "dK")
+    check_grad_close(dv[kk], ref[2][kk], cfg.dtype, "dV")
 
 
 @pytest.mark.slow
@@ -43,11 +72,13 @@ def test_backward_varlen_sampled_rows_and_sums():
     c, cu, g = coords_of("varlen")
     t = tensors_of("varlen", with_grad_out=True)
     plan = make_plan(c, cu, g, cfg.radius)
-    dq, dk, dv = gpu_backward(plan, t, cfg.topk)
+    dq, dk, dv, sel = gpu_backward(plan, t, cfg.topk)
     rows = np.concatenate(workloads.stratified_rows(cu, 512, seed=5099))
-    ref = oracle.backward_dq_rows(c, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], t["dO"],
-                                  cfg.topk, cfg.radius, rows)
-    check_close(dq[rows], ref, cfg.dtype, "dQ rows")
+    ref, ora_sel = oracle.backward_dq_rows(c, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"],
+                                           t["dO"], cfg.topk, cfg.radius, rows, return_sel=True)
+    keep = same_selection(sel[rows], ora_sel)
+    assert keep.mean() >= 0.99
+    check_grad_close(dq[rows][keep], ref[keep], cfg.dtype, "dQ rows")
     gates = t["gates"].double().numpy()
     dO = t["dO"].double().numpy()
     Wc = t["Wc"].double().numpy()

@@ -280,7 +280,7 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
     }
     trace_step("pool", st);
     if (dt == SSA_F32) launch_forward_simt(p, w, q, k, v, gates, out, st);
-    else launch_forward_tc(p, w, q, gates, out, st);
+    else if (!launch_forward_tc(p, w, q, gates, out, st)) return SSA_ERR_CUDA;
     trace_step("forward", st);
     if (sel_out) launch_export_sel(p, w, sel_out, st);
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;

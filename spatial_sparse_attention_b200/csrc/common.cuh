@@ -156,7 +156,7 @@ void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const
                          const void* v, const float* gates, void* out, cudaStream_t s);
 
 // attn_tc.cu (bf16 / fp16 path)
-void launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
+bool launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
                        void* out, cudaStream_t s);
 
 // backward.cu

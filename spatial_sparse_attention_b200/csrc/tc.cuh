@@ -51,6 +51,14 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk) {
     return smem_desc(base + (uint32_t)kk * 1024, kRegion, 512);
 }
 
+// Same, for tiles whose 32-element chunks are `region` bytes apart.
+__device__ __forceinline__ uint64_t desc_kmajor_r(uint32_t base, int kk, uint32_t region) {
+    return smem_desc(base + (uint32_t)(kk >> 1) * region + (uint32_t)(kk & 1) * 32, 16, 512);
+}
+__device__ __forceinline__ uint64_t desc_mnmajor_r(uint32_t base, int kk, uint32_t region) {
+    return smem_desc(base + (uint32_t)kk * 1024, region, 512);
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator (bit 4), A/B type (bits 7-9 / 10-12:
 // 0 = f16, 1 = bf16), A K-major (bit 15 = 0), B major (bit 16), N >> 3 (bits 17-22),
 // M >> 4 (bits 24-28).
@@ -146,6 +154,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
         if (clock64() - t0 > max_cycles) return false;
     }
     return false;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Arrive and add `bytes` to the transaction count the current phase waits for (TMA loads
+// complete_tx against it).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// ---- TMA ----------------------------------------------------------------------------------------
+// 2D tiled bulk tensor load (no multicast): box at coordinates (x = innermost element index,
+// y = row) of the tensor described by `tmap` into shared memory at `dst`, completing `bytes`
+// transactions on `bar`. x * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
 // ---- copies ---------------------------------------------------------------------------------------

@@ -49,8 +49,7 @@ struct QL {
 };
 
 enum : int {
-    KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, SFREE = 10, PFULL = 12, ODONE = 14,
-    NBAR = 15
+    KFULL = 0, KEMPTY = 2, VFULL = 4, VEMPTY = 6, SFULL = 8, SFREE = 10, PFULL = 12, NBAR = 14
 };
 
 struct Sched {
@@ -61,6 +60,87 @@ struct Sched {
     __device__ bool first(int j) const { return j == 0 || j == nc || j == nc + no; }
 };
 
+// Key mask of phase PH for column `col` of the current tile.
+template <int PH>
+__device__ __forceinline__ bool key_valid(int col, const int4* km, int lim, int4 qc, int32_t ob, int rr) {
+    if (PH == 0) return col < lim;
+    const int4 kc = km[col];
+    if (PH == 1) return kc.w == ob;
+    return col < lim && max(abs(kc.x - qc.x), max(abs(kc.y - qc.y), abs(kc.z - qc.z))) <= rr;
+}
+
+// v[e] for a per-thread index e, by a tree of selects (stays in registers)
+__device__ __forceinline__ float pick16(const float (&v)[16], int e) {
+    float a[8], b[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) b[i] = (e & 2) ? a[2 * i + 1] : a[2 * i];
+    const float c0 = (e & 4) ? b[1] : b[0];
+    const float c1 = (e & 4) ? b[3] : b[2];
+    return (e & 8) ? c1 : c0;
+}
+
+// Pass 1 over one S tile: the row max of the valid keys; in phase 0 also the running top-(k-1)
+// of the other blocks (candidates above the current k-1-th logit are collected as a bit mask per
+// 16 columns and inserted one by one).
+template <int PH, int KM>
+__device__ __forceinline__ float softmax_pass1(uint32_t s_tm, const int4* km, int lim, int4 qc,
+                                               int32_t ob, int rr, int32_t bbase, float (&tv)[KM],
+                                               int32_t (&ti)[KM]) {
+    float tmax = -INFINITY;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kKT; c0 += 16) {
+        float sv[16];
+        tc::tmem_ld16(s_tm + c0, sv);
+        uint32_t cand = 0;
+        const float thr = tv[KM - 1];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const bool v = key_valid<PH>(c0 + e, km, lim, qc, ob, rr);
+            tmax = fmaxf(tmax, v ? sv[e] : -INFINITY);
+            if (PH == 0) cand |= (uint32_t)(v && sv[e] > thr && bbase + c0 + e != ob) << e;
+        }
+        if (PH == 0) {
+            while (cand) {
+                const int e = __ffs(cand) - 1;
+                cand &= cand - 1;
+                topk_insert<KM>(tv, ti, pick16(sv, e), bbase + c0 + e);
+            }
+        }
+    }
+    return tmax;
+}
+
+// Pass 2: P = 2^(z*sl - m) rounded to T into this row of the P tile; l accumulates the rounded
+// weights.
+template <typename T, int PH, uint32_t kPReg>
+__device__ __forceinline__ void softmax_pass2(uint32_t s_tm, const int4* km, int lim, int4 qc,
+                                              int32_t ob, int rr, float sl, float m, uint8_t* pbuf,
+                                              int row, float& l) {
+    const bool live = m != -INFINITY;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kKT; c0 += 16) {
+        float sv[16];
+        tc::tmem_ld16(s_tm + c0, sv);
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const bool v0 = live && key_valid<PH>(c0 + 2 * e, km, lim, qc, ob, rr);
+            const bool v1 = live && key_valid<PH>(c0 + 2 * e + 1, km, lim, qc, ob, rr);
+            const float a0 = v0 ? tc::ex2(fmaf(sv[2 * e], sl, -m)) : 0.0f;
+            const float a1 = v1 ? tc::ex2(fmaf(sv[2 * e + 1], sl, -m)) : 0.0f;
+            pk[e] = pack2<T>(a0, a1);
+            l += unpack_lo<T>(pk[e]) + unpack_hi<T>(pk[e]);
+        }
+        const int c16 = c0 >> 3;
+        *reinterpret_cast<uint4*>(pbuf + (c16 >> 2) * kPReg + tc::sw64(row, c16 & 3)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(pbuf + ((c16 + 1) >> 2) * kPReg + tc::sw64(row, (c16 + 1) & 3)) =
+            make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+}
+
 __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int32_t* status) {
     if (tc::mbar_wait(bar, parity, kWaitCycles)) return true;
     atomicOr(status, DEV_TIMEOUT);
@@ -68,7 +148,7 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
 }
 
 template <typename T, int D, int KM>
-__global__ void __launch_bounds__(kThreadsQ) k_qmajor(const __grid_constant__ FwdParams P,
+__global__ void __launch_bounds__(kThreadsQ, 2) k_qmajor(const __grid_constant__ FwdParams P,
                                                       const __grid_constant__ CUtensorMap tm_kc,
                                                       const __grid_constant__ CUtensorMap tm_vc,
                                                       const __grid_constant__ CUtensorMap tm_ks,
@@ -128,6 +208,14 @@ __global__ void __launch_bounds__(kThreadsQ) k_qmajor(const __grid_constant__ Fw
 
     const T* KS = reinterpret_cast<const T*>(P.ks) + (int64_t)h * P.Npad * D;
     const T* VS = reinterpret_cast<const T*>(P.vs) + (int64_t)h * P.Npad * D;
+
+    // P V of tile i has completed. Its barrier (V stage i&1, phase i>>1) is committed right after
+    // that MMA. Waits on a barrier's phases must not skip one: a parity wait only tells the
+    // current phase from the one before it, and the tensor core may finish a later S before an
+    // earlier P V. Every user of these barriers waits for P V of tile i-2 before tile i.
+    auto pv_done = [&](int i) -> bool {
+        return wait_or_flag(&bar[VEMPTY + (i & 1)], (uint32_t)(i >> 1) & 1u, P.status);
+    };
 
     if (warp == 0) {
         // ================================ producer ============================================
@@ -210,8 +298,7 @@ __global__ void __launch_bounds__(kThreadsQ) k_qmajor(const __grid_constant__ Fw
                     tc::mma_f16_ss(tmem + 128, tc::desc_kmajor_r(pbase, kk, L::kPReg),
                                    tc::desc_mnmajor_r(vbase, kk, L::kKVReg), idesc_o,
                                    (sc.first(i) && kk == 0) ? 0u : 1u);
-                tc::mma_commit(&bar[ODONE]);
-                tc::mma_commit(&bar[VEMPTY + bb]);
+                tc::mma_commit(&bar[VEMPTY + bb]);   // P V of tile i done: V stage, P buffer, O
                 return true;
             };
             bool ok = true;
@@ -292,7 +379,7 @@ __global__ void __launch_bounds__(kThreadsQ) k_qmajor(const __grid_constant__ Fw
         for (int j = 0; j < nT; ++j) {
             const int ph = sc.phase(j), t = sc.local(j), b = j & 1;
             if (sc.first(j) && j > 0) {
-                if (!(ok = wait_or_flag(&bar[ODONE], (uint32_t)(j - 1) & 1u, P.status))) break;
+                if (!(ok = pv_done(j - 1))) break;
                 epilogue(sc.phase(j - 1));
                 m = -INFINITY;
                 l = 0.0f;
@@ -304,28 +391,11 @@ __global__ void __launch_bounds__(kThreadsQ) k_qmajor(const __grid_constant__ Fw
             const int4* km = meta + b * kKT;
             const int lim = ph == 0 ? nkeys - kKT * t : nwin - kKT * t;
             const int32_t bbase = bl + kKT * t;
-            auto valid = [&](int col) -> bool {
-                if (ph == 0) return col < lim;
-                const int4 kc = km[col];
-                if (ph == 1) return kc.w == ob;
-                return col < lim && max(abs(kc.x - qc.x), max(abs(kc.y - qc.y), abs(kc.z - qc.z))) <= rr;
-            };
             // pass 1: tile max (+ running top-k of the other blocks in phase 0)
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int c0 = 0; c0 < kKT; c0 += 16) {
-                float sv[16];
-                tc::tmem_ld16(s_tm + c0, sv);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    if (!valid(c0 + e)) continue;
-                    tmax = fmaxf(tmax, sv[e]);
-                    if (ph == 0) {
-                        const int32_t bk = bbase + c0 + e;
-                        if (bk != ob && sv[e] > tv[KM - 1]) topk_insert<KM>(tv, ti, sv[e], bk);
-                    }
-                }
-            }
+            const float tmax =
+                ph == 0 ? softmax_pass1<0, KM>(s_tm, km, lim, qc, ob, rr, bbase, tv, ti)
+                : ph == 1 ? softmax_pass1<1, KM>(s_tm, km, lim, qc, ob, rr, bbase, tv, ti)
+                          : softmax_pass1<2, KM>(s_tm, km, lim, qc, ob, rr, bbase, tv, ti);
             const float tm = tmax * sl;
             bool rescale = false;
             float alpha = 1.0f;
@@ -338,7 +408,7 @@ __global__ void __launch_bounds__(kThreadsQ) k_qmajor(const __grid_constant__ Fw
             }
             if (__any_sync(0xffffffffu, rescale)) {
                 // O must hold P V of the previous tile before it is rescaled
-                if (!(ok = wait_or_flag(&bar[ODONE], (uint32_t)(j - 1) & 1u, P.status))) break;
+                if (!(ok = pv_done(j - 1))) break;
                 tc::fence_after_sync();
                 const float f = rescale ? alpha : 1.0f;
 #pragma unroll 1
@@ -350,33 +420,21 @@ __global__ void __launch_bounds__(kThreadsQ) k_qmajor(const __grid_constant__ Fw
                     tc::tmem_st16(o_tm + d0, o);
                 }
             }
+            // P buffer b was last read by P V of tile j-2: wait for it explicitly (its completion
+            // releases V stage b), MMA completion order is not relied upon
+            if (j >= 2 && !(ok = wait_or_flag(&bar[VEMPTY + b], (uint32_t)((j >> 1) - 1) & 1u, P.status)))
+                break;
             // pass 2: P = 2^(z*sl - m), rounded to T, into P buffer b (this row, swizzled)
-            const bool live = m != -INFINITY;
             uint8_t* pbuf = g + L::kP + b * 2 * L::kPReg;
-#pragma unroll
-            for (int c0 = 0; c0 < kKT; c0 += 16) {
-                float sv[16];
-                tc::tmem_ld16(s_tm + c0, sv);
-                uint32_t pk[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float a0 = (live && valid(c0 + 2 * e)) ? tc::ex2(fmaf(sv[2 * e], sl, -m)) : 0.0f;
-                    const float a1 = (live && valid(c0 + 2 * e + 1)) ? tc::ex2(fmaf(sv[2 * e + 1], sl, -m)) : 0.0f;
-                    pk[e] = pack2<T>(a0, a1);
-                    l += unpack_lo<T>(pk[e]) + unpack_hi<T>(pk[e]);
-                }
-                const int c16 = c0 >> 3;
-                *reinterpret_cast<uint4*>(pbuf + (c16 >> 2) * L::kPReg + tc::sw64(row, c16 & 3)) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(pbuf + ((c16 + 1) >> 2) * L::kPReg + tc::sw64(row, (c16 + 1) & 3)) =
-                    make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
+            if (ph == 0) softmax_pass2<T, 0, L::kPReg>(s_tm, km, lim, qc, ob, rr, sl, m, pbuf, row, l);
+            else if (ph == 1) softmax_pass2<T, 1, L::kPReg>(s_tm, km, lim, qc, ob, rr, sl, m, pbuf, row, l);
+            else softmax_pass2<T, 2, L::kPReg>(s_tm, km, lim, qc, ob, rr, sl, m, pbuf, row, l);
             tc::fence_proxy_async();
             tc::fence_before_sync();
             tc::mbar_arrive(&bar[SFREE + b]);
             tc::mbar_arrive(&bar[PFULL + b]);
         }
-        if (ok && nT > 0 && wait_or_flag(&bar[ODONE], (uint32_t)(nT - 1) & 1u, P.status))
+        if (ok && nT > 0 && pv_done(nT - 1))
             epilogue(sc.phase(nT - 1));
     }
 
@@ -423,14 +481,17 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int D, bool bf16) 
 template <typename T, int D, int KM>
 bool run(const Plan* p, const FwdParams& P, const CUtensorMap* tm, cudaStream_t st) {
     using L = QL<D>;
+    static_assert(L::kAlloc <= 227u * 1024u, "shared-memory layout exceeds the per-CTA limit");
     static bool configured = false;
     if (!configured) {
-        cudaFuncSetAttribute(k_qmajor<T, D, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+        if (cudaFuncSetAttribute(k_qmajor<T, D, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)L::kAlloc) != cudaSuccess)
+            return false;
         configured = true;
     }
     k_qmajor<T, D, KM><<<dim3((unsigned)p->n_qtiles, (unsigned)P.H), kThreadsQ, L::kAlloc, st>>>(
         P, tm[0], tm[1], tm[2], tm[3]);
-    return true;
+    return cudaPeekAtLastError() == cudaSuccess;
 }
 
 template <typename T, int D>

@@ -120,7 +120,7 @@ __global__ void k_inv_count(const int32_t* __restrict__ sel, int64_t NH, int H, 
     const int h = (int)(w % H);
     for (int s = 1; s < k; ++s) {
         int32_t b = sel[w * k + s];
-        if (b >= 0) atomicAdd(&inv_cnt[(int64_t)h * Mb + b], 1);
+        if (b >= 0 && b < Mb) atomicAdd(&inv_cnt[(int64_t)h * Mb + b], 1);
     }
 }
 
@@ -138,7 +138,7 @@ __global__ void k_inv_fill(const int32_t* __restrict__ sel, int64_t NH, int H, i
     const int32_t pos = (int32_t)(w / H);
     for (int s = 1; s < k; ++s) {
         int32_t b = sel[w * k + s];
-        if (b < 0) continue;
+        if (b < 0 || b >= Mb) continue;
         int64_t hb = (int64_t)h * Mb + b;
         inv_list[inv_off[hb] + atomicAdd(&inv_fill[hb], 1)] = (pos << 5) | s;
     }

@@ -106,6 +106,7 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 // 32w..32w+31). Load and wait are fused so no register is read before it is valid.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
+    __syncwarp();   // .sync.aligned: the whole warp must arrive converged
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
         "[%16];\n\ttcgen05.wait::ld.sync.aligned;"
@@ -118,6 +119,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    __syncwarp();
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
         "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
@@ -144,11 +146,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     const long long t0 = clock64();
     for (uint32_t it = 0; it < (1u << 26); ++it) {
         uint32_t ok;
+        // the waiting thread is suspended (not polling) until the phase completes or ~0.1 ms pass
         asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}\n"
             : "=r"(ok)
-            : "r"(addr), "r"(parity)
+            : "r"(addr), "r"(parity), "r"(100000u)
             : "memory");
         if (ok) return true;
         if (clock64() - t0 > max_cycles) return false;

@@ -28,12 +28,13 @@ def gpu_backward(plan, t, topk):
 
 def swapped_keys(gpu_sel, ora_sel, blk_off, perm, H):
     """[N, H] mask of (key, head) pairs whose gradient receives a contribution that differs between
-    the two selections: the tokens of every block in the symmetric difference of a (query, head)
-    pair's two block sets."""
+    the two selections. The selected branch is one softmax over all tokens of a row's selected
+    blocks, so a swapped block changes the normaliser and with it the weight of every selected
+    token: the mask covers the tokens of every block in the union of the pair's two block sets."""
     mask = np.zeros((len(perm), H), bool)
     diff = np.nonzero(~same_selection(gpu_sel, ora_sel))
     for i, h in zip(*diff):
-        for b in set(gpu_sel[i, h].tolist()) ^ set(ora_sel[i, h].tolist()):
+        for b in set(gpu_sel[i, h].tolist()) | set(ora_sel[i, h].tolist()):
             if b >= 0:
                 mask[perm[blk_off[b]:blk_off[b + 1]], h] = True
     return mask

@@ -192,7 +192,7 @@ SSA_API int64_t ssa_launch_count(void);
 
 /*
  * Kernel timing (measurement support, not part of the method). When enabled, each hot step
- * (plan, pool, k_qmajor, selection_inversion, k_kbmajor, k_combine) is bracketed by two CUDA
+ * (plan, pool, k_ssa_fwd) is bracketed by two CUDA
  * events recorded on the stream it is launched on. ssa_profile_read waits for the recorded
  * events, adds their durations to per-name totals and copies up to max_entries totals out:
  * names (host char[max_entries][64], NUL-terminated), total_ms and launches (host arrays; any

@@ -224,24 +224,10 @@ ssa_status_t ensure_workspace(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int
     w.sel = (int32_t*)A(sizeof(int32_t) * N * H * k);
     if (!w.kc || !w.vc || !w.sel) return SSA_ERR_ALLOC;
     if (dt != SSA_F32) {
-        const int64_t HMb = (int64_t)H * Mb;
         w.ks = A(es * H * p->Npad * D);
         w.vs = A(es * H * p->Npad * D);
         w.base = (float*)A(sizeof(float) * N * H * D);
-        // partials: fp16 for fp16 inputs, fp32 for bf16 inputs
-        w.part_o = A((dt == SSA_BF16 ? 4 : 2) * N * H * k * D);
-        w.part_lse = (float*)A(sizeof(float) * N * H * k);
-        w.inv_cnt = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
-        w.inv_off = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
-        w.inv_fill = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
-        w.inv_list = (int32_t*)A(sizeof(int32_t) * std::max<int64_t>(1, N * H * (k - 1)));
-        w.item_cnt = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
-        w.item_off = (int32_t*)A(sizeof(int32_t) * (HMb + 1));
-        w.scan_tmp_len = scan_tmp_len(HMb + 1);
-        w.scan_tmp = (int32_t*)A(sizeof(int32_t) * w.scan_tmp_len);
-        if (!w.ks || !w.vs || !w.base || !w.part_o || !w.part_lse || !w.inv_cnt || !w.inv_off ||
-            !w.inv_fill || !w.inv_list || !w.item_cnt || !w.item_off || !w.scan_tmp)
-            return SSA_ERR_ALLOC;
+        if (!w.ks || !w.vs || !w.base) return SSA_ERR_ALLOC;
         // padding rows of the block-ordered copies stay zero for the life of the workspace
         if (cudaMemsetAsync(w.ks, 0, es * H * p->Npad * D, st) ||
             cudaMemsetAsync(w.vs, 0, es * H * p->Npad * D, st))
@@ -280,7 +266,7 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
     }
     trace_step("pool", st);
     if (dt == SSA_F32) launch_forward_simt(p, w, q, k, v, gates, out, st);
-    else if (!launch_forward_tc(p, w, q, gates, out, st)) return SSA_ERR_CUDA;
+    else if ((rc = launch_forward_tc(p, w, q, gates, out, st)) != SSA_OK) return rc;
     trace_step("forward", st);
     if (sel_out) launch_export_sel(p, w, sel_out, st);
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;

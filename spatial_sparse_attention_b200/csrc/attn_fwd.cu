@@ -1,0 +1,771 @@
+// Fused forward of Spatial Sparse Attention on the sm_100a tensor cores, bf16 / fp16 inputs with
+// fp32 accumulation (Direct3D-S2 summary page, "Technical principles", SSA item: compressed block
+// tokens, selection of the important blocks from the compression branch's attention scores, a
+// local window, and the gated sum of the three branches).
+//
+// One CTA per (query tile of 128 tokens in block order, head). The CTA streams 64-key tiles
+// through three phases, each one softmax per row:
+//   C  the compressed tokens of the sequence (block mean . Wc). Each row keeps a running list of
+//      its top-(k-1) other blocks by compressed logit; the own block is slot 0.
+//   S  the selected tokens: the union over the tile's rows of their k selected blocks, each row
+//      masked to its own k blocks (a row's valid keys are k ranges of the union stream).
+//   W  the tile's window key union (Chebyshev radius r), masked by distance.
+// out = g0 o_cmp + g1 o_sel + g2 o_win is assembled in an fp32 row buffer and written in the
+// input type after phase W.
+//
+// Warp roles (192 threads):
+//   warp 0    producer: K and V tiles into two-stage shared-memory rings by TMA: tiled loads for
+//             the compressed tokens, row gathers (tile::gather4) for the selected and window keys;
+//             the window keys' coordinates;
+//   warp 1    MMA issuer (one thread): S = Q K^T into one of two TMEM buffers; O += P V with P
+//             read from TMEM (it overwrites S in place);
+//   warps 2-5 softmax, one thread per row (its TMEM lane): S into registers once, mask, running
+//             max with a lazy rescale (O and the row sum are rescaled only when the max grows by
+//             more than 2^8), P = 2^(s - m) rounded to the input type back into TMEM.
+// The tensor core computes S of tile j+1 while the softmax works on tile j. Between phases C and S
+// the softmax warps build the union of the selected blocks in shared memory (a bitmap over the
+// sequence's blocks, aliasing the idle K/V rings) and each row's key ranges.
+// Every wait is bounded; a wait that runs out records DEV_TIMEOUT and the CTA winds down.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "attn_common.cuh"
+
+namespace ssa {
+
+namespace {
+
+using namespace attn;
+
+constexpr int kKT = 64;          // keys per tile
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;   // S/P buffers at columns 0 and 64, O at 128
+
+template <int D, int KM>
+struct FL {
+    static constexpr uint32_t kCh = D / 32;              // 32-element column chunks
+    static constexpr uint32_t kQReg = 128 * 64;          // one chunk of the 128-row Q tile
+    static constexpr uint32_t kKVReg = kKT * 64;         // one chunk of a 64-row K or V tile
+    static constexpr uint32_t kTile = kCh * kKVReg;      // one K or V stage
+    static constexpr uint32_t kSlots = KM + 1;           // selected blocks per row (bound)
+    static constexpr uint32_t kUCap = 128 * kSlots;      // union capacity in blocks
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kK = kQ + kCh * kQReg;
+    static constexpr uint32_t kV = kK + 2 * kTile;
+    static constexpr uint32_t kMeta = kV + 2 * kTile;    // int4 [2][64] window key coordinates
+    static constexpr uint32_t kUnion = kMeta + 2 * kKT * 16;   // int2 [kUCap+1] (first row, stream offset)
+    static constexpr uint32_t kRange = kUnion + (kUCap + 1) * 8;   // int2 [kSlots][128] key ranges
+    static constexpr uint32_t kBar = kRange + kSlots * 128 * 8;
+    static constexpr uint32_t kMisc = kBar + 16 * 8;
+    static constexpr uint32_t kBytes = kMisc + 64;
+    static constexpr uint32_t kAlloc = kBytes + 1024;
+    // the union build's bitmap and word prefix alias the two K and two V stages
+    static constexpr uint32_t kScratchWords = (4 * kTile) / 8;
+    static constexpr int64_t kMaxSeqBlocks = 32 * (int64_t)kScratchWords;
+    static constexpr int kMinBlocks = kAlloc <= 113u * 1024u ? 2 : 1;
+};
+
+enum : int { KFULL = 0, KEMPTY = 2, VFULL = 4, PVD = 6, SFULL = 8, PFULL = 10, FIN = 12, NBAR = 13 };
+// misc words
+enum : int { M_TMEM = 0, M_ABORT = 1, M_U = 2, M_L = 3, M_RED = 4 };
+
+__device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int32_t* status,
+                                             volatile int* abort_flag) {
+    if (*abort_flag) return false;
+    if (tc::mbar_wait(bar, parity, kWaitCycles)) return true;
+    atomicOr(status, DEV_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+}
+
+// v[e] for a per-thread index e in [0, 16), by a tree of selects (stays in registers)
+__device__ __forceinline__ float pick16(const float* v, int e) {
+    float a[8], b[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) b[i] = (e & 2) ? a[2 * i + 1] : a[2 * i];
+    const float c0 = (e & 4) ? b[1] : b[0];
+    const float c1 = (e & 4) ? b[3] : b[2];
+    return (e & 8) ? c1 : c0;
+}
+
+// Bits [a, b) of a 64-bit word, a and b clamped to [0, 64].
+__device__ __forceinline__ uint64_t span_bits(int a, int b) {
+    a = max(a, 0);
+    b = min(b, 64);
+    if (a >= b) return 0ull;
+    const uint64_t hi = b >= 64 ? ~0ull : ((1ull << b) - 1ull);
+    return hi & (~0ull << a);
+}
+
+// Exclusive prefix sum over the 128 softmax threads (local index t); `red` holds 4 ints.
+__device__ __forceinline__ int scan128(int v, int t, int* red, int& total) {
+    const int lane = t & 31, w = t >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) red[w] = x;
+    tc::named_sync(2, 128);
+    int pre = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = red[i];
+        pre += i < w ? r : 0;
+        tot += r;
+    }
+    tc::named_sync(2, 128);
+    total = tot;
+    return pre + x - v;
+}
+
+template <typename T, int D, int KM>
+__global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
+    k_ssa_fwd(const __grid_constant__ FwdParams P, const __grid_constant__ CUtensorMap tm_kc,
+              const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kg,
+              const __grid_constant__ CUtensorMap tm_vg) {
+    using L = FL<D, KM>;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* g = align1024(smem_raw);
+    const uint32_t sb = tc::smem_u32(g);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(g + L::kBar);
+    int* misc = reinterpret_cast<int*>(g + L::kMisc);
+    volatile int* abort_flag = misc + M_ABORT;
+    int4* meta = reinterpret_cast<int4*>(g + L::kMeta);
+    int2* un = reinterpret_cast<int2*>(g + L::kUnion);
+    int2* rng = reinterpret_cast<int2*>(g + L::kRange);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tile = blockIdx.x, h = blockIdx.y, H = P.H;
+
+    // ---- per-CTA schedule --------------------------------------------------------------------
+    const int32_t p0 = P.qt_pos[tile], len = P.qt_len[tile], seq = P.qt_seq[tile];
+    const int32_t bl = P.seq_blk[seq], nblk = P.seq_blk[seq + 1] - bl;
+    const int32_t w0 = P.wt_off[tile], nwin = P.wt_off[tile + 1] - w0;
+    const int nc = (nblk + kKT - 1) / kKT;
+    const int nw = (nwin + kKT - 1) / kKT;
+
+    // ---- setup: TMEM, barriers, Q tile -------------------------------------------------------
+    if (warp == 1) {
+        tc::tmem_alloc(reinterpret_cast<uint32_t*>(misc + M_TMEM), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], (i == PFULL || i == PFULL + 1) ? 4u : 1u);
+        misc[M_ABORT] = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&tm_kc);
+        tc::tma_prefetch_desc(&tm_vc);
+        tc::tma_prefetch_desc(&tm_kg);
+        tc::tma_prefetch_desc(&tm_vg);
+    }
+    const T* Q = reinterpret_cast<const T*>(P.q);
+    for (int e = tid; e < 128 * (D / 8); e += kThreads) {
+        const int row = e / (D / 8), c16 = e % (D / 8);
+        const bool ok = row < len;
+        const T* src = ok ? Q + ((int64_t)P.perm[p0 + row] * H + h) * D + c16 * 8 : Q;
+        tc::cp_async16(sb + L::kQ + (c16 >> 2) * L::kQReg + tc::sw64(row, c16 & 3), src, ok ? 16u : 0u);
+    }
+    tc::cp_async_wait_all();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = (uint32_t)misc[M_TMEM];
+
+    if (warp == 0) {
+        // ================================ producer ============================================
+        const int32_t pad_row = (int32_t)(h * P.Npad);   // a valid row; its keys are masked
+        int U = 0, Ltot = 0, ns = 0;
+        // rows (K/V row index in the [H * Npad, D] tensors) of keys `lane` and `lane + 32` of tile t
+        auto rows_of = [&](int ph, int t, int32_t& r0, int32_t& r1) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int i = lane + 32 * half;
+                int32_t row = pad_row;
+                if (ph == 1) {
+                    const int key = kKT * t + i;
+                    if (key < Ltot) {
+                        int lo = 0, hi = U - 1;   // last union block whose stream offset <= key
+                        while (lo < hi) {
+                            const int mid = (lo + hi + 1) >> 1;
+                            if (un[mid].y <= key) lo = mid; else hi = mid - 1;
+                        }
+                        row = pad_row + un[lo].x + (key - un[lo].y);
+                    }
+                } else {
+                    if (kKT * t + i < nwin) row = pad_row + P.wt_keys[w0 + kKT * t + i];
+                }
+                if (half == 0) r0 = row; else r1 = row;
+            }
+        };
+        auto gather = [&](const CUtensorMap* tm, uint32_t dst, uint64_t* fb, int32_t r0, int32_t r1) {
+            if (lane == 0) tc::mbar_arrive_expect_tx(fb, L::kTile);
+            __syncwarp();
+            int32_t y[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int src = (4 * lane + q) & 31;
+                const int32_t a = __shfl_sync(0xffffffffu, r0, src);
+                const int32_t b = __shfl_sync(0xffffffffu, r1, src);
+                y[q] = lane < 8 ? a : b;
+            }
+            if (lane < 16) {
+#pragma unroll
+                for (int c = 0; c < (int)L::kCh; ++c)
+                    tc::tma_gather4(dst + c * L::kKVReg + lane * 256, tm, 32 * c, y[0], y[1], y[2], y[3], fb);
+            }
+        };
+        auto produce = [&](int j, int ph, int t) -> bool {
+            const int s = j & 1;
+            const uint32_t par_e = (uint32_t)((j >> 1) - 1) & 1u;
+            const uint32_t kdst = sb + L::kK + s * L::kTile;
+            const uint32_t vdst = sb + L::kV + s * L::kTile;
+            int32_t r0 = 0, r1 = 0;
+            if (ph > 0) rows_of(ph, t, r0, r1);
+            if (j >= 2 && !wait_or_flag(&bar[KEMPTY + s], par_e, P.status, abort_flag)) return false;
+            if (ph == 0) {
+                if (lane == 0) {
+                    const int32_t y = (int32_t)(h * P.Mb + bl + kKT * t);
+                    tc::mbar_arrive_expect_tx(&bar[KFULL + s], L::kTile);
+                    for (int c = 0; c < (int)L::kCh; ++c)
+                        tc::tma_load_2d(kdst + c * L::kKVReg, &tm_kc, 32 * c, y, &bar[KFULL + s]);
+                }
+            } else {
+                gather(&tm_kg, kdst, &bar[KFULL + s], r0, r1);
+            }
+            // V stage and the key coordinates are free once P V of tile j-2 completed
+            if (j >= 2 && !wait_or_flag(&bar[PVD + s], par_e, P.status, abort_flag)) return false;
+            if (ph == 0) {
+                if (lane == 0) {
+                    const int32_t y = (int32_t)(h * P.Mb + bl + kKT * t);
+                    tc::mbar_arrive_expect_tx(&bar[VFULL + s], L::kTile);
+                    for (int c = 0; c < (int)L::kCh; ++c)
+                        tc::tma_load_2d(vdst + c * L::kKVReg, &tm_vc, 32 * c, y, &bar[VFULL + s]);
+                }
+            } else {
+                if (ph == 2) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int i = lane + 32 * half;
+                        int4 mc = make_int4(1 << 28, 1 << 28, 1 << 28, -1);
+                        if (kKT * t + i < nwin) mc = P.scoord[P.wt_keys[w0 + kKT * t + i]];
+                        meta[s * kKT + i] = mc;
+                    }
+                }
+                gather(&tm_vg, vdst, &bar[VFULL + s], r0, r1);   // its __syncwarp orders meta
+            }
+            return true;
+        };
+        bool ok = true;
+        for (int j = 0; j < nc && ok; ++j) ok = produce(j, 0, j);
+        __syncwarp();
+        tc::named_sync(1, kThreads);   // union of the selected blocks is built
+        U = misc[M_U];
+        Ltot = misc[M_L];
+        ns = (Ltot + kKT - 1) / kKT;
+        for (int j = nc; j < nc + ns + nw && ok && !*abort_flag; ++j)
+            ok = j < nc + ns ? produce(j, 1, j - nc) : produce(j, 2, j - nc - ns);
+    } else if (warp == 1) {
+        // ================================ MMA issuer ==========================================
+        const uint32_t idesc_s = tc::idesc_f16(kBf16, 128, kKT, false);
+        const uint32_t idesc_o = tc::idesc_f16(kBf16, 128, D, true);
+        auto mma_s = [&](int j) -> bool {
+            const int b = j & 1;
+            if (!wait_or_flag(&bar[KFULL + b], (uint32_t)(j >> 1) & 1u, P.status, abort_flag)) return false;
+            // TMEM buffer b holds P of tile j-2 until P V of that tile completed
+            if (j >= 2 && !wait_or_flag(&bar[PVD + b], (uint32_t)((j >> 1) - 1) & 1u, P.status, abort_flag))
+                return false;
+            tc::fence_after_sync();
+            const uint32_t kbase = sb + L::kK + b * L::kTile;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                tc::mma_f16_ss(tmem + b * kKT, tc::desc_kmajor_r(sb + L::kQ, kk, L::kQReg),
+                               tc::desc_kmajor_r(kbase, kk, L::kKVReg), idesc_s, kk > 0 ? 1u : 0u);
+            tc::mma_commit(&bar[SFULL + b]);
+            tc::mma_commit(&bar[KEMPTY + b]);
+            return true;
+        };
+        auto mma_pv = [&](int i, bool first) -> bool {
+            const int b = i & 1;
+            if (!wait_or_flag(&bar[PFULL + b], (uint32_t)(i >> 1) & 1u, P.status, abort_flag)) return false;
+            if (!wait_or_flag(&bar[VFULL + b], (uint32_t)(i >> 1) & 1u, P.status, abort_flag)) return false;
+            tc::fence_after_sync();
+            const uint32_t vbase = sb + L::kV + b * L::kTile;
+#pragma unroll
+            for (int kk = 0; kk < kKT / 16; ++kk)
+                tc::mma_f16_ts(tmem + 128, tmem + b * kKT + kk * 8,
+                               tc::desc_mnmajor_r(vbase, kk, L::kKVReg), idesc_o,
+                               (first && kk == 0) ? 0u : 1u);
+            tc::mma_commit(&bar[PVD + b]);   // P V of tile i done: V stage, P buffer, O
+            return true;
+        };
+        if (lane == 0) {
+            bool ok = true;
+            for (int j = 0; j < nc && ok; ++j) {
+                ok = mma_s(j);
+                if (ok && j >= 1) ok = mma_pv(j - 1, j - 1 == 0);
+            }
+            if (ok) mma_pv(nc - 1, nc == 1);
+        }
+        __syncwarp();
+        tc::named_sync(1, kThreads);
+        const int ns = (misc[M_L] + kKT - 1) / kKT;
+        const int nT = nc + ns + nw;
+        if (lane == 0) {
+            bool ok = !*abort_flag;
+            for (int j = nc; j < nT && ok; ++j) {
+                ok = mma_s(j);
+                if (ok && j > nc) ok = mma_pv(j - 1, j - 1 == nc || j - 1 == nc + ns);
+            }
+            if (ok && nT > nc) ok = mma_pv(nT - 1, nT - 1 == nc || nT - 1 == nc + ns);
+            // drain the tensor pipe before TMEM is released
+            tc::mma_commit(&bar[FIN]);
+            tc::mbar_wait(&bar[FIN], 0u, kWaitCycles);
+        }
+        __syncwarp();
+    } else {
+        // ================================ softmax =============================================
+        const int t128 = tid - 64;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t o_tm = tmem + lane_base + 128;
+        const bool row_ok = row < len;
+        const int32_t pos = p0 + (row_ok ? row : len - 1);
+        const int32_t tok = P.perm[pos];
+        const int32_t ob = P.tok_blk[tok];
+        const int4 qc = P.scoord[P.blk_poff[ob] + (pos - P.blk_off[ob])];
+        const float* gt = P.gates + ((int64_t)tok * H + h) * 3;
+        float* brow = P.base + ((int64_t)pos * H + h) * D;
+        const int rr = P.r;
+        const float sl = P.sl;
+        const int ksel = P.k;
+        float m = -INFINITY, l = 0.0f;
+        int pv_seen = 0;   // P V completions observed, in order (waits never skip a phase)
+        auto wait_pv = [&](int i) -> bool {
+            while (pv_seen <= i) {
+                if (!wait_or_flag(&bar[PVD + (pv_seen & 1)], (uint32_t)(pv_seen >> 1) & 1u, P.status, abort_flag))
+                    return false;
+                ++pv_seen;
+            }
+            return true;
+        };
+        // O of the finished phase -> its destination (warp-collective TMEM reads)
+        auto epilogue = [&](int ph) {
+            tc::fence_after_sync();
+            const float f = row_ok ? gt[ph] / l : 0.0f;
+#pragma unroll 1
+            for (int d0 = 0; d0 < D; d0 += 32) {
+                float o[32];
+                tc::tmem_ld32(o_tm + d0, o);
+                if (!row_ok) continue;
+                if (ph < 2) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        float4 v = make_float4(o[e] * f, o[e + 1] * f, o[e + 2] * f, o[e + 3] * f);
+                        if (ph == 1) {
+                            const float4 bb = *reinterpret_cast<const float4*>(brow + d0 + e);
+                            v.x += bb.x; v.y += bb.y; v.z += bb.z; v.w += bb.w;
+                        }
+                        *reinterpret_cast<float4*>(brow + d0 + e) = v;
+                    }
+                } else {
+                    T* orow = reinterpret_cast<T*>(P.out) + ((int64_t)tok * H + h) * D + d0;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        const float4 b0 = *reinterpret_cast<const float4*>(brow + d0 + e);
+                        const float4 b1 = *reinterpret_cast<const float4*>(brow + d0 + e + 4);
+                        *reinterpret_cast<uint4*>(orow + e) = make_uint4(
+                            pack2<T>(b0.x + o[e] * f, b0.y + o[e + 1] * f),
+                            pack2<T>(b0.z + o[e + 2] * f, b0.w + o[e + 3] * f),
+                            pack2<T>(b1.x + o[e + 4] * f, b1.y + o[e + 5] * f),
+                            pack2<T>(b1.z + o[e + 6] * f, b1.w + o[e + 7] * f));
+                    }
+                }
+            }
+        };
+        // one tile: S from TMEM buffer b, masked by `mask(s)`, then softmax bookkeeping, P to TMEM
+        auto step = [&](int j, bool first, auto&& mask) -> bool {
+            const int b = j & 1;
+            if (!wait_or_flag(&bar[SFULL + b], (uint32_t)(j >> 1) & 1u, P.status, abort_flag)) return false;
+            // Observe P V of tile j-2 (already complete: S of tile j was issued after it). Keeping
+            // the observed count within one phase of the barriers keeps later parity waits exact.
+            if (j >= 2 && !wait_pv(j - 2)) return false;
+            tc::fence_after_sync();
+            const uint32_t s_tm = tmem + lane_base + b * kKT;
+            float s[64];
+            tc::tmem_ld64(s_tm, s);
+            if (!mask(s)) return false;
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[i], s[i + 8]);
+#pragma unroll
+            for (int e = 16; e < 64; e += 8) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[e + i]);
+            }
+            const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float tm = tmax * sl;
+            bool resc = false;
+            float alpha = 1.0f;
+            if (tm > m + 8.0f) {
+                const bool had = m != -INFINITY;
+                alpha = had ? tc::ex2(m - tm) : 0.0f;
+                resc = had && !first;
+                l *= alpha;
+                m = tm;
+            }
+            if (__any_sync(0xffffffffu, resc)) {
+                // O must hold P V of the previous tile before it is rescaled
+                if (!wait_pv(j - 1)) return false;
+                tc::fence_after_sync();
+                const float f = resc ? alpha : 1.0f;
+#pragma unroll 1
+                for (int d0 = 0; d0 < D; d0 += 32) {
+                    float o[32];
+                    tc::tmem_ld32(o_tm + d0, o);
+                    uint32_t ob32[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ob32[e] = __float_as_uint(o[e] * f);
+                    tc::tmem_st32(o_tm + d0, ob32);
+                }
+            }
+            const float mu = m == -INFINITY ? 0.0f : m;
+            uint32_t pk[32];
+            float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float a0 = tc::ex2(fmaf(s[2 * i], sl, -mu));
+                const float a1 = tc::ex2(fmaf(s[2 * i + 1], sl, -mu));
+                pk[i] = pack2<T>(a0, a1);
+                // bf16 weights: the row sum uses the rounded weights the MMA multiplies V with
+                if (kBf16) ls[i & 3] += unpack_lo<T>(pk[i]) + unpack_hi<T>(pk[i]);
+                else ls[i & 3] += a0 + a1;
+            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            tc::tmem_st32(s_tm, pk);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bar[PFULL + b]);
+            return true;
+        };
+
+        // ---- phase C: compressed tokens + top-(k-1) of the other blocks ----------------------
+        float tv[KM];
+        int32_t ti[KM];
+#pragma unroll
+        for (int u = 0; u < KM; ++u) {
+            tv[u] = -INFINITY;
+            ti[u] = -1;
+        }
+        bool ok = true;
+        for (int j = 0; j < nc && ok; ++j) {
+            const int lim = nblk - kKT * j;
+            const int32_t bbase = bl + kKT * j;
+            ok = step(j, j == 0, [&](float (&s)[64]) -> bool {
+                if (lim < kKT) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        if (e >= lim) s[e] = -INFINITY;
+                }
+                if (ksel > 1) {
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq) {
+                        const float thr = tv[KM - 1];
+                        uint32_t cand = 0;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) cand |= (uint32_t)(s[16 * gq + e] > thr) << e;
+                        while (cand) {
+                            const int e = __ffs(cand) - 1;
+                            cand &= cand - 1;
+                            const int32_t bi = bbase + 16 * gq + e;
+                            if (bi != ob) topk_push<KM>(tv, ti, pick16(s + 16 * gq, e), bi);
+                        }
+                    }
+                }
+                return true;
+            });
+        }
+        if (ok) ok = wait_pv(nc - 1);
+        if (ok) {
+            epilogue(0);
+            if (row_ok) {
+                int32_t* srow = P.sel + ((int64_t)pos * H + h) * ksel;
+                srow[0] = ob;
+#pragma unroll
+                for (int u = 0; u < KM; ++u)
+                    if (u + 1 < ksel) srow[u + 1] = ti[u];
+            }
+        }
+
+        // ---- union of the selected blocks and each row's key ranges ---------------------------
+        {
+            uint32_t* words = reinterpret_cast<uint32_t*>(g + L::kK);
+            const int W = (nblk + 31) >> 5;
+            int32_t* wpre = reinterpret_cast<int32_t*>(words + W);
+            int* red = misc + M_RED;
+            for (int i = t128; i < W; i += 128) words[i] = 0u;
+            tc::named_sync(2, 128);
+            // own block, then the top-(k-1) (local block indices; -1 = none)
+            int32_t mine[L::kSlots];
+            mine[0] = row_ok ? ob - bl : -1;
+#pragma unroll
+            for (int u = 0; u < KM; ++u)
+                mine[u + 1] = (row_ok && u + 1 < ksel && ti[u] >= 0) ? ti[u] - bl : -1;
+#pragma unroll
+            for (int a = 0; a < (int)L::kSlots; ++a)
+                if (mine[a] >= 0 && mine[a] < nblk) atomicOr(&words[mine[a] >> 5], 1u << (mine[a] & 31));
+            tc::named_sync(2, 128);
+            // union index of every set bit: exclusive prefix of the word popcounts
+            const int cw = (W + 127) >> 7;
+            const int wl = min(t128 * cw, W), wh = min(wl + cw, W);
+            int cnt = 0;
+            for (int i = wl; i < wh; ++i) cnt += __popc(words[i]);
+            int U = 0;
+            int pre = scan128(cnt, t128, red, U);
+            U = min(U, (int)L::kUCap);
+            for (int i = wl; i < wh; ++i) {
+                wpre[i] = pre;
+                uint32_t wd = words[i];
+                while (wd) {
+                    const int bit = __ffs(wd) - 1;
+                    wd &= wd - 1;
+                    const int32_t gb = bl + 32 * i + bit;
+                    if (pre < (int)L::kUCap)
+                        un[pre] = make_int2(P.blk_poff[gb], P.blk_off[gb + 1] - P.blk_off[gb]);
+                    ++pre;
+                }
+            }
+            tc::named_sync(2, 128);
+            // stream offsets: exclusive prefix of the block sizes
+            const int cu = (U + 127) >> 7;
+            const int ul = min(t128 * cu, U), uh = min(ul + cu, U);
+            int ssum = 0;
+            for (int u = ul; u < uh; ++u) ssum += un[u].y;
+            int Ltot = 0;
+            int off = scan128(ssum, t128, red, Ltot);
+            for (int u = ul; u < uh; ++u) {
+                const int n = un[u].y;
+                un[u].y = off;
+                off += n;
+            }
+            if (t128 == 0) {
+                un[U] = make_int2(0, Ltot);
+                misc[M_U] = U;
+                misc[M_L] = Ltot;
+            }
+            tc::named_sync(2, 128);
+            // this row's ranges, ascending (the union stream is in block order)
+#pragma unroll
+            for (int a = 0; a < (int)L::kSlots; ++a) {
+                if (mine[a] < 0 || mine[a] >= nblk) continue;
+                int rank = 0;
+#pragma unroll
+                for (int c = 0; c < (int)L::kSlots; ++c) rank += (mine[c] >= 0 && mine[c] < mine[a]) ? 1 : 0;
+                const int wi = mine[a] >> 5;
+                const int u = wpre[wi] + __popc(words[wi] & ((1u << (mine[a] & 31)) - 1u));
+                if (u < U) rng[rank * 128 + row] = make_int2(un[u].y, un[u + 1].y);
+            }
+        }
+        int nr = 0;
+#pragma unroll
+        for (int u = 0; u < KM; ++u) nr += (row_ok && u + 1 < ksel && ti[u] >= 0) ? 1 : 0;
+        nr += row_ok ? 1 : 0;
+        tc::named_sync(1, kThreads);   // the producer may now overwrite the rings
+        const int ns = (misc[M_L] + kKT - 1) / kKT;
+        const int nT = nc + ns + nw;
+
+        // ---- phase S: the selected blocks ------------------------------------------------------
+        m = -INFINITY;
+        l = 0.0f;
+        int ri = 0;
+        for (int j = nc; j < nc + ns && ok; ++j) {
+            const int base = kKT * (j - nc);
+            ok = step(j, j == nc, [&](float (&s)[64]) -> bool {
+                uint64_t vm = 0;
+                while (ri < nr) {
+                    const int2 rg = rng[ri * 128 + row];
+                    if (rg.x >= base + kKT) break;
+                    vm |= span_bits(rg.x - base, rg.y - base);
+                    if (rg.y > base + kKT) break;
+                    ++ri;
+                }
+                const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    if (!((lo >> e) & 1u)) s[e] = -INFINITY;
+                    if (!((hi >> e) & 1u)) s[e + 32] = -INFINITY;
+                }
+                return true;
+            });
+        }
+        if (ok && ns > 0 && (ok = wait_pv(nc + ns - 1))) epilogue(1);
+
+        // ---- phase W: the window ---------------------------------------------------------------
+        m = -INFINITY;
+        l = 0.0f;
+        for (int j = nc + ns; j < nT && ok; ++j) {
+            const int b = j & 1;
+            ok = step(j, j == nc + ns, [&](float (&s)[64]) -> bool {
+                // the key coordinates travel with the V stage
+                if (!wait_or_flag(&bar[VFULL + b], (uint32_t)(j >> 1) & 1u, P.status, abort_flag)) return false;
+                const int4* km = meta + b * kKT;
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    const int4 kc = km[e];
+                    const int dd = max(abs(kc.x - qc.x), max(abs(kc.y - qc.y), abs(kc.z - qc.z)));
+                    if (dd > rr) s[e] = -INFINITY;
+                }
+                return true;
+            });
+        }
+        if (ok && nT > nc + ns && wait_pv(nT - 1)) epilogue(2);
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---- selection export -------------------------------------------------------------------------
+__global__ void k_export_sel(const int32_t* __restrict__ sel, const int32_t* __restrict__ tok_pos,
+                             int64_t N, int H, int k, int32_t* __restrict__ out) {
+    int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per_tok = (int64_t)H * k;
+    if (e >= N * per_tok) return;
+    const int64_t tok = e / per_tok, rest = e % per_tok;
+    out[e] = sel[(int64_t)tok_pos[tok] * per_tok + rest];
+}
+
+// ---- host: tensor maps and launch ----------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)f;
+    }
+    return fn;
+}
+
+// rows x D matrix of 16-bit elements, boxes of 32 columns x `box_rows` rows, 64-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int D, bool bf16, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {32, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int KM>
+ssa_status_t run(const Plan* p, const FwdParams& P, const CUtensorMap* tm, int64_t max_seq_blocks,
+                 cudaStream_t st) {
+    using L = FL<D, KM>;
+    static_assert(L::kAlloc <= 227u * 1024u, "shared-memory layout exceeds the per-CTA limit");
+    if (max_seq_blocks > L::kMaxSeqBlocks) return SSA_ERR_UNSUPPORTED;
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(k_ssa_fwd<T, D, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)L::kAlloc) != cudaSuccess)
+            return SSA_ERR_CUDA;
+        configured = true;
+    }
+    k_ssa_fwd<T, D, KM><<<dim3((unsigned)p->n_qtiles, (unsigned)P.H), kThreads, L::kAlloc, st>>>(
+        P, tm[0], tm[1], tm[2], tm[3]);
+    note_launch();
+    return cudaPeekAtLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+template <typename T, int D>
+ssa_status_t run_km(const Plan* p, const FwdParams& P, const CUtensorMap* tm, int64_t mb, cudaStream_t st) {
+    if (P.k - 1 <= 8) return run<T, D, 8>(p, P, tm, mb, st);
+    if (P.k - 1 <= 16) return run<T, D, 16>(p, P, tm, mb, st);
+    return run<T, D, 32>(p, P, tm, mb, st);
+}
+
+template <typename T>
+ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, const CUtensorMap* tm, int64_t mb, cudaStream_t st) {
+    switch (D) {
+    case 32: return run_km<T, 32>(p, P, tm, mb, st);
+    case 64: return run_km<T, 64>(p, P, tm, mb, st);
+    case 96: return run_km<T, 96>(p, P, tm, mb, st);
+    default: return run_km<T, 128>(p, P, tm, mb, st);
+    }
+}
+
+}  // namespace
+
+ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
+                               void* out, cudaStream_t st) {
+    const bool bf16 = w.dtype == SSA_BF16;
+    CUtensorMap tm[4];
+    if (!make_map(&tm[0], w.kc, (int64_t)w.H * p->Mb, w.D, bf16, kKT) ||
+        !make_map(&tm[1], w.vc, (int64_t)w.H * p->Mb, w.D, bf16, kKT) ||
+        !make_map(&tm[2], w.ks, (int64_t)w.H * p->Npad, w.D, bf16, 1) ||
+        !make_map(&tm[3], w.vs, (int64_t)w.H * p->Npad, w.D, bf16, 1))
+        return SSA_ERR_CUDA;
+    int64_t max_seq_blocks = 0;
+    for (size_t s = 0; s + 1 < p->seq_blk.size(); ++s)
+        max_seq_blocks = std::max<int64_t>(max_seq_blocks, p->seq_blk[s + 1] - p->seq_blk[s]);
+    FwdParams P;
+    P.q = q;
+    P.ks = w.ks;
+    P.vs = w.vs;
+    P.kc = w.kc;
+    P.vc = w.vc;
+    P.gates = gates;
+    P.perm = p->perm;
+    P.tok_blk = p->tok_blk;
+    P.blk_off = p->blk_off;
+    P.blk_poff = p->blk_poff;
+    P.scoord = p->scoord;
+    P.qt_pos = p->qt_pos;
+    P.qt_len = p->qt_len;
+    P.qt_seq = p->qt_seq;
+    P.seq_blk = p->seq_blk_d;
+    P.wt_off = p->wt_off;
+    P.wt_keys = p->wt_keys;
+    P.sel = w.sel;
+    P.base = w.base;
+    P.out = out;
+    P.status = p->d_status;
+    P.N = p->N;
+    P.Npad = p->Npad;
+    P.Mb = p->Mb;
+    P.H = w.H;
+    P.k = w.k;
+    P.r = p->r;
+    P.sl = (float)(1.4426950408889634 / sqrt((double)w.D));
+    ProfScope ps("k_ssa_fwd", st);
+    if (bf16) return run_d<__nv_bfloat16>(p, P, w.D, tm, max_seq_blocks, st);
+    return run_d<__half>(p, P, w.D, tm, max_seq_blocks, st);
+}
+
+void launch_export_sel(const Plan* p, const Workspace& w, int32_t* sel_out, cudaStream_t st) {
+    const int64_t n = p->N * w.H * w.k;
+    k_export_sel<<<(unsigned)cdiv(n, 256), 256, 0, st>>>(w.sel, p->tok_pos, p->N, w.H, w.k, sel_out);
+    note_launch();
+}
+
+}  // namespace ssa

@@ -44,18 +44,8 @@ struct Workspace {
     void* vs = nullptr;        // [H, Npad, D] T
     void* kc = nullptr;        // [H, Mb, D]   T (fp32 for the fp32 path)
     void* vc = nullptr;        // [H, Mb, D]
-    float* base = nullptr;     // [N, H, D]    g0*o_cmp + g2*o_win, sorted token order
-    void* part_o = nullptr;    // [N, H, k, D] T   per-(query, head, slot) normalised partial output
-    float* part_lse = nullptr; // [N, H, k]        log2-sum-exp of each partial
+    float* base = nullptr;     // [N, H, D]    running g0*o_cmp + g1*o_sel, sorted token order
     int32_t* sel = nullptr;    // [N, H, k]        selected blocks, sorted token order
-    int32_t* inv_cnt = nullptr;  // [H*Mb + 1]
-    int32_t* inv_off = nullptr;  // [H*Mb + 1]
-    int32_t* inv_fill = nullptr; // [H*Mb]
-    int32_t* inv_list = nullptr; // [N*H*(k-1)]  (sorted query position << 5 | slot)
-    int32_t* item_cnt = nullptr; // [H*Mb + 1]   tiles per (head, block)
-    int32_t* item_off = nullptr; // [H*Mb + 1]
-    int32_t* scan_tmp = nullptr;
-    int64_t scan_tmp_len = 0;
     // host-buffer entry point staging (allocated on first use)
     void* h_q = nullptr; void* h_k = nullptr; void* h_v = nullptr; void* h_out = nullptr;
     float* h_gates = nullptr; float* h_wc = nullptr;
@@ -155,16 +145,16 @@ void launch_pool(const Plan* p, const Workspace& w, const void* k, const void* v
 void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const void* k,
                          const void* v, const float* gates, void* out, cudaStream_t s);
 
-// attn_tc.cu (bf16 / fp16 path)
-bool launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
-                       void* out, cudaStream_t s);
+// attn_fwd.cu (bf16 / fp16 path): the fused tensor-core forward
+ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
+                               void* out, cudaStream_t s);
 
 // backward.cu
 ssa_status_t launch_backward(Plan* p, const Workspace& w, const void* q, const void* k,
                              const void* v, const float* gates, const float* wc, const void* dout,
                              void* dq, void* dk, void* dv, cudaStream_t s);
 
-// selection export (attn_tc.cu): sel_out [N,H,k] in token order from the sorted-order buffer.
+// selection export (attn_fwd.cu): sel_out [N,H,k] in token order from the sorted-order buffer.
 void launch_export_sel(const Plan* p, const Workspace& w, int32_t* sel_out, cudaStream_t s);
 
 // ---- small device helpers -------------------------------------------------------------------

@@ -224,13 +224,18 @@ ssa_status_t ensure_workspace(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int
     w.sel = (int32_t*)A(sizeof(int32_t) * N * H * k);
     if (!w.kc || !w.vc || !w.sel) return SSA_ERR_ALLOC;
     if (dt != SSA_F32) {
+        w.Mb8 = round_up(Mb, 8);
         w.ks = A(es * H * p->Npad * D);
         w.vs = A(es * H * p->Npad * D);
+        w.kcg = A(es * H * w.Mb8 * D);
+        w.vcg = A(es * H * w.Mb8 * D);
         w.base = (float*)A(sizeof(float) * N * H * D);
-        if (!w.ks || !w.vs || !w.base) return SSA_ERR_ALLOC;
+        if (!w.ks || !w.vs || !w.kcg || !w.vcg || !w.base) return SSA_ERR_ALLOC;
         // padding rows of the block-ordered copies stay zero for the life of the workspace
         if (cudaMemsetAsync(w.ks, 0, es * H * p->Npad * D, st) ||
-            cudaMemsetAsync(w.vs, 0, es * H * p->Npad * D, st))
+            cudaMemsetAsync(w.vs, 0, es * H * p->Npad * D, st) ||
+            cudaMemsetAsync(w.kcg, 0, es * H * w.Mb8 * D, st) ||
+            cudaMemsetAsync(w.vcg, 0, es * H * w.Mb8 * D, st))
             return SSA_ERR_CUDA;
     }
     w.H = H;

@@ -14,10 +14,10 @@ constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz
 
 struct FwdParams {
     const void* q;
-    const void* ks;
+    const void* ks;    // grouped order, [H, Npad, D]
     const void* vs;
-    const void* kc;
-    const void* vc;
+    const void* kcg;   // grouped order, [H, Mb8, D]
+    const void* vcg;
     const float* gates;
     const int32_t* perm;
     const int32_t* tok_blk;
@@ -28,13 +28,16 @@ struct FwdParams {
     const int32_t* qt_len;
     const int32_t* qt_seq;
     const int32_t* seq_blk;
-    const int32_t* wt_off;
-    const int32_t* wt_keys;
+    const int32_t* wr_off;
+    const int2* wr_runs;
+    const int32_t* wg_cnt;
+    const int32_t* wm_off;
+    const uint64_t* wmask;
     int32_t* sel;
     float* base;
     void* out;
     int32_t* status;
-    int64_t N, Npad, Mb;
+    int64_t N, Npad, Mb, Mb8;
     int H, k, r;
     float sl;   // softmax scale * log2(e)
 };

@@ -14,9 +14,11 @@
 // input type after phase W.
 //
 // Warp roles (192 threads):
-//   warp 0    producer: K and V tiles into two-stage shared-memory rings by TMA: tiled loads for
-//             the compressed tokens, row gathers (tile::gather4) for the selected and window keys;
-//             the window keys' coordinates;
+//   warp 0    producer: K and V tiles into two-stage shared-memory rings by 1D bulk copies. The
+//             K/V copies in global memory are stored as 8-row groups already in the tensor cores'
+//             swizzled operand order, so a run of consecutive groups is one copy: the compressed
+//             tokens are one run, each selected block is one run, and the window union is the
+//             plan's list of runs (with the keys' coordinates);
 //   warp 1    MMA issuer (one thread): S = Q K^T into one of two TMEM buffers; O += P V with P
 //             read from TMEM (it overwrites S in place);
 //   warps 2-5 softmax, one thread per row (its TMEM lane): S into registers once, mask, running
@@ -26,8 +28,6 @@
 // the softmax warps build the union of the selected blocks in shared memory (a bitmap over the
 // sequence's blocks, aliasing the idle K/V rings) and each row's key ranges.
 // Every wait is bounded; a wait that runs out records DEV_TIMEOUT and the CTA winds down.
-#include <cuda.h>
-
 #include <algorithm>
 
 #include "attn_common.cuh"
@@ -46,15 +46,14 @@ template <int D, int KM>
 struct FL {
     static constexpr uint32_t kCh = D / 32;              // 32-element column chunks
     static constexpr uint32_t kQReg = 128 * 64;          // one chunk of the 128-row Q tile
-    static constexpr uint32_t kKVReg = kKT * 64;         // one chunk of a 64-row K or V tile
-    static constexpr uint32_t kTile = kCh * kKVReg;      // one K or V stage
+    static constexpr uint32_t kGB = kCh * 512;           // one 8-row group (grouped order)
+    static constexpr uint32_t kTile = 8 * kGB;           // one K or V stage: 64 rows
     static constexpr uint32_t kSlots = KM + 1;           // selected blocks per row (bound)
     static constexpr uint32_t kUCap = 128 * kSlots;      // union capacity in blocks
     static constexpr uint32_t kQ = 0;
     static constexpr uint32_t kK = kQ + kCh * kQReg;
     static constexpr uint32_t kV = kK + 2 * kTile;
-    static constexpr uint32_t kMeta = kV + 2 * kTile;    // int4 [2][64] window key coordinates
-    static constexpr uint32_t kUnion = kMeta + 2 * kKT * 16;   // int2 [kUCap+1] (first row, stream offset)
+    static constexpr uint32_t kUnion = kV + 2 * kTile;   // int2 [kUCap+1] (first group, stream group offset)
     static constexpr uint32_t kRange = kUnion + (kUCap + 1) * 8;   // int2 [kSlots][128] key ranges
     static constexpr uint32_t kBar = kRange + kSlots * 128 * 8;
     static constexpr uint32_t kMisc = kBar + 16 * 8;
@@ -100,6 +99,16 @@ __device__ __forceinline__ uint64_t span_bits(int a, int b) {
     return hi & (~0ull << a);
 }
 
+// s[c] = -inf where bit c of vm is clear
+__device__ __forceinline__ void apply_bits(float (&s)[64], uint64_t vm) {
+    const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        s[e] = (lo >> e) & 1u ? s[e] : -INFINITY;
+        s[e + 32] = (hi >> e) & 1u ? s[e + 32] : -INFINITY;
+    }
+}
+
 // Exclusive prefix sum over the 128 softmax threads (local index t); `red` holds 4 ints.
 __device__ __forceinline__ int scan128(int v, int t, int* red, int& total) {
     const int lane = t & 31, w = t >> 5;
@@ -124,10 +133,7 @@ __device__ __forceinline__ int scan128(int v, int t, int* red, int& total) {
 }
 
 template <typename T, int D, int KM>
-__global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
-    k_ssa_fwd(const __grid_constant__ FwdParams P, const __grid_constant__ CUtensorMap tm_kc,
-              const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kg,
-              const __grid_constant__ CUtensorMap tm_vg) {
+__global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(const __grid_constant__ FwdParams P) {
     using L = FL<D, KM>;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     extern __shared__ uint8_t smem_raw[];
@@ -136,7 +142,6 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
     uint64_t* bar = reinterpret_cast<uint64_t*>(g + L::kBar);
     int* misc = reinterpret_cast<int*>(g + L::kMisc);
     volatile int* abort_flag = misc + M_ABORT;
-    int4* meta = reinterpret_cast<int4*>(g + L::kMeta);
     int2* un = reinterpret_cast<int2*>(g + L::kUnion);
     int2* rng = reinterpret_cast<int2*>(g + L::kRange);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -145,11 +150,13 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
     // ---- per-CTA schedule --------------------------------------------------------------------
     const int32_t p0 = P.qt_pos[tile], len = P.qt_len[tile], seq = P.qt_seq[tile];
     const int32_t bl = P.seq_blk[seq], nblk = P.seq_blk[seq + 1] - bl;
-    const int32_t w0 = P.wt_off[tile], nwin = P.wt_off[tile + 1] - w0;
-    const int nc = (nblk + kKT - 1) / kKT;
-    const int nw = (nwin + kKT - 1) / kKT;
+    const int32_t cg0 = bl >> 3, cg1 = (bl + nblk + 7) >> 3;   // groups of the compressed tokens
+    const int32_t wr0 = P.wr_off[tile], nwr = P.wr_off[tile + 1] - wr0;
+    const int nc = (cg1 - cg0 + 7) >> 3;
+    const int nw = (P.wg_cnt[tile] + 7) >> 3;
+    const int32_t wm0 = P.wm_off[tile];
 
-    // ---- setup: TMEM, barriers, Q tile -------------------------------------------------------
+    // ---- setup: TMEM, barriers, Q tile, zeroed K/V stages --------------------------------------
     if (warp == 1) {
         tc::tmem_alloc(reinterpret_cast<uint32_t*>(misc + M_TMEM), kTmemCols);
         tc::tmem_relinquish();
@@ -158,10 +165,6 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
         for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], (i == PFULL || i == PFULL + 1) ? 4u : 1u);
         misc[M_ABORT] = 0;
         tc::fence_mbar_init();
-        tc::tma_prefetch_desc(&tm_kc);
-        tc::tma_prefetch_desc(&tm_vc);
-        tc::tma_prefetch_desc(&tm_kg);
-        tc::tma_prefetch_desc(&tm_vg);
     }
     const T* Q = reinterpret_cast<const T*>(P.q);
     for (int e = tid; e < 128 * (D / 8); e += kThreads) {
@@ -170,6 +173,10 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
         const T* src = ok ? Q + ((int64_t)P.perm[p0 + row] * H + h) * D + c16 * 8 : Q;
         tc::cp_async16(sb + L::kQ + (c16 >> 2) * L::kQReg + tc::sw64(row, c16 & 3), src, ok ? 16u : 0u);
     }
+    // groups a tile does not fill keep the previous contents; start from zeros (finite) so that
+    // masked keys (weight 0) never meet a non-finite V entry
+    for (uint32_t o = tid * 16u; o < 4u * L::kTile; o += kThreads * 16u)
+        *reinterpret_cast<uint4*>(g + L::kK + o) = make_uint4(0u, 0u, 0u, 0u);
     tc::cp_async_wait_all();
     tc::fence_proxy_async();
     tc::fence_before_sync();
@@ -179,97 +186,81 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
 
     if (warp == 0) {
         // ================================ producer ============================================
-        const int32_t pad_row = (int32_t)(h * P.Npad);   // a valid row; its keys are masked
-        int U = 0, Ltot = 0, ns = 0;
-        // rows (K/V row index in the [H * Npad, D] tensors) of keys `lane` and `lane + 32` of tile t
-        auto rows_of = [&](int ph, int t, int32_t& r0, int32_t& r1) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int i = lane + 32 * half;
-                int32_t row = pad_row;
-                if (ph == 1) {
-                    const int key = kKT * t + i;
-                    if (key < Ltot) {
-                        int lo = 0, hi = U - 1;   // last union block whose stream offset <= key
-                        while (lo < hi) {
-                            const int mid = (lo + hi + 1) >> 1;
-                            if (un[mid].y <= key) lo = mid; else hi = mid - 1;
-                        }
-                        row = pad_row + un[lo].x + (key - un[lo].y);
-                    }
-                } else {
-                    if (kKT * t + i < nwin) row = pad_row + P.wt_keys[w0 + kKT * t + i];
-                }
-                if (half == 0) r0 = row; else r1 = row;
-            }
+        // Every phase is a stream of runs of consecutive 8-row groups (compressed tokens: one run;
+        // selected blocks: one run per union block; window: the plan's runs). A 64-key tile takes
+        // the next 8 groups; lane l < 8 copies the part of run ri + l that falls in the tile.
+        const uint8_t* ksh = static_cast<const uint8_t*>(P.ks) + (int64_t)h * P.Npad * D * 2;
+        const uint8_t* vsh = static_cast<const uint8_t*>(P.vs) + (int64_t)h * P.Npad * D * 2;
+        const uint8_t* kch = static_cast<const uint8_t*>(P.kcg) + (int64_t)h * P.Mb8 * D * 2;
+        const uint8_t* vch = static_cast<const uint8_t*>(P.vcg) + (int64_t)h * P.Mb8 * D * 2;
+        int ri = 0, rskip = 0;   // next run, groups of it already streamed
+        int U = 0, ns = 0;
+        auto run_of = [&](int ph, int i) -> int2 {
+            if (ph == 0) return make_int2(cg0, cg1 - cg0);
+            if (ph == 1) return make_int2(un[i].x, un[i + 1].y - un[i].y);
+            return P.wr_runs[wr0 + i];
         };
-        auto gather = [&](const CUtensorMap* tm, uint32_t dst, uint64_t* fb, int32_t r0, int32_t r1) {
-            if (lane == 0) tc::mbar_arrive_expect_tx(fb, L::kTile);
-            __syncwarp();
-            int32_t y[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int src = (4 * lane + q) & 31;
-                const int32_t a = __shfl_sync(0xffffffffu, r0, src);
-                const int32_t b = __shfl_sync(0xffffffffu, r1, src);
-                y[q] = lane < 8 ? a : b;
-            }
-            if (lane < 16) {
-#pragma unroll
-                for (int c = 0; c < (int)L::kCh; ++c)
-                    tc::tma_gather4(dst + c * L::kKVReg + lane * 256, tm, 32 * c, y[0], y[1], y[2], y[3], fb);
-            }
-        };
-        auto produce = [&](int j, int ph, int t) -> bool {
+        auto produce = [&](int j, int ph) -> bool {
             const int s = j & 1;
             const uint32_t par_e = (uint32_t)((j >> 1) - 1) & 1u;
             const uint32_t kdst = sb + L::kK + s * L::kTile;
             const uint32_t vdst = sb + L::kV + s * L::kTile;
-            int32_t r0 = 0, r1 = 0;
-            if (ph > 0) rows_of(ph, t, r0, r1);
-            if (j >= 2 && !wait_or_flag(&bar[KEMPTY + s], par_e, P.status, abort_flag)) return false;
-            if (ph == 0) {
-                if (lane == 0) {
-                    const int32_t y = (int32_t)(h * P.Mb + bl + kKT * t);
-                    tc::mbar_arrive_expect_tx(&bar[KFULL + s], L::kTile);
-                    for (int c = 0; c < (int)L::kCh; ++c)
-                        tc::tma_load_2d(kdst + c * L::kKVReg, &tm_kc, 32 * c, y, &bar[KFULL + s]);
-                }
-            } else {
-                gather(&tm_kg, kdst, &bar[KFULL + s], r0, r1);
+            const int nruns = ph == 0 ? 1 : (ph == 1 ? U : nwr);
+            // this lane's segment: source group, destination group slot, groups
+            int32_t first = 0, n = 0;
+            if (lane < 8 && ri + lane < nruns) {
+                const int2 rr = run_of(ph, ri + lane);
+                first = rr.x + (lane == 0 ? rskip : 0);
+                n = rr.y - (lane == 0 ? rskip : 0);
             }
+            int pre = n;
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, pre, o);
+                if (lane >= o) pre += y;
+            }
+            const int start = pre - n;
+            const int take = lane < 8 ? max(0, min(pre, 8) - start) : 0;
+            const int total = min(__shfl_sync(0xffffffffu, pre, 7), 8);
+            const unsigned over = __ballot_sync(0xffffffffu, lane < 8 && pre > 8);
+            if (over) {
+                const int Lr = __ffs(over) - 1;
+                const int sL = __shfl_sync(0xffffffffu, start, Lr);
+                rskip = (Lr == 0 ? rskip : 0) + (8 - sL);
+                ri += Lr;
+            } else {
+                ri = min(ri + 8, nruns);
+                rskip = 0;
+            }
+            if (j >= 2 && !wait_or_flag(&bar[KEMPTY + s], par_e, P.status, abort_flag)) return false;
+            const uint8_t* ksrc = ph == 0 ? kch : ksh;
+            const uint8_t* vsrc = ph == 0 ? vch : vsh;
+            if (lane == 0) tc::mbar_arrive_expect_tx(&bar[KFULL + s], (uint32_t)total * L::kGB);
+            __syncwarp();
+            if (take > 0)
+                tc::bulk_load(kdst + start * L::kGB, ksrc + (int64_t)first * L::kGB, (uint32_t)take * L::kGB,
+                              &bar[KFULL + s]);
             // V stage and the key coordinates are free once P V of tile j-2 completed
             if (j >= 2 && !wait_or_flag(&bar[PVD + s], par_e, P.status, abort_flag)) return false;
-            if (ph == 0) {
-                if (lane == 0) {
-                    const int32_t y = (int32_t)(h * P.Mb + bl + kKT * t);
-                    tc::mbar_arrive_expect_tx(&bar[VFULL + s], L::kTile);
-                    for (int c = 0; c < (int)L::kCh; ++c)
-                        tc::tma_load_2d(vdst + c * L::kKVReg, &tm_vc, 32 * c, y, &bar[VFULL + s]);
-                }
-            } else {
-                if (ph == 2) {
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int i = lane + 32 * half;
-                        int4 mc = make_int4(1 << 28, 1 << 28, 1 << 28, -1);
-                        if (kKT * t + i < nwin) mc = P.scoord[P.wt_keys[w0 + kKT * t + i]];
-                        meta[s * kKT + i] = mc;
-                    }
-                }
-                gather(&tm_vg, vdst, &bar[VFULL + s], r0, r1);   // its __syncwarp orders meta
-            }
+            if (lane == 0) tc::mbar_arrive_expect_tx(&bar[VFULL + s], (uint32_t)total * L::kGB);
+            __syncwarp();
+            if (take > 0)
+                tc::bulk_load(vdst + start * L::kGB, vsrc + (int64_t)first * L::kGB, (uint32_t)take * L::kGB,
+                              &bar[VFULL + s]);
             return true;
         };
         bool ok = true;
-        for (int j = 0; j < nc && ok; ++j) ok = produce(j, 0, j);
+        for (int j = 0; j < nc && ok; ++j) ok = produce(j, 0);
         __syncwarp();
         tc::named_sync(1, kThreads);   // union of the selected blocks is built
         U = misc[M_U];
-        Ltot = misc[M_L];
-        ns = (Ltot + kKT - 1) / kKT;
-        for (int j = nc; j < nc + ns + nw && ok && !*abort_flag; ++j)
-            ok = j < nc + ns ? produce(j, 1, j - nc) : produce(j, 2, j - nc - ns);
+        ns = (misc[M_L] + 7) >> 3;
+        ri = 0;
+        rskip = 0;
+        for (int j = nc; j < nc + ns && ok && !*abort_flag; ++j) ok = produce(j, 1);
+        ri = 0;
+        rskip = 0;
+        for (int j = nc + ns; j < nc + ns + nw && ok && !*abort_flag; ++j) ok = produce(j, 2);
     } else if (warp == 1) {
         // ================================ MMA issuer ==========================================
         const uint32_t idesc_s = tc::idesc_f16(kBf16, 128, kKT, false);
@@ -285,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
                 tc::mma_f16_ss(tmem + b * kKT, tc::desc_kmajor_r(sb + L::kQ, kk, L::kQReg),
-                               tc::desc_kmajor_r(kbase, kk, L::kKVReg), idesc_s, kk > 0 ? 1u : 0u);
+                               tc::desc_kmajor_g(kbase, kk, L::kCh), idesc_s, kk > 0 ? 1u : 0u);
             tc::mma_commit(&bar[SFULL + b]);
             tc::mma_commit(&bar[KEMPTY + b]);
             return true;
@@ -298,9 +289,8 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
             const uint32_t vbase = sb + L::kV + b * L::kTile;
 #pragma unroll
             for (int kk = 0; kk < kKT / 16; ++kk)
-                tc::mma_f16_ts(tmem + 128, tmem + b * kKT + kk * 8,
-                               tc::desc_mnmajor_r(vbase, kk, L::kKVReg), idesc_o,
-                               (first && kk == 0) ? 0u : 1u);
+                tc::mma_f16_ts(tmem + 128, tmem + b * kKT + kk * 8, tc::desc_mnmajor_g(vbase, kk, L::kCh),
+                               idesc_o, (first && kk == 0) ? 0u : 1u);
             tc::mma_commit(&bar[PVD + b]);   // P V of tile i done: V stage, P buffer, O
             return true;
         };
@@ -314,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
         }
         __syncwarp();
         tc::named_sync(1, kThreads);
-        const int ns = (misc[M_L] + kKT - 1) / kKT;
+        const int ns = (misc[M_L] + 7) >> 3;
         const int nT = nc + ns + nw;
         if (lane == 0) {
             bool ok = !*abort_flag;
@@ -339,10 +329,8 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
         const int32_t pos = p0 + (row_ok ? row : len - 1);
         const int32_t tok = P.perm[pos];
         const int32_t ob = P.tok_blk[tok];
-        const int4 qc = P.scoord[P.blk_poff[ob] + (pos - P.blk_off[ob])];
         const float* gt = P.gates + ((int64_t)tok * H + h) * 3;
         float* brow = P.base + ((int64_t)pos * H + h) * D;
-        const int rr = P.r;
         const float sl = P.sl;
         const int ksel = P.k;
         float m = -INFINITY, l = 0.0f;
@@ -466,13 +454,13 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
         }
         bool ok = true;
         for (int j = 0; j < nc && ok; ++j) {
-            const int lim = nblk - kKT * j;
-            const int32_t bbase = bl + kKT * j;
+            const int32_t bbase = 8 * cg0 + kKT * j;   // block index of column 0
+            const int lo = bl - bbase, hi = bl + nblk - bbase;
             ok = step(j, j == 0, [&](float (&s)[64]) -> bool {
-                if (lim < kKT) {
+                if (lo > 0 || hi < kKT) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e)
-                        if (e >= lim) s[e] = -INFINITY;
+                        if (e < lo || e >= hi) s[e] = -INFINITY;
                 }
                 if (ksel > 1) {
 #pragma unroll
@@ -536,14 +524,18 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
                 while (wd) {
                     const int bit = __ffs(wd) - 1;
                     wd &= wd - 1;
-                    const int32_t gb = bl + 32 * i + bit;
-                    if (pre < (int)L::kUCap)
-                        un[pre] = make_int2(P.blk_poff[gb], P.blk_off[gb + 1] - P.blk_off[gb]);
+                    if (pre < (int)L::kUCap) un[pre].x = 32 * i + bit;   // local block index
                     ++pre;
                 }
             }
             tc::named_sync(2, 128);
-            // stream offsets: exclusive prefix of the block sizes
+            // first group and group count of every union block (independent loads)
+            for (int u = t128; u < U; u += 128) {
+                const int32_t gb = bl + un[u].x;
+                un[u] = make_int2(P.blk_poff[gb] >> 3, (P.blk_off[gb + 1] - P.blk_off[gb] + 7) >> 3);
+            }
+            tc::named_sync(2, 128);
+            // stream offsets (in groups): exclusive prefix of the blocks' group counts
             const int cu = (U + 127) >> 7;
             const int ul = min(t128 * cu, U), uh = min(ul + cu, U);
             int ssum = 0;
@@ -570,7 +562,8 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
                 for (int c = 0; c < (int)L::kSlots; ++c) rank += (mine[c] >= 0 && mine[c] < mine[a]) ? 1 : 0;
                 const int wi = mine[a] >> 5;
                 const int u = wpre[wi] + __popc(words[wi] & ((1u << (mine[a] & 31)) - 1u));
-                if (u < U) rng[rank * 128 + row] = make_int2(un[u].y, un[u + 1].y);
+                const int32_t gb = bl + mine[a];
+                if (u < U) rng[rank * 128 + row] = make_int2(8 * un[u].y, 8 * un[u].y + P.blk_off[gb + 1] - P.blk_off[gb]);
             }
         }
         int nr = 0;
@@ -578,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
         for (int u = 0; u < KM; ++u) nr += (row_ok && u + 1 < ksel && ti[u] >= 0) ? 1 : 0;
         nr += row_ok ? 1 : 0;
         tc::named_sync(1, kThreads);   // the producer may now overwrite the rings
-        const int ns = (misc[M_L] + kKT - 1) / kKT;
+        const int ns = (misc[M_L] + 7) >> 3;
         const int nT = nc + ns + nw;
 
         // ---- phase S: the selected blocks ------------------------------------------------------
@@ -596,32 +589,25 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks)
                     if (rg.y > base + kKT) break;
                     ++ri;
                 }
-                const uint32_t lo = (uint32_t)vm, hi = (uint32_t)(vm >> 32);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    if (!((lo >> e) & 1u)) s[e] = -INFINITY;
-                    if (!((hi >> e) & 1u)) s[e + 32] = -INFINITY;
-                }
+                apply_bits(s, vm);
                 return true;
             });
         }
         if (ok && ns > 0 && (ok = wait_pv(nc + ns - 1))) epilogue(1);
 
         // ---- phase W: the window ---------------------------------------------------------------
+        // the plan's mask words: bit c of this row's word = key c of the tile within distance r;
+        // each is loaded one tile ahead
         m = -INFINITY;
         l = 0.0f;
+        const uint64_t* wrow = P.wmask + (int64_t)wm0 * 128 + row;
+        uint64_t wnext = nw > 0 ? wrow[0] : 0ull;
         for (int j = nc + ns; j < nT && ok; ++j) {
-            const int b = j & 1;
-            ok = step(j, j == nc + ns, [&](float (&s)[64]) -> bool {
-                // the key coordinates travel with the V stage
-                if (!wait_or_flag(&bar[VFULL + b], (uint32_t)(j >> 1) & 1u, P.status, abort_flag)) return false;
-                const int4* km = meta + b * kKT;
-#pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const int4 kc = km[e];
-                    const int dd = max(abs(kc.x - qc.x), max(abs(kc.y - qc.y), abs(kc.z - qc.z)));
-                    if (dd > rr) s[e] = -INFINITY;
-                }
+            const int w = j - nc - ns;
+            const uint64_t wcur = wnext;
+            if (w + 1 < nw) wnext = wrow[(int64_t)(w + 1) * 128];
+            ok = step(j, w == 0, [&](float (&s)[64]) -> bool {
+                apply_bits(s, wcur);
                 return true;
             });
         }
@@ -646,41 +632,9 @@ __global__ void k_export_sel(const int32_t* __restrict__ sel, const int32_t* __r
     out[e] = sel[(int64_t)tok_pos[tok] * per_tok + rest];
 }
 
-// ---- host: tensor maps and launch ----------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (EncodeTiledFn)f;
-    }
-    return fn;
-}
-
-// rows x D matrix of 16-bit elements, boxes of 32 columns x `box_rows` rows, 64-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int D, bool bf16, uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {32, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
+// ---- host: launch -------------------------------------------------------------------------------
 template <typename T, int D, int KM>
-ssa_status_t run(const Plan* p, const FwdParams& P, const CUtensorMap* tm, int64_t max_seq_blocks,
-                 cudaStream_t st) {
+ssa_status_t run(const Plan* p, const FwdParams& P, int64_t max_seq_blocks, cudaStream_t st) {
     using L = FL<D, KM>;
     static_assert(L::kAlloc <= 227u * 1024u, "shared-memory layout exceeds the per-CTA limit");
     if (max_seq_blocks > L::kMaxSeqBlocks) return SSA_ERR_UNSUPPORTED;
@@ -691,26 +645,25 @@ ssa_status_t run(const Plan* p, const FwdParams& P, const CUtensorMap* tm, int64
             return SSA_ERR_CUDA;
         configured = true;
     }
-    k_ssa_fwd<T, D, KM><<<dim3((unsigned)p->n_qtiles, (unsigned)P.H), kThreads, L::kAlloc, st>>>(
-        P, tm[0], tm[1], tm[2], tm[3]);
+    k_ssa_fwd<T, D, KM><<<dim3((unsigned)p->n_qtiles, (unsigned)P.H), kThreads, L::kAlloc, st>>>(P);
     note_launch();
     return cudaPeekAtLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 
 template <typename T, int D>
-ssa_status_t run_km(const Plan* p, const FwdParams& P, const CUtensorMap* tm, int64_t mb, cudaStream_t st) {
-    if (P.k - 1 <= 8) return run<T, D, 8>(p, P, tm, mb, st);
-    if (P.k - 1 <= 16) return run<T, D, 16>(p, P, tm, mb, st);
-    return run<T, D, 32>(p, P, tm, mb, st);
+ssa_status_t run_km(const Plan* p, const FwdParams& P, int64_t mb, cudaStream_t st) {
+    if (P.k - 1 <= 8) return run<T, D, 8>(p, P, mb, st);
+    if (P.k - 1 <= 16) return run<T, D, 16>(p, P, mb, st);
+    return run<T, D, 32>(p, P, mb, st);
 }
 
 template <typename T>
-ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, const CUtensorMap* tm, int64_t mb, cudaStream_t st) {
+ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, int64_t mb, cudaStream_t st) {
     switch (D) {
-    case 32: return run_km<T, 32>(p, P, tm, mb, st);
-    case 64: return run_km<T, 64>(p, P, tm, mb, st);
-    case 96: return run_km<T, 96>(p, P, tm, mb, st);
-    default: return run_km<T, 128>(p, P, tm, mb, st);
+    case 32: return run_km<T, 32>(p, P, mb, st);
+    case 64: return run_km<T, 64>(p, P, mb, st);
+    case 96: return run_km<T, 96>(p, P, mb, st);
+    default: return run_km<T, 128>(p, P, mb, st);
     }
 }
 
@@ -719,12 +672,6 @@ ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, const CUtensorMap* 
 ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
                                void* out, cudaStream_t st) {
     const bool bf16 = w.dtype == SSA_BF16;
-    CUtensorMap tm[4];
-    if (!make_map(&tm[0], w.kc, (int64_t)w.H * p->Mb, w.D, bf16, kKT) ||
-        !make_map(&tm[1], w.vc, (int64_t)w.H * p->Mb, w.D, bf16, kKT) ||
-        !make_map(&tm[2], w.ks, (int64_t)w.H * p->Npad, w.D, bf16, 1) ||
-        !make_map(&tm[3], w.vs, (int64_t)w.H * p->Npad, w.D, bf16, 1))
-        return SSA_ERR_CUDA;
     int64_t max_seq_blocks = 0;
     for (size_t s = 0; s + 1 < p->seq_blk.size(); ++s)
         max_seq_blocks = std::max<int64_t>(max_seq_blocks, p->seq_blk[s + 1] - p->seq_blk[s]);
@@ -732,8 +679,8 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.q = q;
     P.ks = w.ks;
     P.vs = w.vs;
-    P.kc = w.kc;
-    P.vc = w.vc;
+    P.kcg = w.kcg;
+    P.vcg = w.vcg;
     P.gates = gates;
     P.perm = p->perm;
     P.tok_blk = p->tok_blk;
@@ -744,8 +691,11 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.qt_len = p->qt_len;
     P.qt_seq = p->qt_seq;
     P.seq_blk = p->seq_blk_d;
-    P.wt_off = p->wt_off;
-    P.wt_keys = p->wt_keys;
+    P.wr_off = p->wr_off;
+    P.wr_runs = p->wr_runs;
+    P.wg_cnt = p->wg_cnt;
+    P.wm_off = p->wm_off;
+    P.wmask = p->wmask;
     P.sel = w.sel;
     P.base = w.base;
     P.out = out;
@@ -753,13 +703,14 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.N = p->N;
     P.Npad = p->Npad;
     P.Mb = p->Mb;
+    P.Mb8 = w.Mb8;
     P.H = w.H;
     P.k = w.k;
     P.r = p->r;
     P.sl = (float)(1.4426950408889634 / sqrt((double)w.D));
     ProfScope ps("k_ssa_fwd", st);
-    if (bf16) return run_d<__nv_bfloat16>(p, P, w.D, tm, max_seq_blocks, st);
-    return run_d<__half>(p, P, w.D, tm, max_seq_blocks, st);
+    if (bf16) return run_d<__nv_bfloat16>(p, P, w.D, max_seq_blocks, st);
+    return run_d<__half>(p, P, w.D, max_seq_blocks, st);
 }
 
 void launch_export_sel(const Plan* p, const Workspace& w, int32_t* sel_out, cudaStream_t st) {

@@ -24,7 +24,7 @@ enum : int32_t {
 };
 
 constexpr int kBlockEdge = 8;      // block edge in voxels (the only supported value)
-constexpr int kPad = 16;           // blocks start on multiples of 16 rows in the sorted K/V copies
+constexpr int kPad = 8;            // blocks start on multiples of 8 rows (one group) in the K/V copies
 constexpr int kQTile = 128;        // query rows per tensor-core tile
 constexpr int kMaxTopk = 32;
 
@@ -40,10 +40,15 @@ struct SeqInfo {
 struct Workspace {
     int32_t H = 0, D = 0, k = 0;
     ssa_dtype_t dtype = SSA_F32;
-    void* ks = nullptr;        // [H, Npad, D] T   K rows in padded block order
+    // K_s, V_s: per head, the K / V rows in padded block order (Npad rows), stored as 8-row
+    // groups in the tensor cores' swizzled operand order (see pool.cu); padding rows are zero.
+    void* ks = nullptr;        // [H, Npad, D] T
     void* vs = nullptr;        // [H, Npad, D] T
-    void* kc = nullptr;        // [H, Mb, D]   T (fp32 for the fp32 path)
+    void* kc = nullptr;        // [H, Mb, D]   T (fp32 for the fp32 path), row-major
     void* vc = nullptr;        // [H, Mb, D]
+    void* kcg = nullptr;       // [H, Mb8, D]  T   compressed tokens in the grouped order (16-bit path)
+    void* vcg = nullptr;       // [H, Mb8, D]
+    int64_t Mb8 = 0;           // Mb rounded up to a multiple of 8
     float* base = nullptr;     // [N, H, D]    running g0*o_cmp + g1*o_sel, sorted token order
     int32_t* sel = nullptr;    // [N, H, k]        selected blocks, sorted token order
     // host-buffer entry point staging (allocated on first use)
@@ -90,6 +95,11 @@ struct Plan {
     int32_t* qt_seq = nullptr;   // [n_qtiles]
     int32_t* wt_off = nullptr;   // [n_qtiles+1] window key union per query tile (CSR)
     int32_t* wt_keys = nullptr;  // padded rows, ascending
+    int32_t* wr_off = nullptr;   // [n_qtiles+1] runs of consecutive 8-row groups covering wt_keys (CSR)
+    int2* wr_runs = nullptr;     // (first group, groups) of each run
+    int32_t* wg_cnt = nullptr;   // [n_qtiles] groups of each tile's window union
+    int32_t* wm_off = nullptr;   // [n_qtiles+1] first 64-key window tile of each query tile
+    uint64_t* wmask = nullptr;   // [wm_off[T]][128] window mask: bit c of row i = key c within r
     std::vector<void*> owned;
     Workspace ws;
 };

@@ -354,6 +354,89 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
     if (!kFill && threadIdx.x == 0) wt_cnt[t] = total;
 }
 
+// Runs of consecutive 8-row groups that cover each tile's window union (the attention kernel
+// loads every run with one bulk copy). One lane per tile walks the ascending rows.
+// kFill == false writes the run and group counts, kFill == true the runs at wr_off.
+template <bool kFill>
+__global__ void k_window_runs(int64_t T, const int32_t* __restrict__ wt_off,
+                              const int32_t* __restrict__ wt_keys, int32_t* __restrict__ wr_cnt,
+                              int32_t* __restrict__ wg_cnt, int32_t* __restrict__ wm_cnt,
+                              const int32_t* __restrict__ wr_off, int2* __restrict__ runs) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    const int32_t a = wt_off[t], b = wt_off[t + 1];
+    int32_t nr = 0, ng = 0, first = -1, cnt = 0, prev = -2;
+    const int32_t out = kFill ? wr_off[t] : 0;
+    for (int32_t i = a; i < b; ++i) {
+        const int32_t gi = wt_keys[i] >> 3;
+        if (gi == prev) continue;
+        ++ng;
+        if (gi == prev + 1) {
+            ++cnt;
+        } else {
+            if (first >= 0) {
+                if (kFill) runs[out + nr] = make_int2(first, cnt);
+                ++nr;
+            }
+            first = gi;
+            cnt = 1;
+        }
+        prev = gi;
+    }
+    if (first >= 0) {
+        if (kFill) runs[out + nr] = make_int2(first, cnt);
+        ++nr;
+    }
+    if (!kFill) {
+        wr_cnt[t] = nr;
+        wg_cnt[t] = ng;
+        wm_cnt[t] = (ng + 7) >> 3;
+    }
+}
+
+// Window masks: for each query tile and each 64-key tile of its window stream (the runs' groups
+// in order, 8 rows per group), bit c of row i says whether key c lies within Chebyshev distance r
+// of query i. One thread per query row; key coordinates are read once per group by all threads.
+__global__ void __launch_bounds__(kQTile) k_window_masks(const int32_t* __restrict__ qt_pos,
+                                                         const int32_t* __restrict__ qt_len,
+                                                         const int32_t* __restrict__ perm,
+                                                         const int32_t* __restrict__ coords,
+                                                         const int32_t* __restrict__ wr_off,
+                                                         const int2* __restrict__ runs,
+                                                         const int32_t* __restrict__ wm_off,
+                                                         const int4* __restrict__ scoord, int r,
+                                                         uint64_t* __restrict__ wmask) {
+    const int t = blockIdx.x, row = threadIdx.x;
+    const int32_t p0 = qt_pos[t], len = qt_len[t];
+    const bool ok = row < len;
+    int32_t qx = 0, qy = 0, qz = 0;
+    if (ok) {
+        const int32_t i = perm[p0 + row];
+        qx = coords[3 * i];
+        qy = coords[3 * i + 1];
+        qz = coords[3 * i + 2];
+    }
+    uint64_t* out = wmask + (int64_t)wm_off[t] * kQTile + row;
+    uint64_t word = 0;
+    int q = 0;   // groups streamed so far
+    for (int32_t ri = wr_off[t]; ri < wr_off[t + 1]; ++ri) {
+        const int2 run = runs[ri];
+        for (int32_t gi = run.x; gi < run.x + run.y; ++gi, ++q) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int4 kc = scoord[8 * (int64_t)gi + i];
+                const int d = max(abs(kc.x - qx), max(abs(kc.y - qy), abs(kc.z - qz)));
+                if (ok && d <= r) word |= 1ull << (((q & 7) << 3) + i);
+            }
+            if ((q & 7) == 7) {
+                out[(int64_t)(q >> 3) * kQTile] = word;
+                word = 0;
+            }
+        }
+    }
+    if (q & 7) out[(int64_t)(q >> 3) * kQTile] = word;
+}
+
 }  // namespace
 
 #define SSA_ALLOC(ptr, type, count)                                                      \
@@ -507,6 +590,17 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         p->blk_off, key2blk, p->d_seqs, p->scoord, r, nullptr, p->wt_off, p->wt_keys);
     note_launch();
     trace_step("plan window unions", st);
+    int32_t *wr_cnt, *wm_cnt;
+    SSA_ALLOC(wr_cnt, int32_t, T + 1);
+    SSA_ALLOC(wm_cnt, int32_t, T + 1);
+    SSA_ALLOC(p->wr_off, int32_t, T + 1);
+    SSA_ALLOC(p->wg_cnt, int32_t, T);
+    SSA_ALLOC(p->wm_off, int32_t, T + 1);
+    k_window_runs<false><<<(unsigned)cdiv(T, 128), 128, 0, st>>>(T, p->wt_off, p->wt_keys, wr_cnt,
+                                                                  p->wg_cnt, wm_cnt, nullptr, nullptr);
+    note_launch();
+    scan_exclusive(wr_cnt, p->wr_off, T, tmp, st);
+    scan_exclusive(wm_cnt, p->wm_off, T, tmp, st);
 
     // block range of every sequence (host copy for launches)
     p->seq_blk.assign(B + 1, 0);
@@ -516,10 +610,19 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         if (cudaMemcpyAsync(&sb[s], bidx + key, sizeof(int32_t), cudaMemcpyDeviceToHost, st))
             return SSA_ERR_CUDA;
     }
-    int32_t status = 0;
+    int32_t status = 0, n_runs = 0, n_wtiles = 0;
     if (cudaMemcpyAsync(&status, p->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaMemcpyAsync(&n_runs, p->wr_off + T, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaMemcpyAsync(&n_wtiles, p->wm_off + T, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
         cudaStreamSynchronize(st))
         return SSA_ERR_CUDA;
+    SSA_ALLOC(p->wr_runs, int2, n_runs);
+    SSA_ALLOC(p->wmask, uint64_t, (int64_t)n_wtiles * kQTile);
+    k_window_runs<true><<<(unsigned)cdiv(T, 128), 128, 0, st>>>(T, p->wt_off, p->wt_keys, nullptr,
+                                                                 nullptr, nullptr, p->wr_off, p->wr_runs);
+    k_window_masks<<<(unsigned)T, kQTile, 0, st>>>(p->qt_pos, p->qt_len, p->perm, p->coords, p->wr_off,
+                                                   p->wr_runs, p->wm_off, p->scoord, r, p->wmask);
+    note_launch(2);
     for (int s = 0; s <= B; ++s) p->seq_blk[s] = sb[s];
     SSA_ALLOC(p->seq_blk_d, int32_t, B + 1);
     if (cudaMemcpyAsync(p->seq_blk_d, sb.data(), sizeof(int32_t) * (B + 1), cudaMemcpyHostToDevice, st) ||
@@ -529,7 +632,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
 
     // scratch of the plan build is released now
     void* scratch[] = {tok_key, key_cnt, bidx, key2blk, blk_cnt, blk_pcnt, blk_fill,
-                       nbr_cnt, tmp, hkeys, hvals, wt_cnt};
+                       nbr_cnt, tmp, hkeys, hvals, wt_cnt, wr_cnt, wm_cnt};
     for (void* ptr : scratch) {
         auto it = std::find(p->owned.begin(), p->owned.end(), ptr);
         if (it != p->owned.end()) {

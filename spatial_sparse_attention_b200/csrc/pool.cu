@@ -6,12 +6,27 @@
 // One CTA per occupied block. Each thread owns one 16-byte column group of the token rows (all
 // heads of a token are contiguous), so every token row is read with fully coalesced 128-bit loads;
 // sums are fp32. For the tensor-core path the same pass also writes the rows into the padded,
-// head-major, block-ordered copies K_s, V_s [H, Npad, D] that the attention tiles read.
+// head-major, block-ordered copies K_s, V_s [H, Npad, D] that the attention tiles read, and the
+// compressed tokens a second time in the same order.
+//
+// Grouped order (16-bit types): rows are taken 8 at a time; a group stores its D/32 column chunks
+// one after the other, each as a 512-byte atom of 8 rows x 64 bytes in which the four 16-byte
+// units of row i are permuted by unit ^= (i >> 1) & 3. This is the shared-memory operand order of
+// the tensor cores with 64-byte swizzle, so a run of consecutive groups is copied to shared
+// memory with one bulk copy and used there as is.
 #include "common.cuh"
 
 namespace ssa {
 
 namespace {
+
+// byte offset of element column d of row `row` (16-byte unit granularity: d % 8 == 0) inside a
+// grouped matrix with D columns
+__device__ __forceinline__ int64_t grouped_off(int64_t row, int d, int D) {
+    const int64_t g = row >> 3;
+    const int i = (int)(row & 7), c = d >> 5, u = (d & 31) >> 3;
+    return g * (int64_t)(D / 32) * 512 + c * 512 + i * 64 + ((u ^ ((i >> 1) & 3)) << 4);
+}
 
 constexpr int kMaxGroupsPerThread = 2;
 
@@ -23,7 +38,8 @@ __global__ void __launch_bounds__(1024) k_pool(const T* __restrict__ K, const T*
                                                const int32_t* __restrict__ blk_poff, int64_t Mb,
                                                int H, int D, int64_t Npad, T* __restrict__ ks,
                                                T* __restrict__ vs, T* __restrict__ kc,
-                                               T* __restrict__ vc) {
+                                               T* __restrict__ vc, int64_t Mb8,
+                                               T* __restrict__ kcg, T* __restrict__ vcg) {
     constexpr int kVec = 16 / sizeof(T);
     extern __shared__ float mean[];   // [2][H*D]: K means then V means
     const int64_t b = blockIdx.x;
@@ -56,9 +72,9 @@ __global__ void __launch_bounds__(1024) k_pool(const T* __restrict__ K, const T*
             }
             if (kSorted) {
                 const int col = gidx * kVec, h = col / D, d = col % D;
-                const int64_t dst = ((int64_t)h * Npad + prow + t) * D + d;
-                *reinterpret_cast<uint4*>(ks + dst) = kq;
-                *reinterpret_cast<uint4*>(vs + dst) = vq;
+                const int64_t dst = (int64_t)h * Npad * D * (int64_t)sizeof(T) + grouped_off(prow + t, d, D);
+                *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ks) + dst) = kq;
+                *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(vs) + dst) = vq;
             }
         }
     }
@@ -88,6 +104,12 @@ __global__ void __launch_bounds__(1024) k_pool(const T* __restrict__ K, const T*
         const int64_t dst = ((int64_t)h * Mb + b) * D + e;
         kc[dst] = Elem<T>::from_f(ak);
         vc[dst] = Elem<T>::from_f(av);
+        if (kSorted) {
+            const int64_t gd = (int64_t)h * Mb8 * D * (int64_t)sizeof(T) + grouped_off(b, e & ~7, D) +
+                               (e & 7) * (int64_t)sizeof(T);
+            *reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(kcg) + gd) = Elem<T>::from_f(ak);
+            *reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(vcg) + gd) = Elem<T>::from_f(av);
+        }
     }
 }
 
@@ -106,7 +128,7 @@ void run_pool(const Plan* p, const Workspace& w, const void* k, const void* v, c
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kern<<<(unsigned)p->Mb, threads, smem, st>>>(
         (const T*)k, (const T*)v, wc, p->perm, p->blk_off, p->blk_poff, p->Mb, w.H, w.D, p->Npad,
-        (T*)w.ks, (T*)w.vs, (T*)w.kc, (T*)w.vc);
+        (T*)w.ks, (T*)w.vs, (T*)w.kc, (T*)w.vc, w.Mb8, (T*)w.kcg, (T*)w.vcg);
     note_launch();
 }
 

@@ -51,6 +51,18 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk) {
     return smem_desc(base + (uint32_t)kk * 1024, kRegion, 512);
 }
 
+// Grouped layout: a tile is a sequence of 8-row groups; each group holds its kch 32-element
+// chunks as consecutive 512-byte swizzled atoms (group stride kch * 512 bytes). K-major operand
+// (rows = N, K contiguous): K step `kk` is in chunk kk/2 at byte 32*(kk%2) of every atom.
+__device__ __forceinline__ uint64_t desc_kmajor_g(uint32_t base, int kk, uint32_t kch) {
+    return smem_desc(base + (uint32_t)(kk >> 1) * 512 + (uint32_t)(kk & 1) * 32, 16, kch * 512);
+}
+// Grouped layout, MN-major operand (rows = K, N contiguous inside chunks): K step `kk` covers
+// groups 2kk and 2kk+1; N chunks are 512 bytes apart, 8-row groups kch * 512 bytes apart.
+__device__ __forceinline__ uint64_t desc_mnmajor_g(uint32_t base, int kk, uint32_t kch) {
+    return smem_desc(base + (uint32_t)kk * 2 * kch * 512, 512, kch * 512);
+}
+
 // Same, for tiles whose 32-element chunks are `region` bytes apart.
 __device__ __forceinline__ uint64_t desc_kmajor_r(uint32_t base, int kk, uint32_t region) {
     return smem_desc(base + (uint32_t)(kk >> 1) * region + (uint32_t)(kk & 1) * 32, 16, 512);
@@ -241,6 +253,14 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int3
         "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
         "r"(smem_u32(bar))
+        : "memory");
+}
+// 1D bulk copy (no multicast) of `bytes` contiguous bytes from global `src` to shared `dst`,
+// completing `bytes` transactions on `bar`. Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {

@@ -27,8 +27,9 @@
  *     by kernels (bad coordinates, bounded waits that ran out) are recorded in the plan's device
  *     status word, returned by the next call that waits for the device, and readable with
  *     ssa_last_device_status. No kernel traps or asserts.
- *   - Device memory is obtained through the allocator hook (ssa_set_allocator; default
- *     cudaMallocAsync/cudaFreeAsync on the call's stream). A plan owns its buffers until
+ *   - Device memory is obtained through the allocator hook (ssa_set_allocator; default:
+ *     stream-ordered allocation on the call's stream from a memory pool owned by the library,
+ *     one per device, that keeps freed memory cached for reuse). A plan owns its buffers until
  *     ssa_plan_destroy; the forward workspace is cached in the plan and allocated on the first
  *     forward call for a given (H, D, dtype, k), so later calls of that shape allocate nothing.
  *   - Supported: block = 8; 0 <= r <= 8; 1 <= k <= 32; D in {32, 64, 96, 128};
@@ -72,7 +73,7 @@ typedef enum {
 typedef void* (*ssa_alloc_fn)(size_t bytes, void* stream, void* ctx);
 typedef void (*ssa_free_fn)(void* ptr, void* stream, void* ctx);
 
-/* Replace the process-wide allocator (NULL, NULL restores cudaMallocAsync/cudaFreeAsync).
+/* Replace the process-wide allocator (NULL, NULL restores the default pool allocator).
  * Plans keep the hook they were created with. Not thread-safe against concurrent plan calls. */
 SSA_API ssa_status_t ssa_set_allocator(ssa_alloc_fn alloc, ssa_free_fn release, void* ctx);
 

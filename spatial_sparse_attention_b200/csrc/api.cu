@@ -90,9 +90,39 @@ void profile_record(const char* name, cudaEvent_t start, cudaEvent_t stop) {
 
 namespace {
 
+// The default hook allocates stream-ordered from a memory pool owned by this library (one per
+// device) whose release threshold keeps freed memory for reuse: a plan rebuilt every step then
+// allocates from cached memory instead of mapping new pages at every synchronisation.
+cudaMemPool_t library_pool() {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        uint64_t keep = ~0ull;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
 void* default_alloc(size_t bytes, void* stream, void*) {
     void* p = nullptr;
-    if (cudaMallocAsync(&p, bytes, (cudaStream_t)stream) != cudaSuccess) {
+    cudaMemPool_t pool = library_pool();
+    const cudaError_t e = pool ? cudaMallocFromPoolAsync(&p, bytes, pool, (cudaStream_t)stream)
+                               : cudaMallocAsync(&p, bytes, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
         cudaGetLastError();
         return nullptr;
     }
@@ -270,7 +300,11 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
         launch_pool(p, w, k, v, wc, st);
     }
     trace_step("pool", st);
-    if (dt == SSA_F32) launch_forward_simt(p, w, q, k, v, gates, out, st);
+    if (dt == SSA_F32) {
+        // the CUDA-core path walks the per-token neighbour lists
+        if ((rc = ensure_neighbours(p, st)) != SSA_OK) return rc;
+        launch_forward_simt(p, w, q, k, v, gates, out, st);
+    }
     else if ((rc = launch_forward_tc(p, w, q, gates, out, st)) != SSA_OK) return rc;
     trace_step("forward", st);
     if (sel_out) launch_export_sel(p, w, sel_out, st);
@@ -360,6 +394,10 @@ ssa_status_t ssa_plan_export(ssa_plan_t p, int32_t* perm, int32_t* tok_blk, int3
     if (!p) return SSA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const auto D2D = cudaMemcpyDeviceToDevice;
+    if (nbr_idx) {
+        const ssa_status_t rc = ensure_neighbours(p, st);
+        if (rc != SSA_OK) return rc;
+    }
     cudaError_t e = cudaSuccess;
     if (perm && !e) e = cudaMemcpyAsync(perm, p->perm, sizeof(int32_t) * p->N, D2D, st);
     if (tok_blk && !e) e = cudaMemcpyAsync(tok_blk, p->tok_blk, sizeof(int32_t) * p->N, D2D, st);
@@ -456,6 +494,7 @@ ssa_status_t ssa_backward(ssa_plan_t p, const void* q, const void* k, const void
     // which the backward overwrites)
     rc = run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, dq, nullptr, st);
     if (rc != SSA_OK) return rc;
+    if ((rc = ensure_neighbours(p, st)) != SSA_OK) return rc;
     return launch_backward(p, p->ws, q, k, v, gates, wc, dout, dq, dk, dv, st);
 }
 

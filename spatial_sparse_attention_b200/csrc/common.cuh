@@ -89,7 +89,12 @@ struct Plan {
     int32_t* spos_tok = nullptr; // [Npad] token of each padded row, -1 for padding
     int4* scoord = nullptr;      // [Npad] (x, y, z, block) of each padded row; padding far away
     int32_t* nbr_off32 = nullptr;// [N+1]
-    int32_t* nbr_idx = nullptr;  // [nnz]
+    int32_t* nbr_idx = nullptr;  // [nnz], built on first use (backward, export): the forward's
+                                 // window runs and masks do not need per-token lists
+    uint64_t* hkeys = nullptr;   // coordinate hash (kept for the lazy neighbour lists)
+    int32_t* hvals = nullptr;
+    uint64_t hmask = 0;
+    int32_t nbr_cap = 32;        // per-warp sort buffer of the neighbour-list kernel
     int32_t* qt_pos = nullptr;   // [n_qtiles] first sorted position of each query tile
     int32_t* qt_len = nullptr;   // [n_qtiles]
     int32_t* qt_seq = nullptr;   // [n_qtiles]
@@ -146,6 +151,8 @@ void scan_exclusive(const int32_t* in, int32_t* out, int64_t n, int32_t* tmp, cu
 
 // plan.cu
 ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t s);
+// the per-token window neighbour lists (nbr_idx), built once per plan on first use
+ssa_status_t ensure_neighbours(Plan* p, cudaStream_t s);
 
 // pool.cu
 void launch_pool(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,

@@ -265,9 +265,18 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
     const SeqInfo q = seqs[qt_seq[t]];
     if (threadIdx.x == 0) { ncand_s = 0; ntb_s = 0; }
     __syncthreads();
+    __shared__ int box[6];   // bounding box of the tile's tokens: min x, y, z, max x, y, z
+    if (threadIdx.x < 6) box[threadIdx.x] = threadIdx.x < 3 ? 0x7fffffff : -0x7fffffff;
+    __syncthreads();
     for (int a = threadIdx.x; a < len; a += blockDim.x) {
         int32_t i = perm[p0 + a];
         qc[a] = make_int4(coords[3 * i], coords[3 * i + 1], coords[3 * i + 2], 0);
+        atomicMin(&box[0], qc[a].x);
+        atomicMin(&box[1], qc[a].y);
+        atomicMin(&box[2], qc[a].z);
+        atomicMax(&box[3], qc[a].x);
+        atomicMax(&box[4], qc[a].y);
+        atomicMax(&box[5], qc[a].z);
     }
     // distinct blocks of the tile (the tile is a run of consecutive sorted tokens)
     if (threadIdx.x == 0) {
@@ -320,15 +329,22 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
     const int ncand = ncand_s;
     int32_t out_base = kFill ? wt_off[t] : 0;
     int total = 0;
+    const int bx0 = box[0] - r, by0 = box[1] - r, bz0 = box[2] - r;
+    const int bx1 = box[3] + r, by1 = box[4] + r, bz1 = box[5] + r;
     for (int cb = 0; cb < ncand; ++cb) {
         int32_t b = cand[cb];
+        // a block whose 8^3 cube misses the tile's box grown by r holds no window key
+        const int cx = 8 * blk_coord[3 * b], cy = 8 * blk_coord[3 * b + 1], cz = 8 * blk_coord[3 * b + 2];
+        if (cx > bx1 || cx + 7 < bx0 || cy > by1 || cy + 7 < by0 || cz > bz1 || cz + 7 < bz0) continue;
         int32_t r0 = blk_poff[b], nrow = blk_off[b + 1] - blk_off[b];
         for (int a0 = 0; a0 < nrow; a0 += blockDim.x) {
             int a = a0 + threadIdx.x;
             bool keep = false;
             if (a < nrow) {
                 int4 kc = scoord[r0 + a];
-                for (int u = 0; u < len && !keep; ++u) {
+                const bool inbox = kc.x >= bx0 && kc.x <= bx1 && kc.y >= by0 && kc.y <= by1 &&
+                                   kc.z >= bz0 && kc.z <= bz1;
+                for (int u = 0; u < len && !keep && inbox; ++u) {
                     int4 c = qc[u];
                     int d = max(abs(kc.x - c.x), max(abs(kc.y - c.y), abs(kc.z - c.z)));
                     keep = d <= r;
@@ -538,7 +554,6 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     SSA_ALLOC(p->tok_pos, int32_t, N);
     SSA_ALLOC(p->spos_tok, int32_t, p->Npad);
     SSA_ALLOC(p->scoord, int4, p->Npad);
-    SSA_ALLOC(p->nbr_idx, int32_t, p->nnz);
     k_scatter<<<grid_for(N), kThreads, 0, st>>>(tok_key, key2blk, N, p->blk_off, blk_fill, p->perm,
                                                 p->tok_blk);
     k_sort_blocks<<<grid_for(p->Mb, 8), 256, 0, st>>>(p->perm, p->blk_off, p->Mb);
@@ -551,11 +566,12 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     trace_step("plan scatter/sort/positions", st);
     note_launch(5);
 
-    // ---- a2: neighbour lists -----------------------------------------------------------------------
-    k_neighbours<true><<<grid_for(N, warps), warps * 32, (size_t)warps * cap * sizeof(int32_t), st>>>(
-        coords, N, p->d_seqs, B, r, hkeys, hvals, hsize - 1, nullptr, p->nbr_off32, p->nbr_idx,
-        cap, p->d_status);
-    note_launch();
+    // ---- a2: the per-token neighbour lists are built on first use (ensure_neighbours) ----------------
+    p->hkeys = hkeys;
+    p->hvals = hvals;
+    p->hmask = hsize - 1;
+    p->nbr_cap = cap;
+    p->nbr_idx = nullptr;
 
     // ---- query tiles and their window key unions (tensor-core window kernel) ----------------------
     std::vector<int32_t> qpos, qlen, qseq;
@@ -623,6 +639,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     k_window_masks<<<(unsigned)T, kQTile, 0, st>>>(p->qt_pos, p->qt_len, p->perm, p->coords, p->wr_off,
                                                    p->wr_runs, p->wm_off, p->scoord, r, p->wmask);
     note_launch(2);
+    trace_step("plan window runs + masks", st);
     for (int s = 0; s <= B; ++s) p->seq_blk[s] = sb[s];
     SSA_ALLOC(p->seq_blk_d, int32_t, B + 1);
     if (cudaMemcpyAsync(p->seq_blk_d, sb.data(), sizeof(int32_t) * (B + 1), cudaMemcpyHostToDevice, st) ||
@@ -632,7 +649,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
 
     // scratch of the plan build is released now
     void* scratch[] = {tok_key, key_cnt, bidx, key2blk, blk_cnt, blk_pcnt, blk_fill,
-                       nbr_cnt, tmp, hkeys, hvals, wt_cnt, wr_cnt, wm_cnt};
+                       nbr_cnt, tmp, wt_cnt, wr_cnt, wm_cnt};
     for (void* ptr : scratch) {
         auto it = std::find(p->owned.begin(), p->owned.end(), ptr);
         if (it != p->owned.end()) {
@@ -640,6 +657,18 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
             p->owned.erase(it);
         }
     }
+    return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+ssa_status_t ensure_neighbours(Plan* p, cudaStream_t st) {
+    if (p->nbr_idx || p->nnz == 0) return SSA_OK;
+    SSA_ALLOC(p->nbr_idx, int32_t, p->nnz);
+    const int cap = p->nbr_cap;
+    const int warps = std::max(1, std::min(8, 8192 / cap));
+    k_neighbours<true><<<grid_for(p->N, warps), warps * 32, (size_t)warps * cap * sizeof(int32_t), st>>>(
+        p->coords, p->N, p->d_seqs, p->B, p->r, p->hkeys, p->hvals, p->hmask, nullptr, p->nbr_off32,
+        p->nbr_idx, cap, p->d_status);
+    note_launch();
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 

@@ -90,6 +90,14 @@ __device__ __forceinline__ float pick16(const float* v, int e) {
     return (e & 8) ? c1 : c0;
 }
 
+// v[e] for a per-thread index e in [0, 64): a select tree within each 16-group, then across groups
+__device__ __forceinline__ float pick64(const float (&v)[64], int e) {
+    const float g0 = pick16(v, e & 15), g1 = pick16(v + 16, e & 15);
+    const float g2 = pick16(v + 32, e & 15), g3 = pick16(v + 48, e & 15);
+    const float lo = (e & 16) ? g1 : g0, hi = (e & 16) ? g3 : g2;
+    return (e & 32) ? hi : lo;
+}
+
 // Bits [a, b) of a 64-bit word, a and b clamped to [0, 64].
 __device__ __forceinline__ uint64_t span_bits(int a, int b) {
     a = max(a, 0);
@@ -250,17 +258,21 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             return true;
         };
         bool ok = true;
-        for (int j = 0; j < nc && ok; ++j) ok = produce(j, 0);
-        __syncwarp();
-        tc::named_sync(1, kThreads);   // union of the selected blocks is built
-        U = misc[M_U];
-        ns = (misc[M_L] + 7) >> 3;
-        ri = 0;
-        rskip = 0;
-        for (int j = nc; j < nc + ns && ok && !*abort_flag; ++j) ok = produce(j, 1);
-        ri = 0;
-        rskip = 0;
-        for (int j = nc + ns; j < nc + ns + nw && ok && !*abort_flag; ++j) ok = produce(j, 2);
+        for (int j = 0;; ++j) {
+            if (j == nc) {
+                __syncwarp();
+                tc::named_sync(1, kThreads);   // union of the selected blocks is built
+                U = misc[M_U];
+                ns = (misc[M_L] + 7) >> 3;
+            }
+            if (j == nc || j == nc + ns) {
+                ri = 0;
+                rskip = 0;
+            }
+            if (j >= nc && (!ok || *abort_flag || j >= nc + ns + nw)) break;
+            if (!ok) continue;   // phase C stopped early: still meet the others at the union barrier
+            ok = produce(j, j < nc ? 0 : (j < nc + ns ? 1 : 2));
+        }
     } else if (warp == 1) {
         // ================================ MMA issuer ==========================================
         const uint32_t idesc_s = tc::idesc_f16(kBf16, 128, kKT, false);
@@ -320,6 +332,8 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
         __syncwarp();
     } else {
         // ================================ softmax =============================================
+        // One loop over all tiles; the phase only changes how a tile's key mask is formed, so
+        // the tile body, the epilogue and the top-k insertion each exist once in the code.
         const int t128 = tid - 64;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
@@ -343,52 +357,200 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             }
             return true;
         };
-        // O of the finished phase -> its destination (warp-collective TMEM reads)
-        auto epilogue = [&](int ph) {
-            tc::fence_after_sync();
-            const float f = row_ok ? gt[ph] / l : 0.0f;
+        float tv[KM];
+        int32_t ti[KM];
+#pragma unroll
+        for (int u = 0; u < KM; ++u) {
+            tv[u] = -INFINITY;
+            ti[u] = -1;
+        }
+        int ns = 0, nT = 1 << 30, ri = 0, nr = 0;
+        const uint64_t* wrow = P.wmask + (int64_t)wm0 * 128 + row;
+        uint64_t wnext = 0ull;
+        bool ok = true;
+        for (int j = 0;; ++j) {
+            // ---- phase boundaries: O of the finished phase to its destination ----------------
+            const int ph_end = j == nc ? 0 : (j == nc + ns && ns > 0 ? 1 : (j == nT ? 2 : -1));
+            if (ph_end >= 0) {
+                ok = __all_sync(0xffffffffu, ok && wait_pv(j - 1));
+                if (ok) {
+                    tc::fence_after_sync();
+                    const float f = row_ok ? gt[ph_end] / l : 0.0f;
+                    T* orow = reinterpret_cast<T*>(P.out) + ((int64_t)tok * H + h) * D;
 #pragma unroll 1
-            for (int d0 = 0; d0 < D; d0 += 32) {
-                float o[32];
-                tc::tmem_ld32(o_tm + d0, o);
-                if (!row_ok) continue;
-                if (ph < 2) {
+                    for (int d0 = 0; d0 < D; d0 += 32) {
+                        float o[32];
+                        tc::tmem_ld32(o_tm + d0, o);   // warp-collective
+                        if (!row_ok) continue;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        float4 v = make_float4(o[e] * f, o[e + 1] * f, o[e + 2] * f, o[e + 3] * f);
-                        if (ph == 1) {
-                            const float4 bb = *reinterpret_cast<const float4*>(brow + d0 + e);
-                            v.x += bb.x; v.y += bb.y; v.z += bb.z; v.w += bb.w;
+                        for (int e = 0; e < 32; e += 8) {
+                            float4 a = make_float4(o[e] * f, o[e + 1] * f, o[e + 2] * f, o[e + 3] * f);
+                            float4 c = make_float4(o[e + 4] * f, o[e + 5] * f, o[e + 6] * f, o[e + 7] * f);
+                            if (ph_end > 0) {
+                                const float4 a0 = *reinterpret_cast<const float4*>(brow + d0 + e);
+                                const float4 c0 = *reinterpret_cast<const float4*>(brow + d0 + e + 4);
+                                a.x += a0.x; a.y += a0.y; a.z += a0.z; a.w += a0.w;
+                                c.x += c0.x; c.y += c0.y; c.z += c0.z; c.w += c0.w;
+                            }
+                            if (ph_end < 2) {
+                                *reinterpret_cast<float4*>(brow + d0 + e) = a;
+                                *reinterpret_cast<float4*>(brow + d0 + e + 4) = c;
+                            } else {
+                                *reinterpret_cast<uint4*>(orow + d0 + e) =
+                                    make_uint4(pack2<T>(a.x, a.y), pack2<T>(a.z, a.w), pack2<T>(c.x, c.y),
+                                               pack2<T>(c.z, c.w));
+                            }
                         }
-                        *reinterpret_cast<float4*>(brow + d0 + e) = v;
-                    }
-                } else {
-                    T* orow = reinterpret_cast<T*>(P.out) + ((int64_t)tok * H + h) * D + d0;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        const float4 b0 = *reinterpret_cast<const float4*>(brow + d0 + e);
-                        const float4 b1 = *reinterpret_cast<const float4*>(brow + d0 + e + 4);
-                        *reinterpret_cast<uint4*>(orow + e) = make_uint4(
-                            pack2<T>(b0.x + o[e] * f, b0.y + o[e + 1] * f),
-                            pack2<T>(b0.z + o[e + 2] * f, b0.w + o[e + 3] * f),
-                            pack2<T>(b1.x + o[e + 4] * f, b1.y + o[e + 5] * f),
-                            pack2<T>(b1.z + o[e + 6] * f, b1.w + o[e + 7] * f));
                     }
                 }
+                m = -INFINITY;
+                l = 0.0f;
+                if (ph_end == 2) break;
             }
-        };
-        // one tile: S from TMEM buffer b, masked by `mask(s)`, then softmax bookkeeping, P to TMEM
-        auto step = [&](int j, bool first, auto&& mask) -> bool {
+            if (j == nc) {
+                // ---- selection, union of the selected blocks, this row's key ranges ----------
+                if (ok && row_ok) {
+                    int32_t* srow = P.sel + ((int64_t)pos * H + h) * ksel;
+                    srow[0] = ob;
+#pragma unroll
+                    for (int u = 0; u < KM; ++u)
+                        if (u + 1 < ksel) srow[u + 1] = ti[u];
+                }
+                uint32_t* words = reinterpret_cast<uint32_t*>(g + L::kK);
+                const int W = (nblk + 31) >> 5;
+                int32_t* wpre = reinterpret_cast<int32_t*>(words + W);
+                int* red = misc + M_RED;
+                for (int i = t128; i < W; i += 128) words[i] = 0u;
+                tc::named_sync(2, 128);
+                // own block, then the top-(k-1) (local block indices; -1 = none)
+                int32_t mine[L::kSlots];
+                mine[0] = row_ok ? ob - bl : -1;
+#pragma unroll
+                for (int u = 0; u < KM; ++u)
+                    mine[u + 1] = (row_ok && u + 1 < ksel && ti[u] >= 0) ? ti[u] - bl : -1;
+#pragma unroll
+                for (int a = 0; a < (int)L::kSlots; ++a)
+                    if (mine[a] >= 0 && mine[a] < nblk) atomicOr(&words[mine[a] >> 5], 1u << (mine[a] & 31));
+                tc::named_sync(2, 128);
+                // union index of every set bit: exclusive prefix of the word popcounts
+                const int cw = (W + 127) >> 7;
+                const int wl = min(t128 * cw, W), wh = min(wl + cw, W);
+                int cnt = 0;
+                for (int i = wl; i < wh; ++i) cnt += __popc(words[i]);
+                int U = 0;
+                int pre = scan128(cnt, t128, red, U);
+                U = min(U, (int)L::kUCap);
+                for (int i = wl; i < wh; ++i) {
+                    wpre[i] = pre;
+                    uint32_t wd = words[i];
+                    while (wd) {
+                        const int bit = __ffs(wd) - 1;
+                        wd &= wd - 1;
+                        if (pre < (int)L::kUCap) un[pre].x = 32 * i + bit;   // local block index
+                        ++pre;
+                    }
+                }
+                tc::named_sync(2, 128);
+                // first group and group count of every union block (independent loads)
+                for (int u = t128; u < U; u += 128) {
+                    const int32_t gb = bl + un[u].x;
+                    un[u] = make_int2(P.blk_poff[gb] >> 3, (P.blk_off[gb + 1] - P.blk_off[gb] + 7) >> 3);
+                }
+                tc::named_sync(2, 128);
+                // stream offsets (in groups): exclusive prefix of the blocks' group counts
+                const int cu = (U + 127) >> 7;
+                const int ul = min(t128 * cu, U), uh = min(ul + cu, U);
+                int ssum = 0;
+                for (int u = ul; u < uh; ++u) ssum += un[u].y;
+                int Lg = 0;
+                int off = scan128(ssum, t128, red, Lg);
+                for (int u = ul; u < uh; ++u) {
+                    const int n = un[u].y;
+                    un[u].y = off;
+                    off += n;
+                }
+                if (t128 == 0) {
+                    un[U] = make_int2(0, Lg);
+                    misc[M_U] = U;
+                    misc[M_L] = Lg;
+                }
+                tc::named_sync(2, 128);
+                // this row's ranges [first key, last key + 1) in the stream, ascending
+#pragma unroll
+                for (int a = 0; a < (int)L::kSlots; ++a) {
+                    if (mine[a] < 0 || mine[a] >= nblk) continue;
+                    int rank = 0;
+#pragma unroll
+                    for (int c = 0; c < (int)L::kSlots; ++c) rank += (mine[c] >= 0 && mine[c] < mine[a]) ? 1 : 0;
+                    const int wi = mine[a] >> 5;
+                    const int u = wpre[wi] + __popc(words[wi] & ((1u << (mine[a] & 31)) - 1u));
+                    const int32_t gb = bl + mine[a];
+                    if (u < U)
+                        rng[rank * 128 + row] = make_int2(8 * un[u].y, 8 * un[u].y + P.blk_off[gb + 1] - P.blk_off[gb]);
+                    ++nr;
+                }
+                tc::named_sync(1, kThreads);   // the producer may now overwrite the rings
+                ns = (misc[M_L] + 7) >> 3;
+                nT = nc + ns + nw;
+                if (nw > 0) wnext = wrow[0];
+            }
+            // after a wait ran out the tiles of phase C are skipped up to the union build, which
+            // every softmax thread must reach (its barriers have no time limit); then the CTA ends
+            if (!ok && j >= nc) break;
+            if (!ok) continue;
+            const int ph = j < nc ? 0 : (j < nc + ns ? 1 : 2);
+            const bool first = j == 0 || j == nc || j == nc + ns;
             const int b = j & 1;
-            if (!wait_or_flag(&bar[SFULL + b], (uint32_t)(j >> 1) & 1u, P.status, abort_flag)) return false;
+            // ---- the key mask of this tile -------------------------------------------------------
+            uint64_t vm = ~0ull;
+            if (ph == 0) {
+                // compressed tokens: the sequence's blocks [bl, bl + nblk); column 0 is block bbase
+                const int32_t bbase = 8 * cg0 + kKT * j;
+                vm = span_bits(bl - bbase, bl + nblk - bbase);
+            } else if (ph == 1) {
+                const int base = kKT * (j - nc);
+                vm = 0ull;
+                while (ri < nr) {
+                    const int2 rg = rng[ri * 128 + row];
+                    if (rg.x >= base + kKT) break;
+                    vm |= span_bits(rg.x - base, rg.y - base);
+                    if (rg.y > base + kKT) break;
+                    ++ri;
+                }
+            } else {
+                // the plan's window mask words, loaded one tile ahead
+                const int w = j - nc - ns;
+                vm = wnext;
+                if (w + 1 < nw) wnext = wrow[(int64_t)(w + 1) * 128];
+            }
+            // ---- S from TMEM buffer b ------------------------------------------------------------
+            ok = wait_or_flag(&bar[SFULL + b], (uint32_t)(j >> 1) & 1u, P.status, abort_flag);
             // Observe P V of tile j-2 (already complete: S of tile j was issued after it). Keeping
             // the observed count within one phase of the barriers keeps later parity waits exact.
-            if (j >= 2 && !wait_pv(j - 2)) return false;
+            if (ok && j >= 2) ok = wait_pv(j - 2);
+            if (!(ok = __all_sync(0xffffffffu, ok))) continue;
             tc::fence_after_sync();
             const uint32_t s_tm = tmem + lane_base + b * kKT;
             float s[64];
             tc::tmem_ld64(s_tm, s);
-            if (!mask(s)) return false;
+            apply_bits(s, vm);
+            if (ph == 0 && ksel > 1) {
+                // running top-(k-1) of the other blocks: candidates above the list's last entry,
+                // offered in ascending block order
+                const int32_t bbase = 8 * cg0 + kKT * j;
+                uint64_t cand = 0ull;
+                const float thr = tv[KM - 1];
+#pragma unroll
+                for (int e = 0; e < 64; ++e) cand |= (uint64_t)(s[e] > thr) << e;
+                while (cand) {
+                    const int e = __ffsll((long long)cand) - 1;
+                    cand &= cand - 1;
+                    const int32_t bi = bbase + e;
+                    const float z = pick64(s, e);
+                    if (bi != ob && z > tv[KM - 1]) topk_push<KM>(tv, ti, z, bi);
+                }
+            }
+            // ---- running max, lazy rescale, P = 2^(s*sl - m) ------------------------------------
             float mx[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[i], s[i + 8]);
@@ -411,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             }
             if (__any_sync(0xffffffffu, resc)) {
                 // O must hold P V of the previous tile before it is rescaled
-                if (!wait_pv(j - 1)) return false;
+                if (!(ok = __all_sync(0xffffffffu, wait_pv(j - 1)))) continue;
                 tc::fence_after_sync();
                 const float f = resc ? alpha : 1.0f;
 #pragma unroll 1
@@ -441,177 +603,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bar[PFULL + b]);
-            return true;
-        };
-
-        // ---- phase C: compressed tokens + top-(k-1) of the other blocks ----------------------
-        float tv[KM];
-        int32_t ti[KM];
-#pragma unroll
-        for (int u = 0; u < KM; ++u) {
-            tv[u] = -INFINITY;
-            ti[u] = -1;
         }
-        bool ok = true;
-        for (int j = 0; j < nc && ok; ++j) {
-            const int32_t bbase = 8 * cg0 + kKT * j;   // block index of column 0
-            const int lo = bl - bbase, hi = bl + nblk - bbase;
-            ok = step(j, j == 0, [&](float (&s)[64]) -> bool {
-                if (lo > 0 || hi < kKT) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        if (e < lo || e >= hi) s[e] = -INFINITY;
-                }
-                if (ksel > 1) {
-#pragma unroll
-                    for (int gq = 0; gq < 4; ++gq) {
-                        const float thr = tv[KM - 1];
-                        uint32_t cand = 0;
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) cand |= (uint32_t)(s[16 * gq + e] > thr) << e;
-                        while (cand) {
-                            const int e = __ffs(cand) - 1;
-                            cand &= cand - 1;
-                            const int32_t bi = bbase + 16 * gq + e;
-                            if (bi != ob) topk_push<KM>(tv, ti, pick16(s + 16 * gq, e), bi);
-                        }
-                    }
-                }
-                return true;
-            });
-        }
-        if (ok) ok = wait_pv(nc - 1);
-        if (ok) {
-            epilogue(0);
-            if (row_ok) {
-                int32_t* srow = P.sel + ((int64_t)pos * H + h) * ksel;
-                srow[0] = ob;
-#pragma unroll
-                for (int u = 0; u < KM; ++u)
-                    if (u + 1 < ksel) srow[u + 1] = ti[u];
-            }
-        }
-
-        // ---- union of the selected blocks and each row's key ranges ---------------------------
-        {
-            uint32_t* words = reinterpret_cast<uint32_t*>(g + L::kK);
-            const int W = (nblk + 31) >> 5;
-            int32_t* wpre = reinterpret_cast<int32_t*>(words + W);
-            int* red = misc + M_RED;
-            for (int i = t128; i < W; i += 128) words[i] = 0u;
-            tc::named_sync(2, 128);
-            // own block, then the top-(k-1) (local block indices; -1 = none)
-            int32_t mine[L::kSlots];
-            mine[0] = row_ok ? ob - bl : -1;
-#pragma unroll
-            for (int u = 0; u < KM; ++u)
-                mine[u + 1] = (row_ok && u + 1 < ksel && ti[u] >= 0) ? ti[u] - bl : -1;
-#pragma unroll
-            for (int a = 0; a < (int)L::kSlots; ++a)
-                if (mine[a] >= 0 && mine[a] < nblk) atomicOr(&words[mine[a] >> 5], 1u << (mine[a] & 31));
-            tc::named_sync(2, 128);
-            // union index of every set bit: exclusive prefix of the word popcounts
-            const int cw = (W + 127) >> 7;
-            const int wl = min(t128 * cw, W), wh = min(wl + cw, W);
-            int cnt = 0;
-            for (int i = wl; i < wh; ++i) cnt += __popc(words[i]);
-            int U = 0;
-            int pre = scan128(cnt, t128, red, U);
-            U = min(U, (int)L::kUCap);
-            for (int i = wl; i < wh; ++i) {
-                wpre[i] = pre;
-                uint32_t wd = words[i];
-                while (wd) {
-                    const int bit = __ffs(wd) - 1;
-                    wd &= wd - 1;
-                    if (pre < (int)L::kUCap) un[pre].x = 32 * i + bit;   // local block index
-                    ++pre;
-                }
-            }
-            tc::named_sync(2, 128);
-            // first group and group count of every union block (independent loads)
-            for (int u = t128; u < U; u += 128) {
-                const int32_t gb = bl + un[u].x;
-                un[u] = make_int2(P.blk_poff[gb] >> 3, (P.blk_off[gb + 1] - P.blk_off[gb] + 7) >> 3);
-            }
-            tc::named_sync(2, 128);
-            // stream offsets (in groups): exclusive prefix of the blocks' group counts
-            const int cu = (U + 127) >> 7;
-            const int ul = min(t128 * cu, U), uh = min(ul + cu, U);
-            int ssum = 0;
-            for (int u = ul; u < uh; ++u) ssum += un[u].y;
-            int Ltot = 0;
-            int off = scan128(ssum, t128, red, Ltot);
-            for (int u = ul; u < uh; ++u) {
-                const int n = un[u].y;
-                un[u].y = off;
-                off += n;
-            }
-            if (t128 == 0) {
-                un[U] = make_int2(0, Ltot);
-                misc[M_U] = U;
-                misc[M_L] = Ltot;
-            }
-            tc::named_sync(2, 128);
-            // this row's ranges, ascending (the union stream is in block order)
-#pragma unroll
-            for (int a = 0; a < (int)L::kSlots; ++a) {
-                if (mine[a] < 0 || mine[a] >= nblk) continue;
-                int rank = 0;
-#pragma unroll
-                for (int c = 0; c < (int)L::kSlots; ++c) rank += (mine[c] >= 0 && mine[c] < mine[a]) ? 1 : 0;
-                const int wi = mine[a] >> 5;
-                const int u = wpre[wi] + __popc(words[wi] & ((1u << (mine[a] & 31)) - 1u));
-                const int32_t gb = bl + mine[a];
-                if (u < U) rng[rank * 128 + row] = make_int2(8 * un[u].y, 8 * un[u].y + P.blk_off[gb + 1] - P.blk_off[gb]);
-            }
-        }
-        int nr = 0;
-#pragma unroll
-        for (int u = 0; u < KM; ++u) nr += (row_ok && u + 1 < ksel && ti[u] >= 0) ? 1 : 0;
-        nr += row_ok ? 1 : 0;
-        tc::named_sync(1, kThreads);   // the producer may now overwrite the rings
-        const int ns = (misc[M_L] + 7) >> 3;
-        const int nT = nc + ns + nw;
-
-        // ---- phase S: the selected blocks ------------------------------------------------------
-        m = -INFINITY;
-        l = 0.0f;
-        int ri = 0;
-        for (int j = nc; j < nc + ns && ok; ++j) {
-            const int base = kKT * (j - nc);
-            ok = step(j, j == nc, [&](float (&s)[64]) -> bool {
-                uint64_t vm = 0;
-                while (ri < nr) {
-                    const int2 rg = rng[ri * 128 + row];
-                    if (rg.x >= base + kKT) break;
-                    vm |= span_bits(rg.x - base, rg.y - base);
-                    if (rg.y > base + kKT) break;
-                    ++ri;
-                }
-                apply_bits(s, vm);
-                return true;
-            });
-        }
-        if (ok && ns > 0 && (ok = wait_pv(nc + ns - 1))) epilogue(1);
-
-        // ---- phase W: the window ---------------------------------------------------------------
-        // the plan's mask words: bit c of this row's word = key c of the tile within distance r;
-        // each is loaded one tile ahead
-        m = -INFINITY;
-        l = 0.0f;
-        const uint64_t* wrow = P.wmask + (int64_t)wm0 * 128 + row;
-        uint64_t wnext = nw > 0 ? wrow[0] : 0ull;
-        for (int j = nc + ns; j < nT && ok; ++j) {
-            const int w = j - nc - ns;
-            const uint64_t wcur = wnext;
-            if (w + 1 < nw) wnext = wrow[(int64_t)(w + 1) * 128];
-            ok = step(j, w == 0, [&](float (&s)[64]) -> bool {
-                apply_bits(s, wcur);
-                return true;
-            });
-        }
-        if (ok && nT > nc + ns && wait_pv(nT - 1)) epilogue(2);
     }
 
     tc::fence_before_sync();

@@ -55,7 +55,9 @@ struct FL {
     static constexpr uint32_t kV = kK + 2 * kTile;
     static constexpr uint32_t kUnion = kV + 2 * kTile;   // int2 [kUCap+1] (first group, stream group offset)
     static constexpr uint32_t kRange = kUnion + (kUCap + 1) * 8;   // int2 [kSlots][128] key ranges
-    static constexpr uint32_t kBar = kRange + kSlots * 128 * 8;
+    // during phase C the union and range area holds one 64-score tile per row (float4 [16][128])
+    static constexpr uint32_t kUREnd = kRange + kSlots * 128 * 8;
+    static constexpr uint32_t kBar = kUREnd > kUnion + 64u * 128u * 4u ? kUREnd : kUnion + 64u * 128u * 4u;
     static constexpr uint32_t kMisc = kBar + 16 * 8;
     static constexpr uint32_t kBytes = kMisc + 64;
     static constexpr uint32_t kAlloc = kBytes + 1024;
@@ -78,26 +80,6 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, int
     return false;
 }
 
-// v[e] for a per-thread index e in [0, 16), by a tree of selects (stays in registers)
-__device__ __forceinline__ float pick16(const float* v, int e) {
-    float a[8], b[4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) b[i] = (e & 2) ? a[2 * i + 1] : a[2 * i];
-    const float c0 = (e & 4) ? b[1] : b[0];
-    const float c1 = (e & 4) ? b[3] : b[2];
-    return (e & 8) ? c1 : c0;
-}
-
-// v[e] for a per-thread index e in [0, 64): a select tree within each 16-group, then across groups
-__device__ __forceinline__ float pick64(const float (&v)[64], int e) {
-    const float g0 = pick16(v, e & 15), g1 = pick16(v + 16, e & 15);
-    const float g2 = pick16(v + 32, e & 15), g3 = pick16(v + 48, e & 15);
-    const float lo = (e & 16) ? g1 : g0, hi = (e & 16) ? g3 : g2;
-    return (e & 32) ? hi : lo;
-}
-
 // Bits [a, b) of a 64-bit word, a and b clamped to [0, 64].
 __device__ __forceinline__ uint64_t span_bits(int a, int b) {
     a = max(a, 0);
@@ -105,6 +87,13 @@ __device__ __forceinline__ uint64_t span_bits(int a, int b) {
     if (a >= b) return 0ull;
     const uint64_t hi = b >= 64 ? ~0ull : ((1ull << b) - 1ull);
     return hi & (~0ull << a);
+}
+
+// *p += v (four fp32 lanes, one vector reduction; p 16-byte aligned; no value returned)
+__device__ __forceinline__ void red_add4(float* p, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
 }
 
 // s[c] = -inf where bit c of vm is clear
@@ -386,15 +375,19 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                         for (int e = 0; e < 32; e += 8) {
                             float4 a = make_float4(o[e] * f, o[e + 1] * f, o[e + 2] * f, o[e + 3] * f);
                             float4 c = make_float4(o[e + 4] * f, o[e + 5] * f, o[e + 6] * f, o[e + 7] * f);
-                            if (ph_end > 0) {
+                            if (ph_end == 2) {
                                 const float4 a0 = *reinterpret_cast<const float4*>(brow + d0 + e);
                                 const float4 c0 = *reinterpret_cast<const float4*>(brow + d0 + e + 4);
                                 a.x += a0.x; a.y += a0.y; a.z += a0.z; a.w += a0.w;
                                 c.x += c0.x; c.y += c0.y; c.z += c0.z; c.w += c0.w;
                             }
-                            if (ph_end < 2) {
+                            if (ph_end == 0) {
                                 *reinterpret_cast<float4*>(brow + d0 + e) = a;
                                 *reinterpret_cast<float4*>(brow + d0 + e + 4) = c;
+                            } else if (ph_end == 1) {
+                                // added without reading back (no load latency on this thread)
+                                red_add4(brow + d0 + e, a);
+                                red_add4(brow + d0 + e + 4, c);
                             } else {
                                 *reinterpret_cast<uint4*>(orow + d0 + e) =
                                     make_uint4(pack2<T>(a.x, a.y), pack2<T>(a.z, a.w), pack2<T>(c.x, c.y),
@@ -533,24 +526,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             const uint32_t s_tm = tmem + lane_base + b * kKT;
             float s[64];
             tc::tmem_ld64(s_tm, s);
-            apply_bits(s, vm);
-            if (ph == 0 && ksel > 1) {
-                // running top-(k-1) of the other blocks: candidates above the list's last entry,
-                // offered in ascending block order
-                const int32_t bbase = 8 * cg0 + kKT * j;
-                uint64_t cand = 0ull;
-                const float thr = tv[KM - 1];
-#pragma unroll
-                for (int e = 0; e < 64; ++e) cand |= (uint64_t)(s[e] > thr) << e;
-                while (cand) {
-                    const int e = __ffsll((long long)cand) - 1;
-                    cand &= cand - 1;
-                    const int32_t bi = bbase + e;
-                    const float z = pick64(s, e);
-                    if (bi != ob && z > tv[KM - 1]) topk_push<KM>(tv, ti, z, bi);
-                }
-            }
-            // ---- running max, lazy rescale, P = 2^(s*sl - m) ------------------------------------
+            if (__any_sync(0xffffffffu, vm != ~0ull)) apply_bits(s, vm);
             float mx[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[i], s[i + 8]);
@@ -561,6 +537,30 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             }
             const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            if (ph == 0 && ksel > 1 && tmax > tv[KM - 1]) {
+                // running top-(k-1) of the other blocks: candidates above the list's last entry,
+                // offered in ascending block order; the row's scores go to shared memory
+                // (quad q of row r at float4 index q * 128 + r) so a candidate is one load
+                const int32_t bbase = 8 * cg0 + kKT * j;
+                float4* srow4 = reinterpret_cast<float4*>(g + L::kUnion) + row;
+                const float* srow1 = reinterpret_cast<const float*>(srow4);
+                uint64_t cand = 0ull;
+                const float thr = tv[KM - 1];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    srow4[q * 128] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) cand |= (uint64_t)(s[4 * q + i] > thr) << (4 * q + i);
+                }
+                while (cand) {
+                    const int e = __ffsll((long long)cand) - 1;
+                    cand &= cand - 1;
+                    const int32_t bi = bbase + e;
+                    const float z = srow1[(e >> 2) * 512 + (e & 3)];
+                    if (bi != ob && z > tv[KM - 1]) topk_push<KM>(tv, ti, z, bi);
+                }
+            }
+            // ---- running max, lazy rescale, P = 2^(s*sl - m) ------------------------------------
             const float tm = tmax * sl;
             bool resc = false;
             float alpha = 1.0f;

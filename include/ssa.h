@@ -188,6 +188,29 @@ SSA_API ssa_status_t ssa_plan_destroy(ssa_plan_t plan);
 /* Static description of a status code. */
 SSA_API const char* ssa_status_string(ssa_status_t status);
 
+/*
+ * Block offsets of one sequence without allocating device memory. The method has no counterpart
+ * of this call: it is a convenience for callers that must not allocate (for example while other
+ * work owns the allocator). It computes what the plan's block partition yields as blk_off: the
+ * CSR token offsets of the occupied 8^3 blocks in block-key order (x-block major, then y, then z).
+ *   coords:            device int32 [n, 3] voxel coordinates, n >= 1.
+ *   grid:              host int32[3] grid extent, each in 1..65535.
+ *   blk_off:           device int32 [blk_off_capacity]; receives n_blocks + 1 offsets
+ *                      (blk_off[n_blocks] = number of tokens).
+ *   blk_off_capacity:  must be >= min(n, number of grid blocks) + 1.
+ *   n_blocks:          device int32 scalar; receives the number of occupied blocks, or -1 if a
+ *                      coordinate lies outside the grid.
+ * Scratch is one fixed device array inside the library (16.8 MB, enough for grids of up to
+ * 2^21 blocks of 8^3 cells, i.e. 1024^3 cells). Each call clears what it uses first; nothing has
+ * to start at zero. Calls that overlap in time share the array and race: serialise them (one
+ * stream, or ordered with events). The first call on a device looks up the array's address.
+ * Errors: SSA_ERR_INVALID_ARG (null pointer, n < 1, grid out of range, capacity too small),
+ * SSA_ERR_UNSUPPORTED (more than 2^21 grid blocks), SSA_ERR_CUDA. Asynchronous on `stream`.
+ */
+SSA_API ssa_status_t ssa_block_offsets_noalloc(const int32_t* coords, int64_t n, const int32_t* grid,
+                                               int32_t* blk_off, int64_t blk_off_capacity,
+                                               int32_t* n_blocks, void* stream);
+
 /* Number of kernels this library has launched in the process so far. */
 SSA_API int64_t ssa_launch_count(void);
 

@@ -38,6 +38,7 @@ _vp = ctypes.c_void_p
 _i32, _i64 = ctypes.c_int32, ctypes.c_int64
 _SIGS = {
     "ssa_set_allocator": [_vp, _vp, _vp],
+    "ssa_block_offsets_noalloc": [_vp, _i64, _vp, _vp, _i64, _vp, _vp],
     "ssa_plan": [_vp, _i64, _vp, _i32, _i32, _vp, _vp],
     "ssa_plan_varlen": [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp],
     "ssa_plan_rebuild": [_vp, _vp, _vp],
@@ -77,6 +78,26 @@ lib = _load()
 def declared_symbols() -> Sequence[str]:
     """Entry points declared in include/ssa.h."""
     return re.findall(r"SSA_API\s+[\w\s\*]+?\b(ssa_\w+)\s*\(", open(HEADER).read())
+
+
+def block_offsets_noalloc(coords: torch.Tensor, grid, stream=None):
+    """ssa_block_offsets_noalloc: CSR token offsets of the occupied 8^3 blocks of one sequence,
+    computed in the library's fixed scratch (no device allocation by the library). Returns
+    (blk_off [n_blocks + 1] int32 on the device, n_blocks); n_blocks is -1 if a coordinate lies
+    outside the grid."""
+    c = _dev(coords, torch.int32)
+    n = c.shape[0]
+    g = (ctypes.c_int32 * 3)(*[int(x) for x in grid])
+    nb = 1
+    for x in grid:
+        nb *= (int(x) + 7) // 8
+    cap = min(n, nb) + 1
+    blk_off = torch.empty(cap, dtype=torch.int32, device=c.device)
+    nblk = torch.empty(1, dtype=torch.int32, device=c.device)
+    _check(lib.ssa_block_offsets_noalloc(c.data_ptr(), n, g, blk_off.data_ptr(), cap, nblk.data_ptr(),
+                                         _stream(stream)), "ssa_block_offsets_noalloc")
+    k = int(nblk.item())
+    return (blk_off[:k + 1] if k >= 0 else blk_off[:0]), k
 
 
 def launch_count() -> int:

@@ -137,6 +137,16 @@ def algorithmic_flops(plan, sel, cfg, cu):
                                                         "selected_other": other, "window": win}}
 
 
+def max_over_ranks(ms: float, dist, device: str) -> float:
+    """The step time of the slowest rank (every rank calls this once, in the same order)."""
+    if not dist:
+        return ms
+    import torch
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
 def run_ours(args, rank, world, dist):
     import torch
     import spatial_sparse_attention_b200 as ssa
@@ -197,11 +207,7 @@ def run_ours(args, rank, world, dist):
     prof = ssa.profile_read()
     if plan.status() != 0:
         raise RuntimeError("device status set during the timed steps")
-    ms = e0.elapsed_time(e1) / args.steps
-    if dist:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, "cuda")
     clk = clocks.stop() if rank == 0 else None
 
     # end to end through the host-buffer entry point (pinned host memory, copies inside)

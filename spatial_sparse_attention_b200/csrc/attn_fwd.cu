@@ -354,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             ti[u] = -1;
         }
         int ns = 0, nT = 1 << 30, ri = 0, nr = 0;
+        int2 rcur = make_int2(0x7fffffff, 0x7fffffff);
         const uint64_t* wrow = P.wmask + (int64_t)wm0 * 128 + row;
         uint64_t wnext = 0ull;
         bool ok = true;
@@ -483,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                     ++nr;
                 }
                 tc::named_sync(1, kThreads);   // the producer may now overwrite the rings
+                rcur = nr > 0 ? rng[row] : make_int2(0x7fffffff, 0x7fffffff);
                 ns = (misc[M_L] + 7) >> 3;
                 nT = nc + ns + nw;
                 if (nw > 0) wnext = wrow[0];
@@ -501,14 +503,14 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                 const int32_t bbase = 8 * cg0 + kKT * j;
                 vm = span_bits(bl - bbase, bl + nblk - bbase);
             } else if (ph == 1) {
+                // this row's ranges in ascending order; the current one is kept in registers
                 const int base = kKT * (j - nc);
                 vm = 0ull;
-                while (ri < nr) {
-                    const int2 rg = rng[ri * 128 + row];
-                    if (rg.x >= base + kKT) break;
-                    vm |= span_bits(rg.x - base, rg.y - base);
-                    if (rg.y > base + kKT) break;
+                while (rcur.x < base + kKT) {
+                    vm |= span_bits(rcur.x - base, rcur.y - base);
+                    if (rcur.y > base + kKT) break;
                     ++ri;
+                    rcur = ri < nr ? rng[ri * 128 + row] : make_int2(0x7fffffff, 0x7fffffff);
                 }
             } else {
                 // the plan's window mask words, loaded one tile ahead

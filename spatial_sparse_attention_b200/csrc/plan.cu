@@ -371,42 +371,55 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
 }
 
 // Runs of consecutive 8-row groups that cover each tile's window union (the attention kernel
-// loads every run with one bulk copy). One lane per tile walks the ascending rows.
-// kFill == false writes the run and group counts, kFill == true the runs at wr_off.
+// loads every run with one bulk copy). One warp per tile walks the ascending rows 32 at a time:
+// a row opens a group when its group differs from the previous row's, and a group opens a run
+// when it does not follow the previous group. kFill == false writes the run and group counts;
+// kFill == true writes each run (first group, groups) at wr_off.
 template <bool kFill>
 __global__ void k_window_runs(int64_t T, const int32_t* __restrict__ wt_off,
                               const int32_t* __restrict__ wt_keys, int32_t* __restrict__ wr_cnt,
                               int32_t* __restrict__ wg_cnt, int32_t* __restrict__ wm_cnt,
                               const int32_t* __restrict__ wr_off, int2* __restrict__ runs) {
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
     const int32_t a = wt_off[t], b = wt_off[t + 1];
-    int32_t nr = 0, ng = 0, first = -1, cnt = 0, prev = -2;
     const int32_t out = kFill ? wr_off[t] : 0;
-    for (int32_t i = a; i < b; ++i) {
-        const int32_t gi = wt_keys[i] >> 3;
-        if (gi == prev) continue;
-        ++ng;
-        if (gi == prev + 1) {
-            ++cnt;
-        } else {
-            if (first >= 0) {
-                if (kFill) runs[out + nr] = make_int2(first, cnt);
-                ++nr;
-            }
-            first = gi;
-            cnt = 1;
+    int32_t nr = 0, ng = 0, carry = -2;
+    for (int32_t c = a; c < b; c += 32) {
+        const int32_t i = c + lane;
+        const bool valid = i < b;
+        const int32_t gi = valid ? (wt_keys[i] >> 3) : 0x7fffffff;
+        int32_t prev = __shfl_up_sync(0xffffffffu, gi, 1);
+        if (lane == 0) prev = carry;
+        const bool new_group = valid && gi != prev;
+        const bool new_run = new_group && gi != prev + 1;
+        const unsigned bg = __ballot_sync(0xffffffffu, new_group);
+        const unsigned br = __ballot_sync(0xffffffffu, new_run);
+        if (kFill && new_run) {
+            // first group and, for now, the run's position in the group stream
+            runs[out + nr + __popc(br & ((1u << lane) - 1u))] = make_int2(gi, ng + __popc(bg & ((1u << lane) - 1u)));
         }
-        prev = gi;
-    }
-    if (first >= 0) {
-        if (kFill) runs[out + nr] = make_int2(first, cnt);
-        ++nr;
+        nr += __popc(br);
+        ng += __popc(bg);
+        const int last = min(31, b - 1 - c);
+        carry = __shfl_sync(0xffffffffu, gi, last);
     }
     if (!kFill) {
-        wr_cnt[t] = nr;
-        wg_cnt[t] = ng;
-        wm_cnt[t] = (ng + 7) >> 3;
+        if (lane == 0) {
+            wr_cnt[t] = nr;
+            wg_cnt[t] = ng;
+            wm_cnt[t] = (ng + 7) >> 3;
+        }
+        return;
+    }
+    __syncwarp();
+    // group count of every run: the next run's stream position minus its own
+    for (int32_t r = lane; r < nr; r += 32) {
+        const int32_t nxt = r + 1 < nr ? runs[out + r + 1].y : ng;
+        const int32_t cnt = nxt - runs[out + r].y;
+        __syncwarp(__activemask());
+        runs[out + r].y = cnt;
     }
 }
 
@@ -612,8 +625,8 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     SSA_ALLOC(p->wr_off, int32_t, T + 1);
     SSA_ALLOC(p->wg_cnt, int32_t, T);
     SSA_ALLOC(p->wm_off, int32_t, T + 1);
-    k_window_runs<false><<<(unsigned)cdiv(T, 128), 128, 0, st>>>(T, p->wt_off, p->wt_keys, wr_cnt,
-                                                                  p->wg_cnt, wm_cnt, nullptr, nullptr);
+    k_window_runs<false><<<(unsigned)cdiv(T, 4), 128, 0, st>>>(T, p->wt_off, p->wt_keys, wr_cnt,
+                                                                p->wg_cnt, wm_cnt, nullptr, nullptr);
     note_launch();
     scan_exclusive(wr_cnt, p->wr_off, T, tmp, st);
     scan_exclusive(wm_cnt, p->wm_off, T, tmp, st);
@@ -634,8 +647,8 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         return SSA_ERR_CUDA;
     SSA_ALLOC(p->wr_runs, int2, n_runs);
     SSA_ALLOC(p->wmask, uint64_t, (int64_t)n_wtiles * kQTile);
-    k_window_runs<true><<<(unsigned)cdiv(T, 128), 128, 0, st>>>(T, p->wt_off, p->wt_keys, nullptr,
-                                                                 nullptr, nullptr, p->wr_off, p->wr_runs);
+    k_window_runs<true><<<(unsigned)cdiv(T, 4), 128, 0, st>>>(T, p->wt_off, p->wt_keys, nullptr,
+                                                               nullptr, nullptr, p->wr_off, p->wr_runs);
     k_window_masks<<<(unsigned)T, kQTile, 0, st>>>(p->qt_pos, p->qt_len, p->perm, p->coords, p->wr_off,
                                                    p->wr_runs, p->wm_off, p->scoord, r, p->wmask);
     note_launch(2);

@@ -259,7 +259,7 @@ ssa_status_t ensure_workspace(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int
         w.vs = A(es * H * p->Npad * D);
         w.kcg = A(es * H * w.Mb8 * D);
         w.vcg = A(es * H * w.Mb8 * D);
-        w.base = (float*)A(sizeof(float) * N * H * D);
+        w.base = (float*)A(sizeof(float) * p->n_qtiles * kQTile * H * D);
         if (!w.ks || !w.vs || !w.kcg || !w.vcg || !w.base) return SSA_ERR_ALLOC;
         // padding rows of the block-ordered copies stay zero for the life of the workspace
         if (cudaMemsetAsync(w.ks, 0, es * H * p->Npad * D, st) ||

@@ -333,7 +333,9 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
         const int32_t tok = P.perm[pos];
         const int32_t ob = P.tok_blk[tok];
         const float* gt = P.gates + ((int64_t)tok * H + h) * 3;
-        float* brow = P.base + ((int64_t)pos * H + h) * D;
+        // the fp32 row buffer of this (query tile, head): [D/4][128 rows][4] so that a warp's
+        // 16-byte accesses to one column quad cover 512 contiguous bytes
+        float* brow = P.base + ((int64_t)tile * H + h) * 128 * D + row * 4;
         const float sl = P.sl;
         const int ksel = P.k;
         float m = -INFINITY, l = 0.0f;
@@ -376,19 +378,20 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                         for (int e = 0; e < 32; e += 8) {
                             float4 a = make_float4(o[e] * f, o[e + 1] * f, o[e + 2] * f, o[e + 3] * f);
                             float4 c = make_float4(o[e + 4] * f, o[e + 5] * f, o[e + 6] * f, o[e + 7] * f);
+                            float* bq = brow + (d0 + e) * 128;   // column quad (d0+e)/4, this row
                             if (ph_end == 2) {
-                                const float4 a0 = *reinterpret_cast<const float4*>(brow + d0 + e);
-                                const float4 c0 = *reinterpret_cast<const float4*>(brow + d0 + e + 4);
+                                const float4 a0 = *reinterpret_cast<const float4*>(bq);
+                                const float4 c0 = *reinterpret_cast<const float4*>(bq + 512);
                                 a.x += a0.x; a.y += a0.y; a.z += a0.z; a.w += a0.w;
                                 c.x += c0.x; c.y += c0.y; c.z += c0.z; c.w += c0.w;
                             }
                             if (ph_end == 0) {
-                                *reinterpret_cast<float4*>(brow + d0 + e) = a;
-                                *reinterpret_cast<float4*>(brow + d0 + e + 4) = c;
+                                *reinterpret_cast<float4*>(bq) = a;
+                                *reinterpret_cast<float4*>(bq + 512) = c;
                             } else if (ph_end == 1) {
                                 // added without reading back (no load latency on this thread)
-                                red_add4(brow + d0 + e, a);
-                                red_add4(brow + d0 + e + 4, c);
+                                red_add4(bq, a);
+                                red_add4(bq + 512, c);
                             } else {
                                 *reinterpret_cast<uint4*>(orow + d0 + e) =
                                     make_uint4(pack2<T>(a.x, a.y), pack2<T>(a.z, a.w), pack2<T>(c.x, c.y),

@@ -49,7 +49,7 @@ struct Workspace {
     void* kcg = nullptr;       // [H, Mb8, D]  T   compressed tokens in the grouped order (16-bit path)
     void* vcg = nullptr;       // [H, Mb8, D]
     int64_t Mb8 = 0;           // Mb rounded up to a multiple of 8
-    float* base = nullptr;     // [N, H, D]    running g0*o_cmp + g1*o_sel, sorted token order
+    float* base = nullptr;     // [query tiles, H, D/4, 128, 4] running g0*o_cmp + g1*o_sel
     int32_t* sel = nullptr;    // [N, H, k]        selected blocks, sorted token order
     // host-buffer entry point staging (allocated on first use)
     void* h_q = nullptr; void* h_k = nullptr; void* h_v = nullptr; void* h_out = nullptr;

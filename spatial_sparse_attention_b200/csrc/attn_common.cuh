@@ -23,6 +23,7 @@ struct FwdParams {
     const int32_t* tok_blk;
     const int32_t* blk_off;
     const int32_t* blk_poff;
+    const int2* blk_info;     // (first 8-row group, tokens) per block
     const int4* scoord;
     const int32_t* qt_pos;
     const int32_t* qt_len;

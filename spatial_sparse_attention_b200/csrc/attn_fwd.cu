@@ -450,8 +450,8 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                 tc::named_sync(2, 128);
                 // first group and group count of every union block (independent loads)
                 for (int u = t128; u < U; u += 128) {
-                    const int32_t gb = bl + un[u].x;
-                    un[u] = make_int2(P.blk_poff[gb] >> 3, (P.blk_off[gb + 1] - P.blk_off[gb] + 7) >> 3);
+                    const int2 bi = P.blk_info[bl + un[u].x];
+                    un[u] = make_int2(bi.x, (bi.y + 7) >> 3);
                 }
                 tc::named_sync(2, 128);
                 // stream offsets (in groups): exclusive prefix of the blocks' group counts
@@ -481,9 +481,8 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                     for (int c = 0; c < (int)L::kSlots; ++c) rank += (mine[c] >= 0 && mine[c] < mine[a]) ? 1 : 0;
                     const int wi = mine[a] >> 5;
                     const int u = wpre[wi] + __popc(words[wi] & ((1u << (mine[a] & 31)) - 1u));
-                    const int32_t gb = bl + mine[a];
                     if (u < U)
-                        rng[rank * 128 + row] = make_int2(8 * un[u].y, 8 * un[u].y + P.blk_off[gb + 1] - P.blk_off[gb]);
+                        rng[rank * 128 + row] = make_int2(8 * un[u].y, 8 * un[u].y + P.blk_info[bl + mine[a]].y);
                     ++nr;
                 }
                 tc::named_sync(1, kThreads);   // the producer may now overwrite the rings
@@ -683,6 +682,7 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.tok_blk = p->tok_blk;
     P.blk_off = p->blk_off;
     P.blk_poff = p->blk_poff;
+    P.blk_info = p->blk_info;
     P.scoord = p->scoord;
     P.qt_pos = p->qt_pos;
     P.qt_len = p->qt_len;

@@ -83,6 +83,7 @@ struct Plan {
     int32_t* tok_pos = nullptr;  // [N]  position in perm
     int32_t* blk_off = nullptr;  // [Mb+1]
     int32_t* blk_poff = nullptr; // [Mb+1] padded row offsets
+    int2* blk_info = nullptr;    // [Mb] (first 8-row group of the padded rows, tokens)
     int32_t* blk_coord = nullptr;// [Mb,3]
     int32_t* blk_seq = nullptr;  // [Mb]
     int32_t* seq_blk_d = nullptr;// [B+1]

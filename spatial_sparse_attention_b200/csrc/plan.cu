@@ -230,6 +230,13 @@ __global__ void k_positions(const int32_t* __restrict__ perm, const int32_t* __r
     scoord[sp] = make_int4(coords[3 * i], coords[3 * i + 1], coords[3 * i + 2], b);
 }
 
+// (first 8-row group, tokens) of every block, for the attention kernel's union of selected blocks
+__global__ void k_block_info(const int32_t* __restrict__ blk_off, const int32_t* __restrict__ blk_poff,
+                             int64_t Mb, int2* __restrict__ info) {
+    const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < Mb) info[b] = make_int2(blk_poff[b] >> 3, blk_off[b + 1] - blk_off[b]);
+}
+
 __global__ void k_fill_i32(int32_t* __restrict__ a, int64_t n, int32_t v) {
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) a[i] = v;
@@ -567,6 +574,9 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     SSA_ALLOC(p->tok_pos, int32_t, N);
     SSA_ALLOC(p->spos_tok, int32_t, p->Npad);
     SSA_ALLOC(p->scoord, int4, p->Npad);
+    SSA_ALLOC(p->blk_info, int2, p->Mb);
+    k_block_info<<<grid_for(p->Mb), kThreads, 0, st>>>(p->blk_off, p->blk_poff, p->Mb, p->blk_info);
+    note_launch();
     k_scatter<<<grid_for(N), kThreads, 0, st>>>(tok_key, key2blk, N, p->blk_off, blk_fill, p->perm,
                                                 p->tok_blk);
     k_sort_blocks<<<grid_for(p->Mb, 8), 256, 0, st>>>(p->perm, p->blk_off, p->Mb);

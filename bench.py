@@ -42,7 +42,41 @@ def parse():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(workloads.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many heads instead of the config's "
+                         "(a smaller cut for profiling; 0 = the config's own)")
     return ap.parse_args()
+
+
+def config_of(args):
+    import dataclasses
+    cfg = workloads.CONFIGS[args.config]
+    return dataclasses.replace(cfg, H=args.heads) if args.heads > 0 else cfg
+
+
+# DRAM bytes per head of one k_ssa_fwd launch on the pass3 workload, read from one ncu capture
+# (profiles/k_ssa_fwd_pass3_h4.md: dram__bytes_read.sum + dram__bytes_write.sum of the 4-head cut,
+# divided by 4; the launch's traffic grows in proportion to the heads). Valid only for the kernel
+# sources the capture was taken with.
+KERNEL_TRAFFIC = {"sources_sha256": "5157c3a1460df167e10e1b126b96c11b99ab685a78aada9aa4abdc8bdf7441b8",
+                  "config": "pass3", "bytes_per_head": 633601536.0 / 4}
+KERNEL_SOURCES = ("attn_fwd.cu", "attn_common.cuh", "tc.cuh")
+
+
+def kernel_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "spatial_sparse_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def kernel_traffic(cfg_name, H):
+    t = KERNEL_TRAFFIC
+    if t["bytes_per_head"] is None or cfg_name != t["config"] or kernel_sources_sha256() != t["sources_sha256"]:
+        return None
+    return t["bytes_per_head"] * H
 
 
 def describe(cfg, coords, cu):
@@ -151,7 +185,7 @@ def run_ours(args, rank, world, dist):
     import torch
     import spatial_sparse_attention_b200 as ssa
 
-    cfg = workloads.CONFIGS[args.config]
+    cfg = config_of(args)
     coords, cu, grids = workloads.make_coords(cfg)
     t = workloads.make_tensors(cfg, len(coords))
     dev = {k: v.cuda() for k, v in t.items()}
@@ -251,7 +285,8 @@ def run_ours(args, rank, world, dist):
         "forward_only": {"ms": fwd_ms, "tokens_per_s": N / (fwd_ms * 1e-3),
                          "tflops": work["total"] / (fwd_ms * 1e-3) / 1e12},
         "roofline": {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak,
-                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": kernel_traffic(args.config, cfg.H),
+                     "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
                      "algorithmic_tflop_per_launch": work[dominant] / 1e12,
                      "avg_launch_ms": dom_ms, "peak_source": src},
         "e2e": {"value": N / (e2e * 1e-3), "unit": "tokens/s", "ms_per_step": e2e,
@@ -299,7 +334,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     import oracle
-    cfg = workloads.CONFIGS[args.config]
+    cfg = config_of(args)
     coords, cu, grids = workloads.make_coords(cfg)
     t = workloads.make_tensors(cfg, len(coords))
     N = len(coords)

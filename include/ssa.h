@@ -116,7 +116,9 @@ SSA_API ssa_status_t ssa_plan_varlen(const int32_t* coords, const int64_t* cu_se
 SSA_API ssa_status_t ssa_plan_rebuild(ssa_plan_t plan, const int32_t* coords, void* stream);
 
 /* Sizes of a plan (host outputs; any may be NULL): tokens, occupied blocks, total neighbour
- * list length, number of sequences. */
+ * list length, number of sequences. The per-token neighbour lists are not needed by the 16-bit
+ * forward, so they are counted on first request: asking for nnz may launch a kernel on the
+ * plan's stream and wait for it. */
 SSA_API ssa_status_t ssa_plan_info(ssa_plan_t plan, int64_t* n, int64_t* num_blocks, int64_t* nnz,
                            int32_t* batch);
 

@@ -167,10 +167,7 @@ class Plan:
             _check(lib.ssa_plan_varlen(coords.data_ptr(), ctypes.addressof(cu), B,
                                        ctypes.addressof(gr), block, r, st, ctypes.byref(self._h)),
                    "ssa_plan_varlen")
-        n, mb, nnz, b = _i64(), _i64(), _i64(), _i32()
-        _check(lib.ssa_plan_info(self._h, ctypes.byref(n), ctypes.byref(mb), ctypes.byref(nnz),
-                                 ctypes.byref(b)), "ssa_plan_info")
-        self.N, self.num_blocks, self.nnz, self.batch = n.value, mb.value, nnz.value, b.value
+        self._sizes()
         self.r = r
 
     def rebuild(self, coords: torch.Tensor):
@@ -178,11 +175,21 @@ class Plan:
         _dev(coords, torch.int32)
         _check(lib.ssa_plan_rebuild(self._h, coords.data_ptr(), _stream(self.stream)),
                "ssa_plan_rebuild")
-        n, mb, nnz, b = _i64(), _i64(), _i64(), _i32()
-        _check(lib.ssa_plan_info(self._h, ctypes.byref(n), ctypes.byref(mb), ctypes.byref(nnz),
-                                 ctypes.byref(b)), "ssa_plan_info")
-        self.N, self.num_blocks, self.nnz, self.batch = n.value, mb.value, nnz.value, b.value
+        self._sizes()
         return self
+
+    def _sizes(self):
+        n, mb, b = _i64(), _i64(), _i32()
+        _check(lib.ssa_plan_info(self._h, ctypes.byref(n), ctypes.byref(mb), None, ctypes.byref(b)),
+               "ssa_plan_info")
+        self.N, self.num_blocks, self.batch = n.value, mb.value, b.value
+
+    @property
+    def nnz(self) -> int:
+        """Total length of the per-token window neighbour lists (counted on first request)."""
+        v = _i64()
+        _check(lib.ssa_plan_info(self._h, None, None, ctypes.byref(v), None), "ssa_plan_info")
+        return v.value
 
     def close(self):
         if self._h:

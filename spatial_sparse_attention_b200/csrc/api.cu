@@ -383,7 +383,11 @@ ssa_status_t ssa_plan_info(ssa_plan_t plan, int64_t* n, int64_t* num_blocks, int
     if (!plan) return SSA_ERR_INVALID_ARG;
     if (n) *n = plan->N;
     if (num_blocks) *num_blocks = plan->Mb;
-    if (nnz) *nnz = plan->nnz;
+    if (nnz) {
+        const ssa_status_t rc = ensure_neighbour_counts(plan, plan->stream);
+        if (rc != SSA_OK) return rc;
+        *nnz = plan->nnz;
+    }
     if (batch) *batch = plan->B;
     return SSA_OK;
 }
@@ -394,8 +398,8 @@ ssa_status_t ssa_plan_export(ssa_plan_t p, int32_t* perm, int32_t* tok_blk, int3
     if (!p) return SSA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const auto D2D = cudaMemcpyDeviceToDevice;
-    if (nbr_idx) {
-        const ssa_status_t rc = ensure_neighbours(p, st);
+    if (nbr_idx || nbr_off) {
+        const ssa_status_t rc = nbr_idx ? ensure_neighbours(p, st) : ensure_neighbour_counts(p, st);
         if (rc != SSA_OK) return rc;
     }
     cudaError_t e = cudaSuccess;

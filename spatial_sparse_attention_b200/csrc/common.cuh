@@ -70,7 +70,7 @@ struct Plan {
     int64_t G = 0;       // dense block keys over all sequences
     int64_t Mb = 0;      // occupied blocks
     int64_t Npad = 0;    // padded sorted rows
-    int64_t nnz = 0;     // window neighbour pairs
+    int64_t nnz = -1;    // window neighbour pairs (-1 until counted on first use)
     int64_t n_qtiles = 0;
     std::vector<SeqInfo> seqs;
     std::vector<int64_t> seq_blk;   // [B+1] block range of each sequence (host copy)
@@ -152,7 +152,9 @@ void scan_exclusive(const int32_t* in, int32_t* out, int64_t n, int32_t* tmp, cu
 
 // plan.cu
 ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t s);
-// the per-token window neighbour lists (nbr_idx), built once per plan on first use
+// the per-token window neighbour counts (nbr_off32, nnz) and lists (nbr_idx), built once per plan
+// on first use (fp32 forward, backward, export, size query)
+ssa_status_t ensure_neighbour_counts(Plan* p, cudaStream_t s);
 ssa_status_t ensure_neighbours(Plan* p, cudaStream_t s);
 
 // pool.cu

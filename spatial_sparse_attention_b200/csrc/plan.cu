@@ -500,7 +500,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     while (hsize < (uint64_t)(2 * N)) hsize <<= 1;
     int64_t tmp_len = scan_tmp_len(std::max<int64_t>(G, N) + 1);
 
-    int32_t *tok_key, *key_cnt, *bidx, *key2blk, *blk_cnt, *blk_pcnt, *nbr_cnt, *tmp, *blk_fill;
+    int32_t *tok_key, *key_cnt, *bidx, *key2blk, *blk_cnt, *blk_pcnt, *tmp, *blk_fill;
     uint64_t* hkeys;
     int32_t* hvals;
     SSA_ALLOC(tok_key, int32_t, N);
@@ -510,7 +510,6 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     SSA_ALLOC(blk_cnt, int32_t, cap_mb + 1);
     SSA_ALLOC(blk_pcnt, int32_t, cap_mb + 1);
     SSA_ALLOC(blk_fill, int32_t, cap_mb + 1);
-    SSA_ALLOC(nbr_cnt, int32_t, N + 1);
     SSA_ALLOC(tmp, int32_t, tmp_len);
     SSA_ALLOC(hkeys, uint64_t, hsize);
     SSA_ALLOC(hvals, int32_t, hsize);
@@ -518,7 +517,6 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     SSA_ALLOC(p->blk_poff, int32_t, cap_mb + 1);
     SSA_ALLOC(p->blk_coord, int32_t, 3 * cap_mb);
     SSA_ALLOC(p->blk_seq, int32_t, cap_mb);
-    SSA_ALLOC(p->nbr_off32, int32_t, N + 1);
     if (cudaMemsetAsync(key_cnt, 0, sizeof(int32_t) * G, st) ||
         cudaMemsetAsync(blk_cnt, 0, sizeof(int32_t) * (cap_mb + 1), st) ||
         cudaMemsetAsync(blk_pcnt, 0, sizeof(int32_t) * (cap_mb + 1), st) ||
@@ -540,23 +538,15 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     scan_exclusive(blk_pcnt, p->blk_poff, cap_mb, tmp, st);
     trace_step("plan blocks", st);
 
-    // ---- a2: neighbour counts --------------------------------------------------------------------
+    // ---- a2: the per-token neighbour counts and lists are built on first use --------------------
     const int cube = (2 * r + 1) * (2 * r + 1) * (2 * r + 1);
     int cap = 32;
     while (cap < cube) cap <<= 1;
-    const int warps = std::max(1, std::min(8, 8192 / cap));
-    k_neighbours<false><<<grid_for(N, warps), warps * 32, 0, st>>>(
-        coords, N, p->d_seqs, B, r, hkeys, hvals, hsize - 1, nbr_cnt, nullptr, nullptr, cap,
-        p->d_status);
-    note_launch();
-    scan_exclusive(nbr_cnt, p->nbr_off32, N, tmp, st);
-    trace_step("plan neighbour counts", st);
 
     // ---- first wait: sizes and coordinate errors --------------------------------------------------
     int32_t h_sizes[4];
     if (cudaMemcpyAsync(&h_sizes[0], bidx + G, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
         cudaMemcpyAsync(&h_sizes[1], p->blk_poff + cap_mb, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
-        cudaMemcpyAsync(&h_sizes[2], p->nbr_off32 + N, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
         cudaMemcpyAsync(&h_sizes[3], p->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
         cudaStreamSynchronize(st))
         return SSA_ERR_CUDA;
@@ -565,8 +555,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     if (h_sizes[3]) return SSA_ERR_CUDA;
     p->Mb = h_sizes[0];
     p->Npad = h_sizes[1];
-    p->nnz = h_sizes[2];
-    if (p->nnz < 0) return SSA_ERR_UNSUPPORTED;  // more than 2^31 neighbour pairs
+    p->nnz = -1;   // counted on first use
 
     // ---- a1: scatter, per-block sort, positions ------------------------------------------------
     SSA_ALLOC(p->perm, int32_t, N);
@@ -611,7 +600,6 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     SSA_ALLOC(p->qt_len, int32_t, T);
     SSA_ALLOC(p->qt_seq, int32_t, T);
     SSA_ALLOC(p->wt_off, int32_t, T + 1);
-    SSA_ALLOC(p->wt_keys, int32_t, p->nnz);
     if (cudaMemcpyAsync(p->qt_pos, qpos.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st) ||
         cudaMemcpyAsync(p->qt_len, qlen.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st) ||
         cudaMemcpyAsync(p->qt_seq, qseq.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st))
@@ -624,6 +612,12 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     note_launch();
     trace_step("plan neighbour lists + window union counts", st);
     scan_exclusive(wt_cnt, p->wt_off, T, tmp, st);
+    int32_t n_wkeys = 0;
+    if (cudaMemcpyAsync(&n_wkeys, p->wt_off + T, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    if (n_wkeys < 0) return SSA_ERR_UNSUPPORTED;
+    SSA_ALLOC(p->wt_keys, int32_t, n_wkeys);
     k_window_union<true><<<(unsigned)T, 128, 0, st>>>(
         p->qt_pos, p->qt_len, p->qt_seq, p->perm, p->tok_blk, p->coords, p->blk_coord, p->blk_poff,
         p->blk_off, key2blk, p->d_seqs, p->scoord, r, nullptr, p->wt_off, p->wt_keys);
@@ -672,7 +666,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
 
     // scratch of the plan build is released now
     void* scratch[] = {tok_key, key_cnt, bidx, key2blk, blk_cnt, blk_pcnt, blk_fill,
-                       nbr_cnt, tmp, wt_cnt, wr_cnt, wm_cnt};
+                       tmp, wt_cnt, wr_cnt, wm_cnt};
     for (void* ptr : scratch) {
         auto it = std::find(p->owned.begin(), p->owned.end(), ptr);
         if (it != p->owned.end()) {
@@ -683,7 +677,38 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 
+ssa_status_t ensure_neighbour_counts(Plan* p, cudaStream_t st) {
+    if (p->nnz >= 0) return SSA_OK;
+    const int cap = p->nbr_cap;
+    const int warps = std::max(1, std::min(8, 8192 / cap));
+    int32_t *cnt, *tmp;
+    SSA_ALLOC(p->nbr_off32, int32_t, p->N + 1);
+    SSA_ALLOC(cnt, int32_t, p->N + 1);
+    SSA_ALLOC(tmp, int32_t, scan_tmp_len(p->N + 1));
+    k_neighbours<false><<<grid_for(p->N, warps), warps * 32, 0, st>>>(
+        p->coords, p->N, p->d_seqs, p->B, p->r, p->hkeys, p->hvals, p->hmask, cnt, nullptr, nullptr,
+        cap, p->d_status);
+    note_launch();
+    scan_exclusive(cnt, p->nbr_off32, p->N, tmp, st);
+    int32_t total = 0;
+    if (cudaMemcpyAsync(&total, p->nbr_off32 + p->N, sizeof(int32_t), cudaMemcpyDeviceToHost, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    for (void* ptr : {(void*)cnt, (void*)tmp}) {
+        auto it = std::find(p->owned.begin(), p->owned.end(), ptr);
+        if (it != p->owned.end()) {
+            p->release(ptr, st, p->alloc_ctx);
+            p->owned.erase(it);
+        }
+    }
+    if (total < 0) return SSA_ERR_UNSUPPORTED;   // more than 2^31 neighbour pairs
+    p->nnz = total;
+    return SSA_OK;
+}
+
 ssa_status_t ensure_neighbours(Plan* p, cudaStream_t st) {
+    ssa_status_t rc = ensure_neighbour_counts(p, st);
+    if (rc != SSA_OK) return rc;
     if (p->nbr_idx || p->nnz == 0) return SSA_OK;
     SSA_ALLOC(p->nbr_idx, int32_t, p->nnz);
     const int cap = p->nbr_cap;

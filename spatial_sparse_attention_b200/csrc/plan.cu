@@ -266,6 +266,7 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
     __shared__ int4 qc[kQTile];
     __shared__ int32_t cand[kCandCap];
     __shared__ int32_t tile_blocks[kQTile];
+    __shared__ int32_t qblk[kQTile];
     __shared__ int32_t ncand_s, ntb_s;
     const int t = blockIdx.x;
     const int32_t p0 = qt_pos[t], len = qt_len[t];
@@ -278,6 +279,7 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
     for (int a = threadIdx.x; a < len; a += blockDim.x) {
         int32_t i = perm[p0 + a];
         qc[a] = make_int4(coords[3 * i], coords[3 * i + 1], coords[3 * i + 2], 0);
+        qblk[a] = tok_blk[i];
         atomicMin(&box[0], qc[a].x);
         atomicMin(&box[1], qc[a].y);
         atomicMin(&box[2], qc[a].z);
@@ -285,11 +287,12 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
         atomicMax(&box[4], qc[a].y);
         atomicMax(&box[5], qc[a].z);
     }
+    __syncthreads();
     // distinct blocks of the tile (the tile is a run of consecutive sorted tokens)
     if (threadIdx.x == 0) {
         int32_t prev = -1;
         for (int a = 0; a < len; ++a) {
-            int32_t b = tok_blk[perm[p0 + a]];
+            const int32_t b = qblk[a];
             if (b != prev) tile_blocks[ntb_s++] = b;
             prev = b;
         }
@@ -334,45 +337,145 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
         __syncthreads();
     }
     const int ncand = ncand_s;
-    int32_t out_base = kFill ? wt_off[t] : 0;
-    int total = 0;
-    const int bx0 = box[0] - r, by0 = box[1] - r, bz0 = box[2] - r;
-    const int bx1 = box[3] + r, by1 = box[4] + r, bz1 = box[5] + r;
-    for (int cb = 0; cb < ncand; ++cb) {
-        int32_t b = cand[cb];
-        // a block whose 8^3 cube misses the tile's box grown by r holds no window key
-        const int cx = 8 * blk_coord[3 * b], cy = 8 * blk_coord[3 * b + 1], cz = 8 * blk_coord[3 * b + 2];
-        if (cx > bx1 || cx + 7 < bx0 || cy > by1 || cy + 7 < by0 || cz > bz1 || cz + 7 < bz0) continue;
-        int32_t r0 = blk_poff[b], nrow = blk_off[b + 1] - blk_off[b];
-        for (int a0 = 0; a0 < nrow; a0 += blockDim.x) {
-            int a = a0 + threadIdx.x;
-            bool keep = false;
-            if (a < nrow) {
-                int4 kc = scoord[r0 + a];
-                const bool inbox = kc.x >= bx0 && kc.x <= bx1 && kc.y >= by0 && kc.y <= by1 &&
-                                   kc.z >= bz0 && kc.z <= bz1;
-                for (int u = 0; u < len && !keep && inbox; ++u) {
-                    int4 c = qc[u];
-                    int d = max(abs(kc.x - c.x), max(abs(kc.y - c.y), abs(kc.z - c.z)));
-                    keep = d <= r;
-                }
+    // Exact window test through occupancy bitmaps: for each of the tile's blocks (up to 4), the
+    // cells of its queries in a 32^3 box with origin 8 * block - r, dilated by r along z, y and x
+    // (the Chebyshev ball is a box, so the dilation separates by axis). A key is in the union iff
+    // its cell is set in some block's bitmap. Tiles over more blocks test every query.
+    constexpr int kMaxBitmaps = 4;
+    __shared__ uint32_t bmp[kMaxBitmaps][32 * 32];   // words (x, y), bit z
+    __shared__ uint32_t btmp[32 * 32];
+    __shared__ int4 borg[kMaxBitmaps];
+    const int ntb = ntb_s;
+    const bool use_bmp = ntb <= kMaxBitmaps;
+    if (use_bmp) {
+        for (int i = threadIdx.x; i < ntb * 1024; i += blockDim.x) (&bmp[0][0])[i] = 0u;
+        if (threadIdx.x < ntb) {
+            const int32_t b = tile_blocks[threadIdx.x];
+            borg[threadIdx.x] = make_int4(8 * blk_coord[3 * b] - r, 8 * blk_coord[3 * b + 1] - r,
+                                          8 * blk_coord[3 * b + 2] - r, 0);
+        }
+        __syncthreads();
+        for (int a = threadIdx.x; a < len; a += blockDim.x) {
+            const int32_t b = qblk[a];
+            int u = 0;
+            while (u < ntb - 1 && tile_blocks[u] != b) ++u;
+            const int4 o = borg[u];
+            atomicOr(&bmp[u][(qc[a].x - o.x) * 32 + (qc[a].y - o.y)], 1u << (qc[a].z - o.z));
+        }
+        __syncthreads();
+        for (int u = 0; u < ntb; ++u) {
+            uint32_t* B = bmp[u];
+            for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
+                const uint32_t w = B[i];
+                uint32_t d = w;
+                for (int k = 1; k <= r; ++k) d |= (w << k) | (w >> k);
+                B[i] = d;
             }
-            // CTA-wide ordered compaction of `keep`
-            unsigned m = __ballot_sync(0xffffffffu, keep);
-            __shared__ int wcount[32];
-            const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-            if (lane == 0) wcount[wid] = __popc(m);
             __syncthreads();
-            int before = 0, all = 0;
-            for (int u = 0; u < (int)(blockDim.x >> 5); ++u) {
-                if (u < wid) before += wcount[u];
-                all += wcount[u];
+            for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
+                const int x = i >> 5, y = i & 31;
+                uint32_t d = 0u;
+                for (int k = -r; k <= r; ++k)
+                    if (y + k >= 0 && y + k < 32) d |= B[x * 32 + y + k];
+                btmp[i] = d;
             }
-            if (kFill && keep)
-                wt_keys[out_base + total + before + __popc(m & ((1u << lane) - 1))] = r0 + a;
-            total += all;
+            __syncthreads();
+            for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
+                const int x = i >> 5, y = i & 31;
+                uint32_t d = 0u;
+                for (int k = -r; k <= r; ++k)
+                    if (x + k >= 0 && x + k < 32) d |= btmp[(x + k) * 32 + y];
+                B[i] = d;
+            }
             __syncthreads();
         }
+    }
+    int32_t out_base = kFill ? wt_off[t] : 0;
+    const int bx0 = box[0] - r, by0 = box[1] - r, bz0 = box[2] - r;
+    const int bx1 = box[3] + r, by1 = box[4] + r, bz1 = box[5] + r;
+    // keys of the candidate blocks that reach the tile's box grown by r, flattened in ascending
+    // block order: kb_first[cb] = first flattened key of candidate cb (0 keys if it misses). Held in
+    // the dilation scratch when the bitmaps are used (at most 4 x 27 candidates), otherwise in the
+    // unused bitmap area (at most 128 x 27 = 3,456 candidates).
+    int32_t* kb_first = use_bmp ? reinterpret_cast<int32_t*>(btmp) : reinterpret_cast<int32_t*>(&bmp[0][0]);
+    __shared__ int wsum[32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    for (int cb = threadIdx.x; cb < ncand; cb += blockDim.x) {
+        const int32_t b = cand[cb];
+        const int cx = 8 * blk_coord[3 * b], cy = 8 * blk_coord[3 * b + 1], cz = 8 * blk_coord[3 * b + 2];
+        const bool miss = cx > bx1 || cx + 7 < bx0 || cy > by1 || cy + 7 < by0 || cz > bz1 || cz + 7 < bz0;
+        kb_first[cb] = miss ? 0 : blk_off[b + 1] - blk_off[b];
+    }
+    __syncthreads();
+    {
+        // exclusive prefix over the candidates: a contiguous chunk per thread, then across threads
+        const int cw = (ncand + blockDim.x - 1) / blockDim.x;
+        const int c0 = min((int)threadIdx.x * cw, ncand), c1 = min(c0 + cw, ncand);
+        int sum = 0;
+        for (int cb = c0; cb < c1; ++cb) sum += kb_first[cb];
+        int x = sum;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[wid] = x;
+        __syncthreads();
+        int off = x - sum, tot = 0;
+        for (int u = 0; u < nwarps; ++u) {
+            off += u < wid ? wsum[u] : 0;
+            tot += wsum[u];
+        }
+        for (int cb = c0; cb < c1; ++cb) {
+            const int n = kb_first[cb];
+            kb_first[cb] = off;
+            off += n;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) kb_first[ncand] = tot;
+        __syncthreads();
+    }
+    const int nkeys = kb_first[ncand];
+    int total = 0;
+    for (int c0 = 0; c0 < nkeys; c0 += blockDim.x) {
+        const int k = c0 + threadIdx.x;
+        bool keep = false;
+        int32_t row = 0;
+        if (k < nkeys) {
+            int lo = 0, hi = ncand - 1;   // last candidate whose first key is <= k
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (kb_first[mid] <= k) lo = mid; else hi = mid - 1;
+            }
+            row = blk_poff[cand[lo]] + (k - kb_first[lo]);
+            const int4 kc = scoord[row];
+            if (kc.x >= bx0 && kc.x <= bx1 && kc.y >= by0 && kc.y <= by1 && kc.z >= bz0 && kc.z <= bz1) {
+                if (use_bmp) {
+                    for (int u = 0; u < ntb && !keep; ++u) {
+                        const int4 o = borg[u];
+                        const int rx = kc.x - o.x, ry = kc.y - o.y, rz = kc.z - o.z;
+                        if ((unsigned)rx < 32u && (unsigned)ry < 32u && (unsigned)rz < 32u)
+                            keep = (bmp[u][rx * 32 + ry] >> rz) & 1u;
+                    }
+                } else {
+                    for (int u = 0; u < len && !keep; ++u) {
+                        const int4 c = qc[u];
+                        keep = max(abs(kc.x - c.x), max(abs(kc.y - c.y), abs(kc.z - c.z))) <= r;
+                    }
+                }
+            }
+        }
+        // CTA-wide ordered compaction of `keep`
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) wsum[wid] = __popc(m);
+        __syncthreads();
+        int before = 0, all = 0;
+        for (int u = 0; u < nwarps; ++u) {
+            before += u < wid ? wsum[u] : 0;
+            all += wsum[u];
+        }
+        if (kFill && keep) wt_keys[out_base + total + before + __popc(m & ((1u << lane) - 1))] = row;
+        total += all;
+        __syncthreads();
     }
     if (!kFill && threadIdx.x == 0) wt_cnt[t] = total;
 }

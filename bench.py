@@ -112,7 +112,7 @@ class Clocks:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -215,13 +215,15 @@ def run_ours(args, rank, world, dist):
     work = algorithmic_flops(plan, sel, cfg, cu)
     del sel
 
+    # clocks are sampled from the warm-up on (nvidia-smi needs ~0.1 s to start), so every sample
+    # is taken under this workload
+    clocks = Clocks(torch.cuda.current_device())
+    if rank == 0:
+        clocks.start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
 
-    clocks = Clocks(torch.cuda.current_device())
-    if rank == 0:
-        clocks.start()
     ssa.profile_reset()
     ssa.profile_enable(True)
     launches0 = ssa.launch_count()

@@ -148,6 +148,8 @@ SSA_API ssa_status_t ssa_plan_export(ssa_plan_t plan, int32_t* perm, int32_t* to
  * Queues work on `stream` and returns without waiting. The first call for a given
  * (H, D, dtype, k) allocates the plan's workspace; later calls allocate nothing.
  * Not reentrant on one plan: calls that share a plan must be ordered on one stream.
+ * bf16 / fp16: a sequence may hold at most 65,536 * D / 32 occupied blocks (the union of the
+ * selected blocks is built in on-chip memory); more returns SSA_ERR_UNSUPPORTED.
  */
 SSA_API ssa_status_t ssa_forward(ssa_plan_t plan, const void* q, const void* k, const void* v,
                          const float* gates, const float* wc, int32_t heads, int32_t head_dim,

@@ -1,6 +1,6 @@
 // Device-wide exclusive prefix sum of int32 values: three passes (tile sums, scan of the tile
-// sums in one CTA, rescan of each tile with its offset). Used by the plan (block and neighbour
-// offsets) and the forward (inverted selection lists).
+// sums in one CTA, rescan of each tile with its offset). Used by the plan (block, neighbour and
+// window offsets) and the allocation-free block offsets.
 #include "common.cuh"
 
 namespace ssa {

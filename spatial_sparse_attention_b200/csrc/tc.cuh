@@ -1,6 +1,6 @@
 // sm_100a primitives for the tensor-core attention kernels: shared-memory matrix descriptors,
 // instruction descriptors, tcgen05 MMA / TMEM load-store / allocation, mbarriers with bounded
-// waits, and cp.async copies. All inline PTX; written from the PTX ISA's description of these
+// waits, 1D bulk copies and cp.async copies. All inline PTX; written from the PTX ISA's description of these
 // instructions.
 #pragma once
 
@@ -17,17 +17,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // A tile of 16-bit elements is stored as column chunks of 32 elements (64 bytes per row). Inside
 // a chunk, rows are 64 bytes apart, groups of 8 rows ("atoms", 512 bytes) are contiguous, and the
 // four 16-byte units of a row are permuted by unit ^= (row >> 1) & 3 (bits [4,6) of the address
-// XOR bits [7,9)). Chunk regions are kRegion bytes apart (128 rows).
-constexpr uint32_t kRegion = 128 * 64;
+// XOR bits [7,9)).
 
 __device__ __forceinline__ uint32_t sw64(int row, int unit) {
     return (uint32_t)((row >> 3) * 512 + (row & 7) * 64 + ((unit ^ ((row >> 1) & 3)) << 4));
 }
-// byte offset of 16-byte unit `c16` (8 elements) of row `row` in a chunked tile
-__device__ __forceinline__ uint32_t tile_off(int row, int c16) {
-    return (uint32_t)(c16 >> 2) * kRegion + sw64(row, c16 & 3);
-}
-
 // ---- descriptors ------------------------------------------------------------------------------
 // Shared-memory matrix descriptor (sm_100): start address >> 4 in bits [0,14), leading byte
 // offset >> 4 in [16,30), stride byte offset >> 4 in [32,46), version 1 in [46,48), swizzle mode
@@ -40,17 +34,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     d |= (uint64_t)4 << 61;
     return d;
 }
-// K-major operand (rows = M or N, K contiguous inside 32-element chunks): K step `kk` (16
-// elements) starts in chunk kk/2 at byte 32*(kk%2); 8-row groups are 512 bytes apart.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
-    return smem_desc(base + (uint32_t)(kk >> 1) * kRegion + (uint32_t)(kk & 1) * 32, 16, 512);
-}
-// MN-major operand (rows = K, N contiguous inside 32-element chunks): K step `kk` covers rows
-// 16kk..16kk+15 (two 8-row groups, 512 bytes apart); N chunks are kRegion bytes apart.
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk) {
-    return smem_desc(base + (uint32_t)kk * 1024, kRegion, 512);
-}
-
 // Grouped layout: a tile is a sequence of 8-row groups; each group holds its kch 32-element
 // chunks as consecutive 512-byte swizzled atoms (group stride kch * 512 bytes). K-major operand
 // (rows = N, K contiguous): K step `kk` is in chunk kk/2 at byte 32*(kk%2) of every atom.
@@ -63,14 +46,11 @@ __device__ __forceinline__ uint64_t desc_mnmajor_g(uint32_t base, int kk, uint32
     return smem_desc(base + (uint32_t)kk * 2 * kch * 512, 512, kch * 512);
 }
 
-// Same, for tiles whose 32-element chunks are `region` bytes apart.
+// Chunked layout (the Q tile): K-major operand whose 32-element chunks are `region` bytes apart
+// and whose 8-row atoms are 512 bytes apart; K step `kk` is in chunk kk/2 at byte 32*(kk%2).
 __device__ __forceinline__ uint64_t desc_kmajor_r(uint32_t base, int kk, uint32_t region) {
     return smem_desc(base + (uint32_t)(kk >> 1) * region + (uint32_t)(kk & 1) * 32, 16, 512);
 }
-__device__ __forceinline__ uint64_t desc_mnmajor_r(uint32_t base, int kk, uint32_t region) {
-    return smem_desc(base + (uint32_t)kk * 1024, region, 512);
-}
-
 // Instruction descriptor, kind::f16: fp32 accumulator (bit 4), A/B type (bits 7-9 / 10-12:
 // 0 = f16, 1 = bf16), A K-major (bit 15 = 0), B major (bit 16), N >> 3 (bits 17-22),
 // M >> 4 (bits 24-28).
@@ -114,36 +94,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
             smem_u32(bar))
         : "memory");
 }
-// 16 consecutive fp32 columns of this thread's TMEM lane (32x32b shape: warp w reads lanes
-// 32w..32w+31). Load and wait are fused so no register is read before it is valid.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
-    __syncwarp();   // .sync.aligned: the whole warp must arrive converged
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-        "[%16];\n\ttcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-    __syncwarp();
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
-        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15]))
-        : "memory");
-}
-
 // 64 consecutive fp32 columns of this thread's TMEM lane, loaded and waited for in one asm block
 // (no register is read before it is valid). Warp-collective.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
@@ -231,30 +181,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
-// ---- TMA ----------------------------------------------------------------------------------------
-// 2D tiled bulk tensor load (no multicast): box at coordinates (x = innermost element index,
-// y = row) of the tensor described by `tmap` into shared memory at `dst`, completing `bytes`
-// transactions on `bar`. x * element size must be a multiple of 16 bytes.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int32_t x, int32_t y,
-                                            uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-// Row gather (tile::gather4, no multicast): four rows y0..y3 of the 2D tensor, columns
-// [x, x + box width), into four consecutive box rows at `dst`. The tensor map's box is one row
-// high. x * element size must be a multiple of 16 bytes.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int32_t x, int32_t y0,
-                                            int32_t y1, int32_t y2, int32_t y3, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
-        "r"(smem_u32(bar))
-        : "memory");
-}
+// ---- bulk copies -------------------------------------------------------------------------------
 // 1D bulk copy (no multicast) of `bytes` contiguous bytes from global `src` to shared `dst`,
 // completing `bytes` transactions on `bar`. Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -263,10 +190,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
-__device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
-}
-
 // ---- copies ---------------------------------------------------------------------------------------
 // 16-byte asynchronous global->shared copy; src_bytes = 0 writes zeros (nothing is read).
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {

@@ -180,3 +180,19 @@ def test_forward_argument_errors():
     with pytest.raises(ssa.SSAError) as e:
         plan.forward(q, q, q, gates, torch.eye(32, device="cuda"), 33)
     assert e.value.name == "SSA_ERR_UNSUPPORTED"
+
+
+def test_too_many_blocks_in_a_sequence_is_unsupported():
+    """The 16-bit path builds the union of selected blocks in on-chip memory: a sequence with more
+    than 65,536 * D / 32 occupied blocks is rejected before any kernel runs."""
+    import spatial_sparse_attention_b200 as ssa
+    n = 70_000   # one token per block: 70,000 blocks > 65,536 for D = 32
+    i = np.arange(n)
+    coords = np.stack([8 * (i // (128 * 64)), 8 * ((i // 64) % 128), 8 * (i % 64)], 1).astype(np.int32)
+    plan = ssa.Plan(torch.from_numpy(coords).cuda(), grid=(1024, 1024, 512), r=0)
+    assert plan.num_blocks == n
+    q = torch.zeros(n, 1, 32, dtype=torch.bfloat16, device="cuda")
+    gates = torch.zeros(n, 1, 3, device="cuda")
+    with pytest.raises(ssa.SSAError) as e:
+        plan.forward(q, q, q, gates, torch.eye(32, device="cuda"), 2)
+    assert e.value.name == "SSA_ERR_UNSUPPORTED"

@@ -58,8 +58,8 @@ def config_of(args):
 # (profiles/k_ssa_fwd_pass3_h4.md: dram__bytes_read.sum + dram__bytes_write.sum of the 4-head cut,
 # divided by 4; the launch's traffic grows in proportion to the heads). Valid only for the kernel
 # sources the capture was taken with.
-KERNEL_TRAFFIC = {"sources_sha256": "5157c3a1460df167e10e1b126b96c11b99ab685a78aada9aa4abdc8bdf7441b8",
-                  "config": "pass3", "bytes_per_head": 633601536.0 / 4}
+KERNEL_TRAFFIC = {"sources_sha256": "8e9748e3fc62d8e1ab3ab118c33442a71fefd2b2b99e3fb2b989cc8db6b1e25f",
+                  "config": "pass3", "bytes_per_head": 632926208.0 / 4}
 KERNEL_SOURCES = ("attn_fwd.cu", "attn_common.cuh", "tc.cuh")
 
 

@@ -58,17 +58,21 @@ def config_of(args):
 # (profiles/k_ssa_fwd_pass3_h4.md: dram__bytes_read.sum + dram__bytes_write.sum of the 4-head cut,
 # divided by 4; the launch's traffic grows in proportion to the heads). Valid only for the kernel
 # sources the capture was taken with.
-KERNEL_TRAFFIC = {"sources_sha256": "8e9748e3fc62d8e1ab3ab118c33442a71fefd2b2b99e3fb2b989cc8db6b1e25f",
+KERNEL_TRAFFIC = {"sources_sha256": "0e28bab05d86fcb8e98190cc10159222927ac684dd26f4f99db12c35d2f0d10e",
                   "config": "pass3", "bytes_per_head": 632926208.0 / 4}
 KERNEL_SOURCES = ("attn_fwd.cu", "attn_common.cuh", "tc.cuh")
 
 
 def kernel_sources_sha256():
+    """Hash of the kernel's code: comments and whitespace are left out, so that only a change of
+    the code itself invalidates the recorded traffic."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "spatial_sparse_attention_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "spatial_sparse_attention_b200", "csrc", f), encoding="utf-8") as fh:
+            code = re.sub(r"//[^\n]*", "", fh.read())
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()
 
 

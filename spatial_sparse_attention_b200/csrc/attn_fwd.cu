@@ -18,7 +18,7 @@
 //             K/V copies in global memory are stored as 8-row groups already in the tensor cores'
 //             swizzled operand order, so a run of consecutive groups is one copy: the compressed
 //             tokens are one run, each selected block is one run, and the window union is the
-//             plan's list of runs (with the keys' coordinates);
+//             plan's list of runs (its per-row key masks come from the plan as well);
 //   warp 1    MMA issuer (one thread): S = Q K^T into one of two TMEM buffers; O += P V with P
 //             read from TMEM (it overwrites S in place);
 //   warps 2-5 softmax, one thread per row (its TMEM lane): S into registers once, mask, running

@@ -239,6 +239,58 @@ def test_permutation_equivariance():
     assert np.array_equal(shuf["sel"], base["sel"][p])
 
 
+def test_window_of_radius_zero_is_the_token_itself():
+    # W(i) = {i} at r = 0: one key, weight exactly 1, so o_win is the token's own value
+    c, q, k, v, Wc = _tiny_inputs(seed=75)
+    off, idx = oracle.window(c, 0)
+    assert np.array_equal(off, np.arange(len(c) + 1))
+    assert np.array_equal(idx, np.arange(len(c)))
+    res = run(c, q, k, v, _gates(len(c), 2, (0, 0, 1)), Wc, 4, 0)
+    assert np.array_equal(res["o_win"], v)
+    assert np.array_equal(res["out"], v)
+
+
+def test_branches_are_linear_in_the_values():
+    # V enters every branch only through the final weighted sum (the compressed one after the
+    # linear mean and Wc), and the selection depends on Q and K alone
+    c, q, k, v, Wc = _tiny_inputs(seed=76)
+    v2 = _rand(v.shape, 77)
+    g = _gates(len(c), 2, None)
+    a = run(c, q, k, v, g, Wc, 4, 2)
+    b = run(c, q, k, v2, g, Wc, 4, 2)
+    ab = run(c, q, k, 2.0 * v - 3.0 * v2, g, Wc, 4, 2)
+    for name in ("o_cmp", "o_sel", "o_win", "out"):
+        np.testing.assert_allclose(ab[name], 2.0 * a[name] - 3.0 * b[name], rtol=0, atol=1e-12)
+    assert np.array_equal(a["sel"], b["sel"]) and np.array_equal(a["sel"], ab["sel"])
+
+
+def test_packed_sequences_are_independent():
+    # a second, different shell packed behind the first: each sequence's rows equal a run on
+    # that sequence alone; its block indices continue after the first sequence's blocks
+    c1, q1, k1, v1, Wc = _tiny_inputs(seed=78)
+    c2 = np.ascontiguousarray(c1[::2][:, [1, 0, 2]] + np.array([0, 3, 5], np.int32))
+    n1, n2 = len(c1), len(c2)
+    q2, k2, v2 = (_rand((n2, 2, 32), 79 + t) for t in range(3))
+    g1, g2 = _gates(n1, 2, None, seed=3), _gates(n2, 2, None, seed=4)
+    cat = lambda a, b: np.concatenate([a, b], axis=0)
+    cu = np.array([0, n1, n1 + n2])
+    both = oracle.forward(cat(c1, c2), cu, cat(q1, q2), cat(k1, k2), cat(v1, v2), cat(g1, g2),
+                          Wc, 4, 2)
+    one = run(c1, q1, k1, v1, g1, Wc, 4, 2)
+    two = run(c2, q2, k2, v2, g2, Wc, 4, 2)
+    mb1 = len(oracle.partition(c1)[3])
+    for name in ("o_cmp", "o_sel", "o_win", "out"):
+        np.testing.assert_allclose(both[name][:n1], one[name], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(both[name][n1:], two[name], rtol=0, atol=1e-13)
+    assert np.array_equal(both["sel"][:n1], one["sel"])
+    assert np.array_equal(both["sel"][n1:], np.where(two["sel"] >= 0, two["sel"] + mb1, -1))
+    p = oracle.plan(cat(c1, c2), cu, r=2)
+    p1, p2 = oracle.plan(c1, [0, n1], r=2), oracle.plan(c2, [0, n2], r=2)
+    assert np.array_equal(p["perm"], cat(p1["perm"], p2["perm"] + n1))
+    assert np.array_equal(p["blk_off"], cat(p1["blk_off"][:-1], p2["blk_off"] + n1))
+    assert np.array_equal(p["nbr_idx"], cat(p1["nbr_idx"], p2["nbr_idx"] + n1))
+
+
 def test_translation_by_whole_blocks():
     c, q, k, v, Wc = _tiny_inputs(seed=80)
     g = _gates(len(c), 2, None)

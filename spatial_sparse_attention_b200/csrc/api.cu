@@ -255,15 +255,15 @@ ssa_status_t ensure_workspace(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int
     if (!w.kc || !w.vc || !w.sel) return SSA_ERR_ALLOC;
     if (dt != SSA_F32) {
         w.Mb8 = round_up(Mb, 8);
-        w.ks = A(es * H * p->Npad * D);
-        w.vs = A(es * H * p->Npad * D);
+        w.ks = A(es * H * p->Nks * D);
+        w.vs = A(es * H * p->Nks * D);
         w.kcg = A(es * H * w.Mb8 * D);
         w.vcg = A(es * H * w.Mb8 * D);
         w.base = (float*)A(sizeof(float) * p->n_qtiles * kQTile * H * D);
         if (!w.ks || !w.vs || !w.kcg || !w.vcg || !w.base) return SSA_ERR_ALLOC;
         // padding rows of the block-ordered copies stay zero for the life of the workspace
-        if (cudaMemsetAsync(w.ks, 0, es * H * p->Npad * D, st) ||
-            cudaMemsetAsync(w.vs, 0, es * H * p->Npad * D, st) ||
+        if (cudaMemsetAsync(w.ks, 0, es * H * p->Nks * D, st) ||
+            cudaMemsetAsync(w.vs, 0, es * H * p->Nks * D, st) ||
             cudaMemsetAsync(w.kcg, 0, es * H * w.Mb8 * D, st) ||
             cudaMemsetAsync(w.vcg, 0, es * H * w.Mb8 * D, st))
             return SSA_ERR_CUDA;
@@ -355,7 +355,7 @@ ssa_status_t ssa_plan_varlen(const int32_t* coords, const int64_t* cu_seqlens, i
 ssa_status_t ssa_plan_rebuild(ssa_plan_t p, const int32_t* coords, void* stream) {
     if (!p || !coords) return SSA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    const int64_t old_mb = p->Mb, old_npad = p->Npad;
+    const int64_t old_mb = p->Mb, old_nks = p->Nks;
     plan_free_all(p, p->owned);
     p->stream = st;
     ssa_status_t rc;
@@ -371,7 +371,7 @@ ssa_status_t ssa_plan_rebuild(ssa_plan_t p, const int32_t* coords, void* stream)
         p->ws = Workspace();
         return rc;
     }
-    if (p->Mb != old_mb || p->Npad != old_npad) {
+    if (p->Mb != old_mb || p->Nks != old_nks) {
         plan_free_all(p, p->ws.owned);
         p->ws = Workspace();
     }

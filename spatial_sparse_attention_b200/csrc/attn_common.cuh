@@ -14,7 +14,7 @@ constexpr long long kWaitCycles = 4000000000LL;   // ~2 s at 2 GHz
 
 struct FwdParams {
     const void* q;
-    const void* ks;    // grouped order, [H, Npad, D]
+    const void* ks;    // grouped order, [H, Nks, D]: padded block rows, then the pools
     const void* vs;
     const void* kcg;   // grouped order, [H, Mb8, D]
     const void* vcg;
@@ -24,6 +24,8 @@ struct FwdParams {
     const int32_t* blk_off;
     const int32_t* blk_poff;
     const int2* blk_info;     // (first 8-row group, tokens) per block
+    const int32_t* blk_tpool; // row of a small block in its sequence's pool (relative), -1 if none
+    const int2* seq_pool;     // (first 8-row group, groups) of each sequence's pool
     const int4* scoord;
     const int32_t* qt_pos;
     const int32_t* qt_len;
@@ -38,7 +40,7 @@ struct FwdParams {
     float* base;
     void* out;
     int32_t* status;
-    int64_t N, Npad, Mb, Mb8;
+    int64_t N, Nks, Mb, Mb8;
     int H, k, r;
     float sl;   // softmax scale * log2(e)
 };

@@ -186,8 +186,8 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
         // Every phase is a stream of runs of consecutive 8-row groups (compressed tokens: one run;
         // selected blocks: one run per union block; window: the plan's runs). A 64-key tile takes
         // the next 8 groups; lane l < 8 copies the part of run ri + l that falls in the tile.
-        const uint8_t* ksh = static_cast<const uint8_t*>(P.ks) + (int64_t)h * P.Npad * D * 2;
-        const uint8_t* vsh = static_cast<const uint8_t*>(P.vs) + (int64_t)h * P.Npad * D * 2;
+        const uint8_t* ksh = static_cast<const uint8_t*>(P.ks) + (int64_t)h * P.Nks * D * 2;
+        const uint8_t* vsh = static_cast<const uint8_t*>(P.vs) + (int64_t)h * P.Nks * D * 2;
         const uint8_t* kch = static_cast<const uint8_t*>(P.kcg) + (int64_t)h * P.Mb8 * D * 2;
         const uint8_t* vch = static_cast<const uint8_t*>(P.vcg) + (int64_t)h * P.Mb8 * D * 2;
         int ri = 0, rskip = 0;   // next run, groups of it already streamed
@@ -448,42 +448,91 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                     }
                 }
                 tc::named_sync(2, 128);
-                // first group and group count of every union block (independent loads)
+                // first group and group count of every union block (independent loads); a block
+                // with a copy in the sequence's pool (always one group) is marked by a count of -1
+                int tcnt = 0;
                 for (int u = t128; u < U; u += 128) {
-                    const int2 bi = P.blk_info[bl + un[u].x];
-                    un[u] = make_int2(bi.x, (bi.y + 7) >> 3);
+                    const int b = bl + un[u].x;
+                    const int2 bi = P.blk_info[b];
+                    const bool small = P.blk_tpool[b] >= 0;
+                    un[u] = make_int2(bi.x, small ? -1 : (bi.y + 7) >> 3);
+                    tcnt += small ? 1 : 0;
                 }
-                tc::named_sync(2, 128);
+                // The pool replaces the small blocks' own groups when it is shorter than they are
+                // together (one group each); it then follows the other blocks in the stream.
+                int Ut = 0;
+                scan128(tcnt, t128, red, Ut);   // its barriers also publish the entries above
+                const int2 sp = P.seq_pool[seq];
+                const bool use_pool = sp.y > 0 && Ut > sp.y;
                 // stream offsets (in groups): exclusive prefix of the blocks' group counts
                 const int cu = (U + 127) >> 7;
                 const int ul = min(t128 * cu, U), uh = min(ul + cu, U);
                 int ssum = 0;
-                for (int u = ul; u < uh; ++u) ssum += un[u].y;
+                for (int u = ul; u < uh; ++u) {
+                    const int n = un[u].y;
+                    ssum += n >= 0 ? n : (use_pool ? 0 : 1);
+                }
                 int Lg = 0;
                 int off = scan128(ssum, t128, red, Lg);
                 for (int u = ul; u < uh; ++u) {
                     const int n = un[u].y;
                     un[u].y = off;
-                    off += n;
-                }
-                if (t128 == 0) {
-                    un[U] = make_int2(0, Lg);
-                    misc[M_U] = U;
-                    misc[M_L] = Lg;
+                    if (n < 0 && use_pool) un[u].x = -1;   // left out of the stream below
+                    off += n >= 0 ? n : (use_pool ? 0 : 1);
                 }
                 tc::named_sync(2, 128);
-                // this row's ranges [first key, last key + 1) in the stream, ascending
+                // this row's ranges [first key, last key + 1) in the stream, ascending; with the
+                // pool, the keys of pooled blocks follow all others (sort key raised by nblk)
 #pragma unroll
                 for (int a = 0; a < (int)L::kSlots; ++a) {
-                    if (mine[a] < 0 || mine[a] >= nblk) continue;
+                    if (mine[a] >= nblk) mine[a] = -1;
+                    if (use_pool && mine[a] >= 0 && P.blk_tpool[bl + mine[a]] >= 0) mine[a] += nblk;
+                }
+#pragma unroll
+                for (int a = 0; a < (int)L::kSlots; ++a) {
+                    if (mine[a] < 0) continue;
                     int rank = 0;
 #pragma unroll
                     for (int c = 0; c < (int)L::kSlots; ++c) rank += (mine[c] >= 0 && mine[c] < mine[a]) ? 1 : 0;
-                    const int wi = mine[a] >> 5;
-                    const int u = wpre[wi] + __popc(words[wi] & ((1u << (mine[a] & 31)) - 1u));
-                    if (u < U)
-                        rng[rank * 128 + row] = make_int2(8 * un[u].y, 8 * un[u].y + P.blk_info[bl + mine[a]].y);
+                    const bool pooled = mine[a] >= nblk;
+                    const int b = pooled ? mine[a] - nblk : mine[a];
+                    const int nb = P.blk_info[bl + b].y;
+                    if (pooled) {
+                        const int k0 = 8 * Lg + P.blk_tpool[bl + b];
+                        rng[rank * 128 + row] = make_int2(k0, k0 + nb);
+                    } else {
+                        const int wi = b >> 5;
+                        const int u = wpre[wi] + __popc(words[wi] & ((1u << (b & 31)) - 1u));
+                        if (u < U) rng[rank * 128 + row] = make_int2(8 * un[u].y, 8 * un[u].y + nb);
+                    }
                     ++nr;
+                }
+                tc::named_sync(2, 128);
+                if (use_pool) {
+                    // drop the pooled blocks' runs in place, 128 entries at a time (an entry only
+                    // moves down, to a place whose entry was read in this or an earlier step),
+                    // and append the pool as the last run
+                    int kept = 0;
+                    for (int c0 = 0; c0 < U; c0 += 128) {
+                        const int e = c0 + t128;
+                        const int2 v = e < U ? un[e] : make_int2(-1, 0);
+                        const int keep = v.x >= 0 ? 1 : 0;
+                        int tot = 0;
+                        const int at = scan128(keep, t128, red, tot);
+                        if (keep) un[kept + at] = v;
+                        kept += tot;
+                        tc::named_sync(2, 128);
+                    }
+                    if (t128 == 0) {
+                        un[kept] = make_int2(sp.x, Lg);
+                        un[kept + 1] = make_int2(0, Lg + sp.y);
+                        misc[M_U] = kept + 1;
+                        misc[M_L] = Lg + sp.y;
+                    }
+                } else if (t128 == 0) {
+                    un[U] = make_int2(0, Lg);
+                    misc[M_U] = U;
+                    misc[M_L] = Lg;
                 }
                 tc::named_sync(1, kThreads);   // the producer may now overwrite the rings
                 rcur = nr > 0 ? rng[row] : make_int2(0x7fffffff, 0x7fffffff);
@@ -683,6 +732,8 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.blk_off = p->blk_off;
     P.blk_poff = p->blk_poff;
     P.blk_info = p->blk_info;
+    P.blk_tpool = p->blk_tpool;
+    P.seq_pool = p->seq_pool;
     P.scoord = p->scoord;
     P.qt_pos = p->qt_pos;
     P.qt_len = p->qt_len;
@@ -698,7 +749,7 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.out = out;
     P.status = p->d_status;
     P.N = p->N;
-    P.Npad = p->Npad;
+    P.Nks = p->Nks;
     P.Mb = p->Mb;
     P.Mb8 = w.Mb8;
     P.H = w.H;

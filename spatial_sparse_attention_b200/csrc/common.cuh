@@ -27,6 +27,9 @@ constexpr int kBlockEdge = 8;      // block edge in voxels (the only supported v
 constexpr int kPad = 8;            // blocks start on multiples of 8 rows (one group) in the K/V copies
 constexpr int kQTile = 128;        // query rows per tensor-core tile
 constexpr int kMaxTopk = 32;
+// blocks of at most this many tokens (less than one 8-row group) also get a packed copy in
+// their sequence's pool, which the selected branch may stream in their place
+constexpr int kPoolMaxTokens = 7;
 
 // Per-sequence constants, mirrored on the device.
 struct SeqInfo {
@@ -40,10 +43,11 @@ struct SeqInfo {
 struct Workspace {
     int32_t H = 0, D = 0, k = 0;
     ssa_dtype_t dtype = SSA_F32;
-    // K_s, V_s: per head, the K / V rows in padded block order (Npad rows), stored as 8-row
-    // groups in the tensor cores' swizzled operand order (see pool.cu); padding rows are zero.
-    void* ks = nullptr;        // [H, Npad, D] T
-    void* vs = nullptr;        // [H, Npad, D] T
+    // K_s, V_s: per head, the K / V rows in padded block order (Npad rows) followed by each
+    // sequence's pool of small blocks (their rows again, packed), stored as 8-row groups in the
+    // tensor cores' swizzled operand order (see pool.cu); padding rows are zero.
+    void* ks = nullptr;        // [H, Nks, D] T
+    void* vs = nullptr;        // [H, Nks, D] T
     void* kc = nullptr;        // [H, Mb, D]   T (fp32 for the fp32 path), row-major
     void* vc = nullptr;        // [H, Mb, D]
     void* kcg = nullptr;       // [H, Mb8, D]  T   compressed tokens in the grouped order (16-bit path)
@@ -70,6 +74,7 @@ struct Plan {
     int64_t G = 0;       // dense block keys over all sequences
     int64_t Mb = 0;      // occupied blocks
     int64_t Npad = 0;    // padded sorted rows
+    int64_t Nks = 0;     // rows per head of K_s / V_s: the Npad padded rows, then the pools
     int64_t nnz = -1;    // window neighbour pairs (-1 until counted on first use)
     int64_t n_qtiles = 0;
     std::vector<SeqInfo> seqs;
@@ -84,6 +89,9 @@ struct Plan {
     int32_t* blk_off = nullptr;  // [Mb+1]
     int32_t* blk_poff = nullptr; // [Mb+1] padded row offsets
     int2* blk_info = nullptr;    // [Mb] (first 8-row group of the padded rows, tokens)
+    int32_t* blk_tpool = nullptr;// [Mb] row of a small block's copy in its sequence's pool
+                                 //      (relative to the pool's first row), -1 for other blocks
+    int2* seq_pool = nullptr;    // [B] (first 8-row group, groups) of each sequence's pool
     int32_t* blk_coord = nullptr;// [Mb,3]
     int32_t* blk_seq = nullptr;  // [Mb]
     int32_t* seq_blk_d = nullptr;// [B+1]

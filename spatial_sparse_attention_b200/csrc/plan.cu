@@ -237,6 +237,44 @@ __global__ void k_block_info(const int32_t* __restrict__ blk_off, const int32_t*
     if (b < Mb) info[b] = make_int2(blk_poff[b] >> 3, blk_off[b + 1] - blk_off[b]);
 }
 
+// One CTA per sequence. The sequence's blocks of at most kPoolMaxTokens tokens get consecutive
+// rows of its pool in block order: tpool[b] = first row relative to the pool, -1 for the other
+// blocks; ptok[s] = rows of the pool (its tokens).
+__global__ void __launch_bounds__(256) k_tiny_pool(const int32_t* __restrict__ blk_off,
+                                                   const int32_t* __restrict__ seq_blk,
+                                                   int32_t* __restrict__ tpool, int32_t* __restrict__ ptok) {
+    __shared__ int wsum[8];
+    __shared__ int carry;
+    const int s = blockIdx.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int32_t b0 = seq_blk[s], b1 = seq_blk[s + 1];
+    if (t == 0) carry = 0;
+    __syncthreads();
+    for (int32_t base = b0; base < b1; base += 256) {
+        const int32_t b = base + t;
+        const int32_t n = b < b1 ? blk_off[b + 1] - blk_off[b] : 0;
+        const int v = (b < b1 && n <= kPoolMaxTokens) ? n : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[w] = x;
+        __syncthreads();
+        int before = carry, total = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            before += i < w ? wsum[i] : 0;
+            total += wsum[i];
+        }
+        if (b < b1) tpool[b] = n <= kPoolMaxTokens ? before + x - v : -1;
+        __syncthreads();
+        if (t == 0) carry += total;
+        __syncthreads();
+    }
+    if (t == 0) ptok[s] = carry;
+}
+
 __global__ void k_fill_i32(int32_t* __restrict__ a, int64_t n, int32_t v) {
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < n) a[i] = v;
@@ -767,9 +805,32 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         return SSA_ERR_CUDA;
     if (status) return SSA_ERR_CUDA;
 
+    // ---- pools of small blocks: per sequence, after all padded block rows -------------------------
+    int32_t* ptok;
+    SSA_ALLOC(p->blk_tpool, int32_t, std::max<int64_t>(p->Mb, 1));
+    SSA_ALLOC(ptok, int32_t, B);
+    k_tiny_pool<<<(unsigned)B, 256, 0, st>>>(p->blk_off, p->seq_blk_d, p->blk_tpool, ptok);
+    note_launch();
+    std::vector<int32_t> hp(B);
+    if (cudaMemcpyAsync(hp.data(), ptok, sizeof(int32_t) * B, cudaMemcpyDeviceToHost, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    std::vector<int2> sp(B);
+    int64_t pg = p->Npad / 8;
+    for (int s = 0; s < B; ++s) {
+        const int32_t groups = (hp[s] + 7) / 8;
+        sp[s] = make_int2((int32_t)pg, groups);
+        pg += groups;
+    }
+    p->Nks = 8 * pg;
+    SSA_ALLOC(p->seq_pool, int2, B);
+    if (cudaMemcpyAsync(p->seq_pool, sp.data(), sizeof(int2) * B, cudaMemcpyHostToDevice, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+
     // scratch of the plan build is released now
     void* scratch[] = {tok_key, key_cnt, bidx, key2blk, blk_cnt, blk_pcnt, blk_fill,
-                       tmp, wt_cnt, wr_cnt, wm_cnt};
+                       tmp, wt_cnt, wr_cnt, wm_cnt, ptok};
     for (void* ptr : scratch) {
         auto it = std::find(p->owned.begin(), p->owned.end(), ptr);
         if (it != p->owned.end()) {

@@ -6,8 +6,10 @@
 // One CTA per occupied block. Each thread owns one 16-byte column group of the token rows (all
 // heads of a token are contiguous), so every token row is read with fully coalesced 128-bit loads;
 // sums are fp32. For the tensor-core path the same pass also writes the rows into the padded,
-// head-major, block-ordered copies K_s, V_s [H, Npad, D] that the attention tiles read, and the
-// compressed tokens a second time in the same order.
+// head-major, block-ordered copies K_s, V_s [H, Nks, D] that the attention tiles read, and the
+// compressed tokens a second time in the same order. A block of at most kPoolMaxTokens tokens is
+// written twice: at its padded rows and, packed with the other small blocks of its sequence, in
+// that sequence's pool after all padded rows.
 //
 // Grouped order (16-bit types): rows are taken 8 at a time; a group stores its D/32 column chunks
 // one after the other, each as a 512-byte atom of 8 rows x 64 bytes in which the four 16-byte
@@ -35,8 +37,11 @@ __global__ void __launch_bounds__(1024) k_pool(const T* __restrict__ K, const T*
                                                const float* __restrict__ Wc,
                                                const int32_t* __restrict__ perm,
                                                const int32_t* __restrict__ blk_off,
-                                               const int32_t* __restrict__ blk_poff, int64_t Mb,
-                                               int H, int D, int64_t Npad, T* __restrict__ ks,
+                                               const int32_t* __restrict__ blk_poff,
+                                               const int32_t* __restrict__ blk_tpool,
+                                               const int32_t* __restrict__ blk_seq,
+                                               const int2* __restrict__ seq_pool, int64_t Mb,
+                                               int H, int D, int64_t Nks, T* __restrict__ ks,
                                                T* __restrict__ vs, T* __restrict__ kc,
                                                T* __restrict__ vc, int64_t Mb8,
                                                T* __restrict__ kcg, T* __restrict__ vcg) {
@@ -47,6 +52,8 @@ __global__ void __launch_bounds__(1024) k_pool(const T* __restrict__ K, const T*
     const int groups = HD / kVec;
     const int32_t lo = blk_off[b], n = blk_off[b + 1] - lo;
     const int32_t prow = blk_poff[b];
+    // row of the block's copy in its sequence's pool, -1 if it has none
+    const int32_t trow = kSorted && blk_tpool[b] >= 0 ? 8 * seq_pool[blk_seq[b]].x + blk_tpool[b] : -1;
 
     float sk[kMaxGroupsPerThread][kVec], sv[kMaxGroupsPerThread][kVec];
 #pragma unroll
@@ -72,9 +79,15 @@ __global__ void __launch_bounds__(1024) k_pool(const T* __restrict__ K, const T*
             }
             if (kSorted) {
                 const int col = gidx * kVec, h = col / D, d = col % D;
-                const int64_t dst = (int64_t)h * Npad * D * (int64_t)sizeof(T) + grouped_off(prow + t, d, D);
+                const int64_t hoff = (int64_t)h * Nks * D * (int64_t)sizeof(T);
+                const int64_t dst = hoff + grouped_off(prow + t, d, D);
                 *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ks) + dst) = kq;
                 *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(vs) + dst) = vq;
+                if (trow >= 0) {
+                    const int64_t tdst = hoff + grouped_off(trow + t, d, D);
+                    *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ks) + tdst) = kq;
+                    *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(vs) + tdst) = vq;
+                }
             }
         }
     }
@@ -127,7 +140,8 @@ void run_pool(const Plan* p, const Workspace& w, const void* k, const void* v, c
     auto kern = sorted ? k_pool<T, true> : k_pool<T, false>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kern<<<(unsigned)p->Mb, threads, smem, st>>>(
-        (const T*)k, (const T*)v, wc, p->perm, p->blk_off, p->blk_poff, p->Mb, w.H, w.D, p->Npad,
+        (const T*)k, (const T*)v, wc, p->perm, p->blk_off, p->blk_poff, p->blk_tpool, p->blk_seq,
+        p->seq_pool, p->Mb, w.H, w.D, p->Nks,
         (T*)w.ks, (T*)w.vs, (T*)w.kc, (T*)w.vc, w.Mb8, (T*)w.kcg, (T*)w.vcg);
     note_launch();
 }

@@ -8,7 +8,9 @@
 //   C  the compressed tokens of the sequence (block mean . Wc). Each row keeps a running list of
 //      its top-(k-1) other blocks by compressed logit; the own block is slot 0.
 //   S  the selected tokens: the union over the tile's rows of their k selected blocks, each row
-//      masked to its own k blocks (a row's valid keys are k ranges of the union stream).
+//      masked to its own k blocks (a row's valid keys are k ranges of the union stream). Blocks
+//      of at most 7 tokens come from their sequence's packed pool instead when the tile selects
+//      more of them than the pool has 8-row groups.
 //   W  the tile's window key union (Chebyshev radius r), masked by distance.
 // out = g0 o_cmp + g1 o_sel + g2 o_win is assembled in an fp32 row buffer and written in the
 // input type after phase W.
@@ -17,8 +19,9 @@
 //   warp 0    producer: K and V tiles into two-stage shared-memory rings by 1D bulk copies. The
 //             K/V copies in global memory are stored as 8-row groups already in the tensor cores'
 //             swizzled operand order, so a run of consecutive groups is one copy: the compressed
-//             tokens are one run, each selected block is one run, and the window union is the
-//             plan's list of runs (its per-row key masks come from the plan as well);
+//             tokens are one run, each selected block is one run (or the small blocks together
+//             are the one run of their pool), and the window union is the plan's list of runs
+//             (its per-row key masks come from the plan as well);
 //   warp 1    MMA issuer (one thread): S = Q K^T into one of two TMEM buffers; O += P V with P
 //             read from TMEM (it overwrites S in place);
 //   warps 2-5 softmax, one thread per row (its TMEM lane): S into registers once, mask, running
@@ -184,8 +187,9 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
     if (warp == 0) {
         // ================================ producer ============================================
         // Every phase is a stream of runs of consecutive 8-row groups (compressed tokens: one run;
-        // selected blocks: one run per union block; window: the plan's runs). A 64-key tile takes
-        // the next 8 groups; lane l < 8 copies the part of run ri + l that falls in the tile.
+        // selected blocks: one run per union block, or per kept block plus the pool; window: the
+        // plan's runs). A 64-key tile takes the next 8 groups; lane l < 8 copies the part of run
+        // ri + l that falls in the tile.
         const uint8_t* ksh = static_cast<const uint8_t*>(P.ks) + (int64_t)h * P.Nks * D * 2;
         const uint8_t* vsh = static_cast<const uint8_t*>(P.vs) + (int64_t)h * P.Nks * D * 2;
         const uint8_t* kch = static_cast<const uint8_t*>(P.kcg) + (int64_t)h * P.Mb8 * D * 2;

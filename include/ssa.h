@@ -109,9 +109,10 @@ SSA_API ssa_status_t ssa_plan_varlen(const int32_t* coords, const int64_t* cu_se
 /*
  * Recompute a plan in place for new coordinates with the same token count, sequence layout,
  * grids and radius (e.g. the next refinement pass over a re-voxelised support of equal size).
- * coords: device int32 [N, 3]. The forward workspace is kept when the block count and padded row
- * count are unchanged, so a following ssa_forward allocates nothing. Waits for the device like
- * ssa_plan. On error the plan is left empty (only ssa_plan_destroy is valid).
+ * coords: device int32 [N, 3]. The forward workspace is kept when the block count and the row
+ * count of the block-ordered key/value copies (padded block rows plus each sequence's pool of
+ * blocks of at most 7 tokens) are unchanged, so a following ssa_forward allocates nothing. Waits
+ * for the device like ssa_plan. On error the plan is left empty (only ssa_plan_destroy is valid).
  */
 SSA_API ssa_status_t ssa_plan_rebuild(ssa_plan_t plan, const int32_t* coords, void* stream);
 

@@ -83,6 +83,18 @@ def kernel_traffic(cfg_name, H):
     return t["bytes_per_head"] * H
 
 
+def traffic_source(cfg_name):
+    """Where roofline.traffic comes from, or why it is null."""
+    t = KERNEL_TRAFFIC
+    if t["bytes_per_head"] is None:
+        return "no ncu capture recorded"
+    if cfg_name != t["config"]:
+        return f"captured for {t['config']} only"
+    if kernel_sources_sha256() != t["sources_sha256"]:
+        return "null: the kernel's code changed since the recorded ncu capture"
+    return "ncu dram__bytes_read.sum + dram__bytes_write.sum of a 4-head launch, scaled by heads"
+
+
 def describe(cfg, coords, cu):
     return {
         "workload": f"{cfg.name}: {cfg.description}; H={cfg.H}, D={cfg.D}, {cfg.dtype}, "
@@ -293,6 +305,7 @@ def run_ours(args, rank, world, dist):
         "roofline": {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": kernel_traffic(args.config, cfg.H),
                      "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                     "traffic_source": traffic_source(args.config),
                      "algorithmic_tflop_per_launch": work[dominant] / 1e12,
                      "avg_launch_ms": dom_ms, "peak_source": src},
         "e2e": {"value": N / (e2e * 1e-3), "unit": "tokens/s", "ms_per_step": e2e,

@@ -33,7 +33,9 @@ def test_traffic_is_reported_only_for_the_captured_build(monkeypatch):
     monkeypatch.setattr(bench, "KERNEL_TRAFFIC", rec)
     assert bench.kernel_traffic("pass3", 22) == 22000.0     # scaled by the heads of the launch
     assert bench.kernel_traffic("small", 22) is None        # another workload
+    assert "scaled" in bench.traffic_source("pass3")
     monkeypatch.setattr(bench, "KERNEL_TRAFFIC", dict(rec, sources_sha256="0" * 64))
     assert bench.kernel_traffic("pass3", 22) is None        # the kernel changed since the capture
+    assert bench.traffic_source("pass3").startswith("null")
     monkeypatch.setattr(bench, "KERNEL_TRAFFIC", dict(rec, bytes_per_head=None))
     assert bench.kernel_traffic("pass3", 22) is None

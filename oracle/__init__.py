@@ -79,7 +79,7 @@ def lib():
         L.oracle_backward_dq_rows.argtypes = [
             ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
             c_f32p, c_f32p, c_vp, ctypes.c_int32, ctypes.c_int32, c_i32p, c_i32p, c_i32p,
-            ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_f64p, c_i32p]
+            ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_i32p, c_f64p, c_i32p]
     return _lib
 
 
@@ -221,12 +221,15 @@ def _seq_plan(coords, lo, hi, block, r):
 
 
 def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None,
-            block: int = 8, round_compressed: bool = True, sel_in=None,
-            want_z: bool = False) -> Dict[str, object]:
+            block: int = 8, round_compressed: bool = False, sel_in=None,
+            want_z: bool = False, branches: bool = True) -> Dict[str, object]:
     """Oracle forward for the query rows `rows` (global indices; None = all tokens).
 
     Returns out, o_cmp, o_sel, o_win ([R, H, D] float64), sel ([R, H, k] int32 global block
     indices, -1 = empty slot) and, if want_z, z: list of [H, Mb_seq] scaled compressed logits.
+    sel_in ([R, H, k] global block indices) replaces the selection of the rows. With
+    branches=False only the compressed attention and the selection run: the result has o_cmp
+    and sel, and out / o_sel / o_win are left at zero.
     """
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
@@ -265,8 +268,9 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
                 int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
                 _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p),
                 n_r, _ptr(local, c_i64p), _ptr(sin, c_i32p),
-                _ptr(outs["out"], c_f64p), _ptr(outs["o_cmp"], c_f64p),
-                _ptr(outs["o_sel"], c_f64p), _ptr(outs["o_win"], c_f64p),
+                _ptr(outs["out"] if branches else None, c_f64p), _ptr(outs["o_cmp"], c_f64p),
+                _ptr(outs["o_sel"] if branches else None, c_f64p),
+                _ptr(outs["o_win"] if branches else None, c_f64p),
                 _ptr(sel, c_i32p), _ptr(zc, c_f64p))
             if rc != 0:
                 raise RuntimeError("oracle_forward failed")
@@ -284,8 +288,11 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
 
 
 def backward(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, block: int = 8,
-             round_compressed: bool = True):
-    """Full fp64 backward: (dQ, dK, dV) [N, H, D] of sum(dO * out), selection held fixed."""
+             round_compressed: bool = False, sel=None):
+    """Full fp64 backward: (dQ, dK, dV) [N, H, D] of sum(dO * out), selection held fixed.
+
+    sel ([N, H, k] global block indices, -1 = empty slot) is the selection to hold; None = the
+    oracle's own."""
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     q, dt = _raw(Q)
@@ -297,25 +304,31 @@ def backward(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, bloc
     N, H, D = q.shape
     dQ, dK, dV = (np.zeros((N, H, D)) for _ in range(3))
     L = lib()
+    blk_base = 0
     for s in range(len(cu) - 1):
         lo, hi = int(cu[s]), int(cu[s + 1])
         n = hi - lo
         perm, tok_blk, blk_off, mb, no, ni = _seq_plan(coords, lo, hi, block, r)
-        sel = np.zeros((n, H, topk), np.int32)
         gs = np.ascontiguousarray(g[lo:hi])
-        rc = L.oracle_forward(n, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data,
-                              v[lo:hi].ctypes.data, _ptr(gs, c_f32p), _ptr(w, c_f32p), topk,
-                              int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
-                              _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p),
-                              n, None, None, None, None, None, None, _ptr(sel, c_i32p), None)
-        if rc != 0:
-            raise RuntimeError("oracle_forward failed")
+        if sel is not None:
+            ss = np.asarray(sel, dtype=np.int64)[lo:hi]
+            ssel = np.ascontiguousarray(np.where(ss >= 0, ss - blk_base, -1), dtype=np.int32)
+        else:
+            ssel = np.zeros((n, H, topk), np.int32)
+            rc = L.oracle_forward(n, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data,
+                                  v[lo:hi].ctypes.data, _ptr(gs, c_f32p), _ptr(w, c_f32p), topk,
+                                  int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
+                                  _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p),
+                                  n, None, None, None, None, None, None, _ptr(ssel, c_i32p), None)
+            if rc != 0:
+                raise RuntimeError("oracle_forward failed")
+        blk_base += mb
         a, b, c = (np.zeros((n, H, D)) for _ in range(3))
         rc = L.oracle_backward(n, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data,
                                v[lo:hi].ctypes.data, _ptr(gs, c_f32p), _ptr(w, c_f32p),
                                go[lo:hi].ctypes.data, topk, int(round_compressed),
                                _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p), _ptr(blk_off, c_i32p),
-                               mb, _ptr(no, c_i64p), _ptr(ni, c_i32p), _ptr(sel, c_i32p),
+                               mb, _ptr(no, c_i64p), _ptr(ni, c_i32p), _ptr(ssel, c_i32p),
                                _ptr(a, c_f64p), _ptr(b, c_f64p), _ptr(c, c_f64p))
         if rc != 0:
             raise RuntimeError("oracle_backward failed")
@@ -324,10 +337,12 @@ def backward(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, bloc
 
 
 def backward_dq_rows(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: int, rows,
-                     block: int = 8, round_compressed: bool = True, return_sel: bool = False):
+                     block: int = 8, round_compressed: bool = False, return_sel: bool = False,
+                     sel_in=None):
     """dQ [R, H, D] for the given global rows, evaluated row by row (any size).
 
-    With return_sel, also returns the selection used ([R, H, k] global block indices)."""
+    sel_in ([R, H, k] global block indices) replaces the rows' selection. With return_sel, also
+    returns the selection used ([R, H, k] global block indices)."""
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     q, dt = _raw(Q)
@@ -353,12 +368,16 @@ def backward_dq_rows(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: i
         local = np.ascontiguousarray(rows[pick] - lo)
         out = np.zeros((len(local), H, D))
         sel = np.zeros((len(local), H, topk), np.int32)
+        sin = None
+        if sel_in is not None:
+            si = np.asarray(sel_in, dtype=np.int64)[pick]
+            sin = np.ascontiguousarray(np.where(si >= 0, si - blk_base, -1), dtype=np.int32)
         rc = L.oracle_backward_dq_rows(
             hi - lo, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data, v[lo:hi].ctypes.data,
             _ptr(np.ascontiguousarray(g[lo:hi]), c_f32p), _ptr(w, c_f32p), go[lo:hi].ctypes.data,
             topk, int(round_compressed), _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p),
             _ptr(blk_off, c_i32p), mb, _ptr(no, c_i64p), _ptr(ni, c_i32p), len(local),
-            _ptr(local, c_i64p), _ptr(out, c_f64p), _ptr(sel, c_i32p))
+            _ptr(local, c_i64p), _ptr(sin, c_i32p), _ptr(out, c_f64p), _ptr(sel, c_i32p))
         if rc != 0:
             raise RuntimeError("oracle_backward_dq_rows failed")
         dQ[pick] = out

@@ -34,6 +34,7 @@
  * All functions are re-entrant; OpenMP parallelises over (row, head) pairs.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -369,7 +370,10 @@ static void select_blocks(int64_t mb, const double* z, int32_t own, int32_t k, i
  *   out, o_cmp, o_sel, o_win: [n_rows, H, D];  sel: [n_rows, H, k] (local block indices);
  *   zc: [n_rows, H, Mb] scaled compressed logits.
  * If sel_in is non-NULL ([n_rows, H, k], -1 = empty slot) it replaces the computed selection
- * (used by tests to pin the selection branch with planted block sets).
+ * (used by tests to pin the selection branch with planted block sets, and to evaluate the
+ * branches with another implementation's validated choice among near-tied blocks).
+ * When out, o_sel and o_win are all NULL only steps 3-4 run (compressed attention and the
+ * selection), so the selection of many rows can be had at the cost of the compressed branch.
  */
 int oracle_forward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q, const void* K,
                    const void* V, const float* gates, const float* Wc, int32_t topk,
@@ -438,6 +442,13 @@ int oracle_forward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q
             }
             if (sel)
                 for (int32_t s = 0; s < topk; ++s) sel[(ri * H + h) * topk + s] = s_loc[s];
+
+            /* selection only (no branch output requested): steps 5-7 are not needed */
+            if (!out && !o_sel && !o_win) {
+                if (o_cmp)
+                    for (int32_t d = 0; d < D; ++d) o_cmp[(ri * H + h) * D + d] = oc[d];
+                continue;
+            }
 
             /* 5. one softmax over the tokens of all selected blocks */
             int64_t nk = 0;
@@ -540,7 +551,9 @@ static void attend_backward(int32_t D, const double* q, const double* dO, double
  * with the selection held at `sel` ([n, H, k], local block indices, as produced by
  * oracle_forward for all rows) and the compressed tokens' rounding treated as identity.
  * Compression: dK_j += (1/n_b) * (dKc_b . Wc^T) for every token j of block b; same for V.
- * Parallel over heads (each head's gradients are independent).
+ * Heads are independent and are taken one after the other. Inside a head the query rows are
+ * shared among the threads; each thread adds its rows' key and value gradients into its own
+ * zeroed copy of dK, dV, dKc, dVc, and the copies are summed in thread order at the end.
  */
 int oracle_backward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q, const void* K,
                     const void* V, const float* gates, const float* Wc, const void* dO,
@@ -565,71 +578,115 @@ int oracle_backward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* 
         if (nbr_off[i + 1] - nbr_off[i] > max_keys) max_keys = nbr_off[i + 1] - nbr_off[i];
     if (mb > max_keys) max_keys = mb;
 
-#pragma omp parallel for schedule(dynamic)
+    const int nt = omp_get_max_threads();
+    const size_t tok_elems = (size_t)(n * D + 1), blk_elems = (size_t)(mb * D + 1);
+    double* kall = (double*)malloc(sizeof(double) * tok_elems);
+    double* vall = (double*)malloc(sizeof(double) * tok_elems);
+    double* dkall = (double*)malloc(sizeof(double) * tok_elems * (size_t)nt);  /* one per thread */
+    double* dvall = (double*)malloc(sizeof(double) * tok_elems * (size_t)nt);
+    double* dKc = (double*)malloc(sizeof(double) * blk_elems * (size_t)nt);
+    double* dVc = (double*)malloc(sizeof(double) * blk_elems * (size_t)nt);
+    if (!kall || !vall || !dkall || !dvall || !dKc || !dVc) {
+        free(Kc); free(Vc); free(kall); free(vall); free(dkall); free(dvall); free(dKc); free(dVc);
+        return -1;
+    }
+
     for (int32_t h = 0; h < H; ++h) {
-        double* kall = (double*)malloc(sizeof(double) * (size_t)(n * D));
-        double* vall = (double*)malloc(sizeof(double) * (size_t)(n * D));
-        double* dkall = (double*)calloc((size_t)(n * D), sizeof(double));
-        double* dvall = (double*)calloc((size_t)(n * D), sizeof(double));
-        double* dKc = (double*)calloc((size_t)(mb * D + 1), sizeof(double));
-        double* dVc = (double*)calloc((size_t)(mb * D + 1), sizeof(double));
-        double* q = (double*)malloc(sizeof(double) * (size_t)D);
-        double* go = (double*)malloc(sizeof(double) * (size_t)D);
-        double* dq = (double*)malloc(sizeof(double) * (size_t)D);
-        double* P = (double*)malloc(sizeof(double) * (size_t)(max_keys + 1));
-        double* dP = (double*)malloc(sizeof(double) * (size_t)(max_keys + 1));
-        const double** kr = (const double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
-        const double** vr = (const double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
-        double** dkr = (double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
-        double** dvr = (double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
+#pragma omp parallel for schedule(static)
         for (int64_t j = 0; j < n; ++j)
             for (int32_t d = 0; d < D; ++d) {
                 kall[j * D + d] = load_elem(K, dtype, (j * H + h) * D + d);
                 vall[j * D + d] = load_elem(V, dtype, (j * H + h) * D + d);
             }
-        for (int64_t i = 0; i < n; ++i) {
-            const float* g = &gates[(i * H + h) * 3];
-            for (int32_t d = 0; d < D; ++d) {
-                q[d] = load_elem(Q, dtype, (i * H + h) * D + d);
-                go[d] = load_elem(dO, dtype, (i * H + h) * D + d);
-                dq[d] = 0.0;
-            }
-            /* compressed branch: keys Kc_b, values Vc_b */
-            for (int64_t b = 0; b < mb; ++b) {
-                kr[b] = &Kc[(b * H + h) * D];
-                vr[b] = &Vc[(b * H + h) * D];
-                dkr[b] = &dKc[b * D];
-                dvr[b] = &dVc[b * D];
-            }
-            attend_backward(D, q, go, (double)g[0], mb, kr, vr, scale, P, dP, dq, dkr, dvr);
-            /* selected branch */
-            int64_t nk = 0;
-            for (int32_t s = 0; s < topk; ++s) {
-                int32_t b = sel[(i * H + h) * topk + s];
-                if (b < 0) continue;
-                for (int64_t p = blk_off[b]; p < blk_off[b + 1]; ++p) {
-                    int64_t j = perm[p];
+        memset(dkall, 0, sizeof(double) * tok_elems * (size_t)nt);
+        memset(dvall, 0, sizeof(double) * tok_elems * (size_t)nt);
+        memset(dKc, 0, sizeof(double) * blk_elems * (size_t)nt);
+        memset(dVc, 0, sizeof(double) * blk_elems * (size_t)nt);
+
+#pragma omp parallel
+        {
+            const int t = omp_get_thread_num();
+            double* my_dk = dkall + (size_t)t * tok_elems;
+            double* my_dv = dvall + (size_t)t * tok_elems;
+            double* my_dKc = dKc + (size_t)t * blk_elems;
+            double* my_dVc = dVc + (size_t)t * blk_elems;
+            double* q = (double*)malloc(sizeof(double) * (size_t)D);
+            double* go = (double*)malloc(sizeof(double) * (size_t)D);
+            double* dq = (double*)malloc(sizeof(double) * (size_t)D);
+            double* P = (double*)malloc(sizeof(double) * (size_t)(max_keys + 1));
+            double* dP = (double*)malloc(sizeof(double) * (size_t)(max_keys + 1));
+            const double** kr = (const double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
+            const double** vr = (const double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
+            double** dkr = (double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
+            double** dvr = (double**)malloc(sizeof(double*) * (size_t)(max_keys + 1));
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t i = 0; i < n; ++i) {
+                const float* g = &gates[(i * H + h) * 3];
+                for (int32_t d = 0; d < D; ++d) {
+                    q[d] = load_elem(Q, dtype, (i * H + h) * D + d);
+                    go[d] = load_elem(dO, dtype, (i * H + h) * D + d);
+                    dq[d] = 0.0;
+                }
+                /* compressed branch: keys Kc_b, values Vc_b */
+                for (int64_t b = 0; b < mb; ++b) {
+                    kr[b] = &Kc[(b * H + h) * D];
+                    vr[b] = &Vc[(b * H + h) * D];
+                    dkr[b] = &my_dKc[b * D];
+                    dvr[b] = &my_dVc[b * D];
+                }
+                attend_backward(D, q, go, (double)g[0], mb, kr, vr, scale, P, dP, dq, dkr, dvr);
+                /* selected branch */
+                int64_t nk = 0;
+                for (int32_t s = 0; s < topk; ++s) {
+                    int32_t b = sel[(i * H + h) * topk + s];
+                    if (b < 0) continue;
+                    for (int64_t p = blk_off[b]; p < blk_off[b + 1]; ++p) {
+                        int64_t j = perm[p];
+                        kr[nk] = &kall[j * D];
+                        vr[nk] = &vall[j * D];
+                        dkr[nk] = &my_dk[j * D];
+                        dvr[nk] = &my_dv[j * D];
+                        nk += 1;
+                    }
+                }
+                attend_backward(D, q, go, (double)g[1], nk, kr, vr, scale, P, dP, dq, dkr, dvr);
+                /* window branch */
+                nk = 0;
+                for (int64_t tt = nbr_off[i]; tt < nbr_off[i + 1]; ++tt) {
+                    int64_t j = nbr_idx[tt];
                     kr[nk] = &kall[j * D];
                     vr[nk] = &vall[j * D];
-                    dkr[nk] = &dkall[j * D];
-                    dvr[nk] = &dvall[j * D];
+                    dkr[nk] = &my_dk[j * D];
+                    dvr[nk] = &my_dv[j * D];
                     nk += 1;
                 }
+                attend_backward(D, q, go, (double)g[2], nk, kr, vr, scale, P, dP, dq, dkr, dvr);
+                for (int32_t d = 0; d < D; ++d) dQ[(i * H + h) * D + d] = dq[d];
             }
-            attend_backward(D, q, go, (double)g[1], nk, kr, vr, scale, P, dP, dq, dkr, dvr);
-            /* window branch */
-            nk = 0;
-            for (int64_t t = nbr_off[i]; t < nbr_off[i + 1]; ++t) {
-                int64_t j = nbr_idx[t];
-                kr[nk] = &kall[j * D];
-                vr[nk] = &vall[j * D];
-                dkr[nk] = &dkall[j * D];
-                dvr[nk] = &dvall[j * D];
-                nk += 1;
-            }
-            attend_backward(D, q, go, (double)g[2], nk, kr, vr, scale, P, dP, dq, dkr, dvr);
-            for (int32_t d = 0; d < D; ++d) dQ[(i * H + h) * D + d] = dq[d];
+            free(q); free(go); free(dq); free(P); free(dP); free(kr); free(vr); free(dkr); free(dvr);
         }
+
+        /* the threads' partial key / value gradients, summed in thread order into copy 0 */
+#pragma omp parallel for schedule(static)
+        for (int64_t e = 0; e < n * D; ++e) {
+            double sk = 0.0, sv = 0.0;
+            for (int t = 0; t < nt; ++t) {
+                sk += dkall[(size_t)t * tok_elems + (size_t)e];
+                sv += dvall[(size_t)t * tok_elems + (size_t)e];
+            }
+            dkall[e] = sk;
+            dvall[e] = sv;
+        }
+        for (int64_t e = 0; e < mb * D; ++e) {
+            double sk = 0.0, sv = 0.0;
+            for (int t = 0; t < nt; ++t) {
+                sk += dKc[(size_t)t * blk_elems + (size_t)e];
+                sv += dVc[(size_t)t * blk_elems + (size_t)e];
+            }
+            dKc[e] = sk;
+            dVc[e] = sv;
+        }
+
         /* through the compression: Kc_b = mean(K_b) . Wc  =>  dK_j += (1/n_b) dKc_b . Wc^T */
         for (int64_t b = 0; b < mb; ++b) {
             double inv = 1.0 / (double)(blk_off[b + 1] - blk_off[b]);
@@ -651,9 +708,8 @@ int oracle_backward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* 
                 dK[(j * H + h) * D + d] = dkall[j * D + d];
                 dV[(j * H + h) * D + d] = dvall[j * D + d];
             }
-        free(kall); free(vall); free(dkall); free(dvall); free(dKc); free(dVc);
-        free(q); free(go); free(dq); free(P); free(dP); free(kr); free(vr); free(dkr); free(dvr);
     }
+    free(kall); free(vall); free(dkall); free(dvall); free(dKc); free(dVc);
     free(Kc);
     free(Vc);
     return 0;
@@ -662,13 +718,16 @@ int oracle_backward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* 
 /*
  * dQ only, for a set of rows: dQ_i needs nothing but row i's own forward quantities, so it
  * can be evaluated at any size. Same conventions as oracle_backward; dQ is [n_rows, H, D].
+ * sel_in ([n_rows, H, k] local block indices) replaces the computed selection when non-NULL;
+ * sel_out receives the selection used.
  */
 int oracle_backward_dq_rows(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q,
                             const void* K, const void* V, const float* gates, const float* Wc,
                             const void* dO, int32_t topk, int32_t round_compressed,
                             const int32_t* perm, const int32_t* tok_blk, const int32_t* blk_off,
                             int64_t mb, const int64_t* nbr_off, const int32_t* nbr_idx,
-                            int64_t n_rows, const int64_t* rows, double* dQ, int32_t* sel_out) {
+                            int64_t n_rows, const int64_t* rows, const int32_t* sel_in,
+                            double* dQ, int32_t* sel_out) {
     double* Kc = (double*)malloc(sizeof(double) * (size_t)(mb * H * D + 1));
     double* Vc = (double*)malloc(sizeof(double) * (size_t)(mb * H * D + 1));
     if (!Kc || !Vc) return -1;
@@ -713,7 +772,11 @@ int oracle_backward_dq_rows(int64_t n, int32_t H, int32_t D, int32_t dtype, cons
                 vr[b] = &Vc[(b * H + h) * D];
             }
             attend_backward(D, q, go, (double)g[0], mb, kr, vr, scale, P, dP, dq, NULL, NULL);
-            select_blocks(mb, z, tok_blk[i], topk, s_loc);
+            if (sel_in) {
+                for (int32_t s = 0; s < topk; ++s) s_loc[s] = sel_in[(ri * H + h) * topk + s];
+            } else {
+                select_blocks(mb, z, tok_blk[i], topk, s_loc);
+            }
             if (sel_out)
                 for (int32_t s = 0; s < topk; ++s) sel_out[(ri * H + h) * topk + s] = s_loc[s];
             int64_t nk = 0;

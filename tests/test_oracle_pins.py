@@ -11,6 +11,8 @@ The method: Direct3D-S2 summary page, "Technical principles", SSA item
 (partition by 3D coordinates; block compression; top-k blocks by compression
 scores; local window; gated aggregation).
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -489,3 +491,94 @@ def test_backward_gradient_sums():
     ref = (np.einsum("nh,nhd->hd", gd[:, :, 0], dO) @ Wc.astype(np.float64).T
            + np.einsum("nh,nhd->hd", gd[:, :, 1] + gd[:, :, 2], dO))
     np.testing.assert_allclose(dV.sum(axis=0), ref, atol=1e-10)
+
+
+def _random_selection(tok_blk_global, blk_seq, topk, H, seed):
+    """A valid selection that is not the oracle's: slot 0 the own block, then topk-1 distinct
+    other blocks of the token's own sequence drawn at random (-1 where the sequence has fewer)."""
+    rng = np.random.default_rng(seed)
+    N = len(tok_blk_global)
+    sel = np.full((N, H, topk), -1, np.int32)
+    for i in range(N):
+        own = tok_blk_global[i]
+        pool = np.nonzero(blk_seq == blk_seq[own])[0]
+        pool = pool[pool != own]
+        for h in range(H):
+            pick = rng.permutation(pool)[:topk - 1]
+            sel[i, h, 0] = own
+            sel[i, h, 1:1 + len(pick)] = pick
+    return sel
+
+
+def test_backward_with_a_given_selection_matches_finite_differences():
+    # two packed sequences and a random valid selection (global block indices): the backward that
+    # holds this selection is the derivative of the forward that uses it (central differences,
+    # fp64), and dQ by rows with the same selection equals the full backward's rows
+    c1, _ = _tiny_coords()
+    c1 = c1[:120]
+    c2 = np.ascontiguousarray(c1[::2][:, [2, 0, 1]])
+    c = np.concatenate([c1, c2])
+    cu = np.array([0, len(c1), len(c)])
+    N, H, D, topk, r = len(c), 2, 8, 3, 1
+    rng = np.random.default_rng(160)
+    q, k, v, dO = (rng.standard_normal((N, H, D)) for _ in range(4))
+    Wc = (rng.standard_normal((D, D)) / np.sqrt(D)).astype(np.float32)
+    g = _gates(N, H, None, seed=13)
+    p = oracle.plan(c, cu, r=r)
+    sel = _random_selection(p["tok_blk"], p["blk_seq"], topk, H, seed=161)
+    own = oracle.forward(c, cu, q, k, v, g, Wc, topk, r)["sel"]
+    assert not np.array_equal(np.sort(own, 2), np.sort(sel, 2))   # a different choice
+    dQ, dK, dV = oracle.backward(c, cu, q, k, v, g, Wc, dO, topk, r, sel=sel)
+
+    def loss(qq, kk, vv):
+        return float((oracle.forward(c, cu, qq, kk, vv, g, Wc, topk, r, sel_in=sel)["out"] * dO).sum())
+
+    eps = 1e-6
+    for name, x, grad in (("q", q, dQ), ("k", k, dK), ("v", v, dV)):
+        for t in rng.choice(x.size, 10, replace=False):
+            xp, xm = x.copy(), x.copy()
+            xp.flat[t] += eps
+            xm.flat[t] -= eps
+            args_p = [xp if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            args_m = [xm if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad.flat[t]) <= 1e-6 * max(1.0, abs(fd)), (name, t, fd, grad.flat[t])
+    rows = np.array([0, 7, len(c1) - 1, len(c1), N - 1])
+    dq, used = oracle.backward_dq_rows(c, cu, q, k, v, g, Wc, dO, topk, r, rows, sel_in=sel[rows],
+                                       return_sel=True)
+    assert np.array_equal(used, sel[rows])
+    np.testing.assert_allclose(dq, dQ[rows], atol=1e-13)
+
+
+def test_selection_only_mode_gives_the_same_selection_and_compressed_branch():
+    c, q, k, v, Wc = _tiny_inputs(seed=170)
+    g = _gates(len(c), 2, None, seed=14)
+    full = run(c, q, k, v, g, Wc, 4, 2, want_z=True)
+    part = run(c, q, k, v, g, Wc, 4, 2, want_z=True, branches=False)
+    assert np.array_equal(full["sel"], part["sel"])
+    np.testing.assert_array_equal(full["o_cmp"], part["o_cmp"])
+    for a, b in zip(full["z"], part["z"]):
+        np.testing.assert_array_equal(a, b)
+    assert not part["out"].any() and not part["o_sel"].any() and not part["o_win"].any()
+
+
+def test_backward_is_the_same_with_any_thread_count():
+    # the key / value gradients are summed over per-thread copies; with one thread or several the
+    # result agrees to rounding
+    import subprocess
+    import sys
+    code = ("import numpy as np, sys; sys.path.insert(0, %r); import oracle, workloads;"
+            "c, cu, g = workloads.make_coords(workloads.CONFIGS['tiny']); N = len(c);"
+            "r = np.random.default_rng(180); q, k, v, d = (r.standard_normal((N, 2, 8)) for _ in range(4));"
+            "W = (r.standard_normal((8, 8)) / 3).astype(np.float32); gt = r.random((N, 2, 3)).astype(np.float32);"
+            "out = oracle.backward(c, cu, q, k, v, gt, W, d, 4, 2);"
+            "np.save(sys.argv[1], np.stack(out))") % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))),)
+    import tempfile
+    res = []
+    with tempfile.TemporaryDirectory() as tmp:
+        for threads in ("1", "5"):
+            f = os.path.join(tmp, f"g{threads}.npy")
+            env = dict(os.environ, OMP_NUM_THREADS=threads)
+            subprocess.check_call([sys.executable, "-c", code, f], env=env)
+            res.append(np.load(f))
+    np.testing.assert_allclose(res[0], res[1], rtol=0, atol=1e-12)

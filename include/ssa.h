@@ -78,9 +78,12 @@ typedef void (*ssa_free_fn)(void* ptr, void* stream, void* ctx);
 SSA_API ssa_status_t ssa_set_allocator(ssa_alloc_fn alloc, ssa_free_fn release, void* ctx);
 
 /*
- * Build the plan of one sequence: rows a1 (block partition) and a2 (coordinate hash and window
- * neighbour lists) of the method (Direct3D-S2 model page, "What is Direct3D-S2?": tokens are
- * partitioned by 3D coordinates; summary page, SSA item: local window operations).
+ * Build the plan of one sequence: the block partition and the window neighbour lists.
+ * Direct3D-S2 model page, "What is Direct3D-S2?": SSA partitions the sparse tokens into blocks
+ * by their 3D coordinates. Direct3D-S2 summary page, "Technical principles of Direct3D-S2", SSA
+ * item: the local window branch attends to nearby tokens. Blocks are the occupied aligned 8^3
+ * cells in lexicographic (bx, by, bz) order; the window of a token is every token of its
+ * sequence within Chebyshev distance r (itself included).
  *   coords: device int32 [n, 3] voxel coordinates (x, y, z), each in [0, grid[axis]).
  *   n:      number of tokens (>= 1).
  *   grid:   host int32[3] grid extent.
@@ -139,7 +142,12 @@ SSA_API ssa_status_t ssa_plan_export(ssa_plan_t plan, int32_t* perm, int32_t* to
                              int32_t* nbr_idx, void* stream);
 
 /*
- * Forward pass (rows a3-a8): out = g0*o_cmp + g1*o_sel + g2*o_win for every token and head.
+ * Forward pass: out = g0*o_cmp + g1*o_sel + g2*o_win for every token and head.
+ * Direct3D-S2 summary page, "Technical principles of Direct3D-S2", SSA item: each block is
+ * compressed into a block-level token (here block mean times Wc), important blocks are selected
+ * from the compression module's attention scores (own block plus the top k-1 others), the local
+ * window adds fine detail, and the three outputs are aggregated with gating scores (given here
+ * as the `gates` input).
  *   q, k, v:  device [N, H, D] of dtype.
  *   gates:    device fp32 [N, H, 3].
  *   wc:       device fp32 [D, D].
@@ -156,12 +164,20 @@ SSA_API ssa_status_t ssa_forward(ssa_plan_t plan, const void* q, const void* k, 
                          const float* gates, const float* wc, int32_t heads, int32_t head_dim,
                          ssa_dtype_t dtype, int32_t topk, void* out, void* stream);
 
-/* As ssa_forward, and also writes the selected blocks: sel_out device int32 [N, H, k] (global
- * block indices; slot 0 = own block; -1 = empty slot). */
+/*
+ * As ssa_forward, and also writes what the three branches produced (same passage as
+ * ssa_forward). Every extra output is optional (NULL = not written):
+ *   sel_out: device int32 [N, H, k], the selected blocks (global block indices; slot 0 = own
+ *            block, then the others by descending compressed score; -1 = empty slot);
+ *   o_cmp, o_sel, o_win: device fp32 [N, H, D] in token order, each branch's normalised
+ *            attention output before the gates (the kernels' fp32 accumulators).
+ * Same errors and stream behaviour as ssa_forward.
+ */
 SSA_API ssa_status_t ssa_forward_debug(ssa_plan_t plan, const void* q, const void* k, const void* v,
                                const float* gates, const float* wc, int32_t heads,
                                int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
-                               int32_t* sel_out, void* stream);
+                               int32_t* sel_out, float* o_cmp, float* o_sel, float* o_win,
+                               void* stream);
 
 /*
  * ssa_forward on HOST buffers: copies q, k, v, gates, wc (host) to plan-owned device buffers,
@@ -174,7 +190,9 @@ SSA_API ssa_status_t ssa_forward_host(ssa_plan_t plan, const void* q, const void
                               void* stream);
 
 /*
- * Backward pass (row a9): gradients of sum(dO * out) with respect to q, k, v, with the block
+ * Backward pass (Direct3D-S2 model page, "What is Direct3D-S2?" and "Technical snapshot": the
+ * method trains through SSA, with a faster backward than baseline sparse attention): gradients
+ * of sum(dO * out) with respect to q, k, v, with the block
  * selection held fixed (it is not differentiable) and the compressed tokens' rounding treated as
  * identity. dq, dk, dv: device [N, H, D] of dtype. Accumulates in fp32 (CUDA cores); intended for
  * correctness, not speed. Queues work and returns without waiting.

@@ -4,8 +4,8 @@ Argument marshalling only. Every step of the method runs in the library's CUDA k
 provides device memory and the current stream. There is no CPU fallback: importing this package
 without the built library raises.
 
-    plan = ssa.Plan(coords, grid=(192, 192, 192), r=3)          # rows a1, a2
-    out = plan.forward(q, k, v, gates, wc, topk=16)             # rows a3-a8
+    plan = ssa.Plan(coords, grid=(192, 192, 192), r=3)          # block partition, window lists
+    out = plan.forward(q, k, v, gates, wc, topk=16)             # three branches, gated sum
 """
 from __future__ import annotations
 
@@ -45,7 +45,8 @@ _SIGS = {
     "ssa_plan_info": [_vp, _vp, _vp, _vp, _vp],
     "ssa_plan_export": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "ssa_forward": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp],
-    "ssa_forward_debug": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "ssa_forward_debug": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
+                          _vp, _vp],
     "ssa_forward_host": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp],
     "ssa_backward": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "ssa_last_device_status": [_vp, _vp],
@@ -92,11 +93,16 @@ def block_offsets_noalloc(coords: torch.Tensor, grid, stream=None):
     for x in grid:
         nb *= (int(x) + 7) // 8
     cap = min(n, nb) + 1
-    blk_off = torch.empty(cap, dtype=torch.int32, device=c.device)
-    nblk = torch.empty(1, dtype=torch.int32, device=c.device)
-    _check(lib.ssa_block_offsets_noalloc(c.data_ptr(), n, g, blk_off.data_ptr(), cap, nblk.data_ptr(),
-                                         _stream(stream)), "ssa_block_offsets_noalloc")
-    k = int(nblk.item())
+    # the library finds its scratch array on the current device: make it the coordinates' device
+    with torch.cuda.device(c.device):
+        blk_off = torch.empty(cap, dtype=torch.int32, device=c.device)
+        nblk = torch.empty(1, dtype=torch.int32, device=c.device)
+        st = torch.cuda.current_stream() if stream is None else stream
+        _check(lib.ssa_block_offsets_noalloc(c.data_ptr(), n, g, blk_off.data_ptr(), cap,
+                                             nblk.data_ptr(), st.cuda_stream),
+               "ssa_block_offsets_noalloc")
+        st.synchronize()   # the count is read on the host: wait for the stream the work went to
+        k = int(nblk.item())
     return (blk_off[:k + 1] if k >= 0 else blk_off[:0]), k
 
 
@@ -230,16 +236,26 @@ class Plan:
         return dt, q.shape[1], q.shape[2]
 
     def forward(self, q, k, v, gates, wc, topk: int, out: Optional[torch.Tensor] = None,
-                return_sel: bool = False):
+                return_sel: bool = False, return_branches: bool = False):
+        """out [N, H, D]; with return_sel also the selection [N, H, k] (int32, global block
+        indices); with return_branches also (o_cmp, o_sel, o_win), fp32 [N, H, D] each."""
         dt, H, D = self._args(q, k, v, gates, wc)
         out = torch.empty_like(q) if out is None else _dev(out, dt)
         st = _stream(self.stream)
-        if return_sel:
-            sel = torch.empty(self.N, H, topk, dtype=torch.int32, device=q.device)
+        if return_sel or return_branches:
+            sel = torch.empty(self.N, H, topk, dtype=torch.int32, device=q.device) if return_sel else None
+            br = [torch.empty(self.N, H, D, dtype=torch.float32, device=q.device)
+                  for _ in range(3)] if return_branches else [None] * 3
             _check(lib.ssa_forward_debug(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                          gates.data_ptr(), wc.data_ptr(), H, D, _DTYPE[dt], topk,
-                                         out.data_ptr(), sel.data_ptr(), st), "ssa_forward_debug")
-            return out, sel
+                                         out.data_ptr(), _ptr(sel), *[_ptr(b) for b in br], st),
+                   "ssa_forward_debug")
+            res = (out,)
+            if return_sel:
+                res += (sel,)
+            if return_branches:
+                res += (tuple(br),)
+            return res
         _check(lib.ssa_forward(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), gates.data_ptr(),
                                wc.data_ptr(), H, D, _DTYPE[dt], topk, out.data_ptr(), st),
                "ssa_forward")

@@ -291,7 +291,8 @@ ssa_status_t check_forward_args(Plan* p, const void* q, const void* k, const voi
 
 ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, const float* gates,
                          const float* wc, int32_t H, int32_t D, ssa_dtype_t dt, int32_t topk,
-                         void* out, int32_t* sel_out, cudaStream_t st) {
+                         void* out, int32_t* sel_out, cudaStream_t st,
+                         const BranchOut& bo = BranchOut()) {
     ssa_status_t rc = ensure_workspace(p, H, D, dt, topk, st);
     if (rc != SSA_OK) return rc;
     const Workspace& w = p->ws;
@@ -303,9 +304,9 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
     if (dt == SSA_F32) {
         // the CUDA-core path walks the per-token neighbour lists
         if ((rc = ensure_neighbours(p, st)) != SSA_OK) return rc;
-        launch_forward_simt(p, w, q, k, v, gates, out, st);
+        launch_forward_simt(p, w, q, k, v, gates, out, bo, st);
     }
-    else if ((rc = launch_forward_tc(p, w, q, gates, out, st)) != SSA_OK) return rc;
+    else if ((rc = launch_forward_tc(p, w, q, gates, out, bo, st)) != SSA_OK) return rc;
     trace_step("forward", st);
     if (sel_out) launch_export_sel(p, w, sel_out, st);
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
@@ -433,12 +434,16 @@ ssa_status_t ssa_forward(ssa_plan_t p, const void* q, const void* k, const void*
 ssa_status_t ssa_forward_debug(ssa_plan_t p, const void* q, const void* k, const void* v,
                                const float* gates, const float* wc, int32_t heads,
                                int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
-                               int32_t* sel_out, void* stream) {
+                               int32_t* sel_out, float* o_cmp, float* o_sel, float* o_win,
+                               void* stream) {
     ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out);
     if (rc != SSA_OK) return rc;
-    if (!sel_out) return SSA_ERR_INVALID_ARG;
+    BranchOut bo;
+    bo.o[0] = o_cmp;
+    bo.o[1] = o_sel;
+    bo.o[2] = o_win;
     return run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, sel_out,
-                       (cudaStream_t)stream);
+                       (cudaStream_t)stream, bo);
 }
 
 ssa_status_t ssa_forward_host(ssa_plan_t p, const void* q, const void* k, const void* v,

@@ -39,6 +39,7 @@ struct FwdParams {
     int32_t* sel;
     float* base;
     void* out;
+    float* bout[3];   // optional per-branch outputs (fp32, token order), null when not wanted
     int32_t* status;
     int64_t N, Nks, Mb, Mb8;
     int H, k, r;

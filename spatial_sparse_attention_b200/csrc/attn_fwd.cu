@@ -13,7 +13,7 @@
 //      more of them than the pool has 8-row groups.
 //   W  the tile's window key union (Chebyshev radius r), masked by distance.
 // out = g0 o_cmp + g1 o_sel + g2 o_win is assembled in an fp32 row buffer and written in the
-// input type after phase W.
+// input type after phase W. On request each phase also writes its normalised output (fp32).
 //
 // Warp roles (192 threads):
 //   warp 0    producer: K and V tiles into two-stage shared-memory rings by 1D bulk copies. The
@@ -373,11 +373,21 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
                     tc::fence_after_sync();
                     const float f = row_ok ? gt[ph_end] / l : 0.0f;
                     T* orow = reinterpret_cast<T*>(P.out) + ((int64_t)tok * H + h) * D;
+                    // optional branch output (normalised, before the gate), token order
+                    float* bo = P.bout[ph_end];
+                    if (bo) bo += ((int64_t)tok * H + h) * D;
+                    const float il = 1.0f / l;
 #pragma unroll 1
                     for (int d0 = 0; d0 < D; d0 += 32) {
                         float o[32];
                         tc::tmem_ld32(o_tm + d0, o);   // warp-collective
                         if (!row_ok) continue;
+                        if (bo) {
+#pragma unroll
+                            for (int e = 0; e < 32; e += 4)
+                                *reinterpret_cast<float4*>(bo + d0 + e) =
+                                    make_float4(o[e] * il, o[e + 1] * il, o[e + 2] * il, o[e + 3] * il);
+                        }
 #pragma unroll
                         for (int e = 0; e < 32; e += 8) {
                             float4 a = make_float4(o[e] * f, o[e + 1] * f, o[e + 2] * f, o[e + 3] * f);
@@ -719,7 +729,7 @@ ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, int64_t mb, cudaStr
 }  // namespace
 
 ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
-                               void* out, cudaStream_t st) {
+                               void* out, const BranchOut& bo, cudaStream_t st) {
     const bool bf16 = w.dtype == SSA_BF16;
     int64_t max_seq_blocks = 0;
     for (size_t s = 0; s + 1 < p->seq_blk.size(); ++s)
@@ -751,6 +761,7 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.sel = w.sel;
     P.base = w.base;
     P.out = out;
+    for (int b = 0; b < 3; ++b) P.bout[b] = bo.o[b];
     P.status = p->d_status;
     P.N = p->N;
     P.Nks = p->Nks;

@@ -1,5 +1,5 @@
-// fp32 forward of Spatial Sparse Attention on the CUDA cores (rows a4-a8 for fp32 inputs, where
-// the fp32 tolerance rules out 16-bit tensor-core operands). One warp per (token, head); lanes
+// fp32 forward of Spatial Sparse Attention on the CUDA cores: the three branches and the gated
+// sum for fp32 inputs, where the fp32 tolerance rules out 16-bit tensor-core operands. One warp per (token, head); lanes
 // split the head dimension; every branch is an online softmax over its key list:
 //   compressed tokens of the sequence (with the running top-(k-1) of the other blocks),
 //   the tokens of the selected blocks (own block first), the window neighbour list.
@@ -29,6 +29,7 @@ struct SimtParams {
     const int32_t* nbr_idx;
     int32_t* sel;
     float* out;
+    float* bout[3];   // optional per-branch outputs (o_cmp, o_sel, o_win), null when not wanted
     int64_t N, Mb;
     int H, D, topk, B;
     float scale;
@@ -148,12 +149,24 @@ __global__ void __launch_bounds__(kWarps * 32) k_forward_simt(const SimtParams P
         const int d = lane + 32 * t;
         if (d < D) P.out[(i * H + h) * D + d] = a0 * cmp.o[t] + a1 * sel.o[t] + a2 * win.o[t];
     }
+    const Online* br[3] = {&cmp, &sel, &win};
+#pragma unroll
+    for (int b = 0; b < 3; ++b) {
+        if (!P.bout[b]) continue;
+        const float il = 1.0f / br[b]->l;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int d = lane + 32 * t;
+            if (d < D) P.bout[b][(i * H + h) * D + d] = br[b]->o[t] * il;
+        }
+    }
 }
 
 }  // namespace
 
 void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const void* k,
-                         const void* v, const float* gates, void* out, cudaStream_t st) {
+                         const void* v, const float* gates, void* out, const BranchOut& bo,
+                         cudaStream_t st) {
     SimtParams P;
     P.q = (const float*)q;
     P.k = (const float*)k;
@@ -171,6 +184,7 @@ void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const
     P.nbr_idx = p->nbr_idx;
     P.sel = w.sel;
     P.out = (float*)out;
+    for (int b = 0; b < 3; ++b) P.bout[b] = bo.o[b];
     P.N = p->N;
     P.Mb = p->Mb;
     P.H = w.H;

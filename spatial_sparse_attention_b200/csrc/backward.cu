@@ -1,4 +1,4 @@
-// Backward of Spatial Sparse Attention (row a9; Direct3D-S2 model page, "What is Direct3D-S2?":
+// Backward of Spatial Sparse Attention (Direct3D-S2 model page, "What is Direct3D-S2?":
 // the method has a backward pass, reported ~9.6x faster than baseline sparse attention).
 // Gradients of L = sum(dO * out) with respect to Q, K, V, with the block selection held at the
 // forward's choice and the rounding of the compressed tokens treated as identity.

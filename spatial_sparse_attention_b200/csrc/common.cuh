@@ -169,13 +169,20 @@ ssa_status_t ensure_neighbours(Plan* p, cudaStream_t s);
 void launch_pool(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,
                  cudaStream_t s);
 
+// Per-branch outputs of the forward, fp32 [N, H, D] in token order each: o_cmp, o_sel, o_win
+// (normalised branch attention outputs before the gates). Any entry may be null.
+struct BranchOut {
+    float* o[3] = {nullptr, nullptr, nullptr};
+};
+
 // attn_simt.cu (fp32 path)
 void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const void* k,
-                         const void* v, const float* gates, void* out, cudaStream_t s);
+                         const void* v, const float* gates, void* out, const BranchOut& bo,
+                         cudaStream_t s);
 
 // attn_fwd.cu (bf16 / fp16 path): the fused tensor-core forward
 ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
-                               void* out, cudaStream_t s);
+                               void* out, const BranchOut& bo, cudaStream_t s);
 
 // backward.cu
 ssa_status_t launch_backward(Plan* p, const Workspace& w, const void* q, const void* k,

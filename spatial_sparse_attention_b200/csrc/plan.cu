@@ -1,5 +1,4 @@
-// Plan kernels: coordinate-block partition (row a1) and coordinate hash + window neighbour lists
-// (row a2).
+// Plan kernels: coordinate-block partition and coordinate hash + window neighbour lists.
 //
 // Direct3D-S2 model page, "What is Direct3D-S2?": SSA partitions sparse tokens by their 3D
 // coordinates. Direct3D-S2 summary page, "Technical principles", SSA item: compression per

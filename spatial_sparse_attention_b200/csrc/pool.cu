@@ -1,4 +1,4 @@
-// Compression pooling (row a3): Kc_b = mean_{j in b}(K_j) . Wc and Vc_b likewise, per head, with
+// Compression pooling: Kc_b = mean_{j in b}(K_j) . Wc and Vc_b likewise, per head, with
 // one D x D map Wc shared by K, V and all heads (Direct3D-S2 summary page, "Technical
 // principles", SSA item: block-level tokens from a compression of each block; the concrete
 // mean-then-linear-map form is the formulation this library implements).

@@ -1,8 +1,11 @@
-"""Forward parity (rows a3-a8) of the CUDA path against the fp64 oracle, through the C ABI.
+"""Forward parity (pooling, the three branches, gated combine) of the CUDA path against the fp64
+oracle, through the C ABI.
 
-Small configurations are compared on every output element; the full-size configurations
-(80k, 110k and the 340k-token varlen batch, H=22, D=96, fp16) on 512 seeded rows per sequence,
-in the same launch configuration the benchmark times.
+Every compared row is compared on every element, against the oracle evaluated on the GPU's
+selection once that selection has been validated (near ties only). Small configurations: every
+row and head, and the three branch outputs. Full-size configurations (80k, 110k and the 340k-token
+varlen batch, H=22, D=96, fp16, in the launch configuration the benchmark times): every row of a
+seeded subset of heads, and every head of rows drawn from every 128-token query tile.
 """
 import numpy as np
 import pytest
@@ -10,49 +13,77 @@ import torch
 
 import oracle
 import workloads
-from ssa_testlib import (blk_base_of_rows, check_close, coords_of, make_plan, selection_agreement,
-                         tensors_of, to_gpu)
+from ssa_testlib import (check_close, coords_of, make_plan, oracle_on_gpu_selection, tensors_of,
+                         tile_rows, to_gpu)
 
 pytestmark = pytest.mark.gpu
 
+BRANCHES = ("o_cmp", "o_sel", "o_win")
 
-def gpu_forward(plan, t, topk):
+
+def gpu_forward(plan, t, topk, branches=False):
+    """(out, sel, (o_cmp, o_sel, o_win) or None) as CUDA tensors."""
     g = to_gpu(t)
-    out, sel = plan.forward(g["Q"], g["K"], g["V"], g["gates"], g["Wc"], topk, return_sel=True)
+    res = plan.forward(g["Q"], g["K"], g["V"], g["gates"], g["Wc"], topk, return_sel=True,
+                       return_branches=branches)
     torch.cuda.synchronize()
     assert plan.status() == 0
-    return out.double().cpu().numpy(), sel.cpu().numpy()
+    return res[0], res[1], (res[2] if branches else None)
 
 
-def compare(name_or_cfg, coords, cu, grids, t, topk, r, dtype, rows=None, max_mismatch=0.01):
+def _pick(x, rows, heads):
+    """Rows and heads of a CUDA tensor [N, H, D] as fp64 numpy."""
+    y = x[torch.from_numpy(np.asarray(rows)).to(x.device)]
+    if heads is not None:
+        y = y[:, list(heads)]
+    return y.double().cpu().numpy()
+
+
+def compare(name, coords, cu, grids, t, topk, r, dtype, rows=None, heads=None, branches=False):
     plan = make_plan(coords, cu, grids, r)
-    out, sel = gpu_forward(plan, t, topk)
-    ref = oracle.forward(coords, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], topk, r,
-                         rows=rows, want_z=True)
-    rows = ref["rows"]
+    out, sel, br = gpu_forward(plan, t, topk, branches)
     bs = plan.export()["blk_seq"].cpu().numpy()
-    mism, rep = selection_agreement(sel[rows], ref["sel"], ref["z"], blk_base_of_rows(cu, rows, bs),
-                                    dtype)
-    assert rep["mismatched"] <= max_mismatch * rep["rows"], rep
-    keep = ~mism
-    check_close(out[rows][keep], ref["out"][keep], dtype, f"{name_or_cfg} out")
-    return plan, out, sel, ref, rep
+    ref, rep = oracle_on_gpu_selection(coords, cu, t, topk, r, sel.cpu().numpy(), bs, dtype,
+                                       rows=rows, heads=heads)
+    R = ref["rows"]
+    check_close(_pick(out, R, heads), ref["out"], dtype, f"{name} out")
+    if branches:
+        for x, nm in zip(br, BRANCHES):
+            check_close(_pick(x, R, heads), ref[nm], dtype, f"{name} {nm}")
+    return plan, out, sel, ref, br
 
 
 @pytest.mark.parametrize("name", ["tiny", "small"])
 def test_forward_full_output(name):
     cfg = workloads.CONFIGS[name]
     c, cu, g = coords_of(name)
-    compare(name, c, cu, g, tensors_of(name), cfg.topk, cfg.radius, cfg.dtype)
+    compare(name, c, cu, g, tensors_of(name), cfg.topk, cfg.radius, cfg.dtype, branches=True)
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name", ["pass1", "pass3", "varlen"])
-def test_forward_full_size_sampled_rows(name):
+def test_forward_full_size_every_query_tile(name):
+    """Every head of rows from every query tile (one per 32-row quarter plus the tile's last row),
+    so that no tile of the union build, the pool compaction or the window masks goes unchecked."""
     cfg = workloads.CONFIGS[name]
     c, cu, g = coords_of(name)
-    rows = np.concatenate(workloads.stratified_rows(cu, 512, seed=cfg.index * 1000 + 99))
-    compare(name, c, cu, g, tensors_of(name), cfg.topk, cfg.radius, cfg.dtype, rows=rows)
+    perm = oracle.plan(c, cu, 8, cfg.radius)["perm"]
+    rows = tile_rows(perm, cu, seed=cfg.index * 1000 + 99)
+    compare(name, c, cu, g, tensors_of(name), cfg.topk, cfg.radius, cfg.dtype, rows=rows,
+            branches=True)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["pass1", "pass3", "varlen"])
+def test_forward_full_size_every_row(name):
+    """Every row of the full-size output for a seeded subset of heads (heads are independent:
+    the oracle runs on those heads alone)."""
+    cfg = workloads.CONFIGS[name]
+    c, cu, g = coords_of(name)
+    n_heads = 1 if name == "varlen" else 2
+    heads = sorted(np.random.default_rng(cfg.index * 1000 + 98).choice(cfg.H, n_heads,
+                                                                        replace=False).tolist())
+    compare(name, c, cu, g, tensors_of(name), cfg.topk, cfg.radius, cfg.dtype, heads=heads)
 
 
 def _branch_inputs(name, dtype):
@@ -68,12 +99,25 @@ def _branch_inputs(name, dtype):
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("branch", [0, 1, 2])
 def test_each_branch_alone(dtype, branch):
-    """One-hot gates isolate the compressed, selected and window branches."""
+    """One-hot gates isolate the compressed, selected and window branches in the gated sum."""
     cfg, c, cu, g, t = _branch_inputs("small", dtype)
     gates = torch.zeros_like(t["gates"])
     gates[:, :, branch] = 1.0
     t["gates"] = gates
     compare(f"branch{branch}", c, cu, g, t, cfg.topk, cfg.radius, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_branch_outputs_with_mixed_gates(dtype):
+    """The three branch outputs of ssa_forward_debug, with random gates, each against the oracle's
+    o_cmp, o_sel, o_win; and the gated sum of the GPU's branch outputs against its out."""
+    name = "tiny" if dtype == "f32" else "small"
+    cfg, c, cu, g, t = _branch_inputs(name, dtype)
+    plan, out, sel, ref, br = compare(f"branches {dtype}", c, cu, g, t, cfg.topk, cfg.radius,
+                                      dtype, branches=True)
+    gates = t["gates"].cuda()
+    mix = sum(gates[:, :, i:i + 1] * br[i] for i in range(3))
+    check_close(out.double().cpu().numpy(), mix.double().cpu().numpy(), dtype, "gated sum")
 
 
 @pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
@@ -93,7 +137,8 @@ def test_planted_topk_is_exact(dtype):
              gates=torch.rand(N, H, 3, generator=torch.Generator().manual_seed(4)),
              Wc=torch.eye(D))
     plan = make_plan(c, cu, g, 2)
-    out, sel = gpu_forward(plan, t, topk)
+    out, sel, _ = gpu_forward(plan, t, topk)
+    out, sel = out.double().cpu().numpy(), sel.cpu().numpy()
     exp = np.full((N, H, topk), -1)
     for i in range(N):
         for h in range(H):
@@ -117,7 +162,8 @@ def test_fewer_blocks_than_k_and_dense_limit(dtype):
     gates = torch.zeros_like(t["gates"])
     gates[:, :, 1] = 1.0
     t["gates"] = gates
-    plan, out, sel, ref, rep = compare("dense", c, cu, g, t, mb + 2, 2, dtype)
+    plan, out, sel, ref, _ = compare("dense", c, cu, g, t, mb + 2, 2, dtype)
+    out, sel = out.double().cpu().numpy(), sel.cpu().numpy()
     assert np.all(sel[:, :, mb:] == -1)
     # textbook dense attention over all tokens (library routine, fp64)
     q, k, v = (x.double().permute(1, 0, 2) for x in (t["Q"], t["K"], t["V"]))

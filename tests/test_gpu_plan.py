@@ -1,4 +1,4 @@
-"""Plan parity (rows a1, a2): the GPU block partition and window lists are bit-exact with the
+"""Plan parity (block partition and window lists): the GPU block partition and window lists are bit-exact with the
 oracle's, through the C ABI (ssa_plan / ssa_plan_varlen / ssa_plan_export)."""
 import numpy as np
 import pytest

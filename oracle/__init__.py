@@ -80,6 +80,12 @@ def lib():
             ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
             c_f32p, c_f32p, c_vp, ctypes.c_int32, ctypes.c_int32, c_i32p, c_i32p, c_i32p,
             ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_i32p, c_f64p, c_i32p]
+        L.oracle_rope_split.restype = None
+        L.oracle_rope_split.argtypes = [ctypes.c_int32, c_i32p, c_i32p, c_i32p]
+        L.oracle_qk_prologue.restype = ctypes.c_int
+        L.oracle_qk_prologue.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                         ctypes.c_int32, c_vp, c_i32p, c_f32p, ctypes.c_double,
+                                         ctypes.c_double, c_f64p]
     return _lib
 
 
@@ -220,17 +226,59 @@ def _seq_plan(coords, lo, hi, block, r):
     return perm, tok_blk, blk_off, len(blk_coord), no, ni
 
 
+def rope_split(D: int):
+    """Widths of the x, y and z parts of the head dimension in the 3D rotary embedding."""
+    a, b, c = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    lib().oracle_rope_split(D, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+    return a.value, b.value, c.value
+
+
+def qk_prologue(X, coords, gamma, eps: float = 1e-6, theta: float = 10000.0) -> np.ndarray:
+    """RMS normalisation over the head dimension (weight gamma [D]) followed by the 3D rotary
+    embedding at the tokens' voxel coordinates; X [N, H, D] -> float64 [N, H, D]."""
+    x, dt = _raw(X)
+    N, H, D = x.shape
+    c = np.ascontiguousarray(coords, dtype=np.int32)
+    g = _f32(gamma)
+    out = np.zeros((N, H, D))
+    if lib().oracle_qk_prologue(N, H, D, dt, x.ctypes.data, _ptr(c, c_i32p), _ptr(g, c_f32p),
+                                float(eps), float(theta), _ptr(out, c_f64p)) != 0:
+        raise ValueError("oracle_qk_prologue failed")
+    return out
+
+
+def _exact_f64(t) -> np.ndarray:
+    """Storage values of a CPU tensor or array as float64 (every f32/f16/bf16 value is exact)."""
+    try:
+        import torch
+        if isinstance(t, torch.Tensor):
+            return t.detach().cpu().double().numpy()
+    except ImportError:
+        pass
+    return np.asarray(t, dtype=np.float64)
+
+
 def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None,
             block: int = 8, round_compressed: bool = False, sel_in=None,
-            want_z: bool = False, branches: bool = True) -> Dict[str, object]:
+            want_z: bool = False, branches: bool = True, prologue=None) -> Dict[str, object]:
     """Oracle forward for the query rows `rows` (global indices; None = all tokens).
 
     Returns out, o_cmp, o_sel, o_win ([R, H, D] float64), sel ([R, H, k] int32 global block
     indices, -1 = empty slot) and, if want_z, z: list of [H, Mb_seq] scaled compressed logits.
     sel_in ([R, H, k] global block indices) replaces the selection of the rows. With
     branches=False only the compressed attention and the selection run: the result has o_cmp
-    and sel, and out / o_sel / o_win are left at zero.
+    and sel, and out / o_sel / o_win are left at zero. prologue = dict(q_gamma, k_gamma, eps,
+    theta) first replaces Q and K by qk_prologue(Q), qk_prologue(K) (float64, unrounded).
     """
+    if prologue is not None:
+        pr = dict(prologue)
+        kw = dict(eps=pr.get("eps", 1e-6), theta=pr.get("theta", 10000.0))
+        Q = qk_prologue(Q, coords, pr["q_gamma"], **kw)
+        K = qk_prologue(K, coords, pr["k_gamma"], **kw)
+        V = _exact_f64(V)
+        return forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk, r, rows=rows, block=block,
+                       round_compressed=round_compressed, sel_in=sel_in, want_z=want_z,
+                       branches=branches)
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     q, dt = _raw(Q)

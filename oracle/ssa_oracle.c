@@ -816,3 +816,60 @@ int oracle_backward_dq_rows(int64_t n, int32_t H, int32_t D, int32_t dtype, cons
     free(Vc);
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* 9. attention prologue: RMS normalisation of queries and keys, 3D rotary position embedding  */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * Hi3D v1.0 pipeline page, "Stage 3: sparse flow sampling": the transformer that runs attention
+ * over the sparse voxel tokens applies rotary position embeddings and RMS normalisation to the
+ * self-attention queries and keys. The page gives no formulas; this is the plain reading:
+ *   1. RMS normalisation over the head dimension, one weight vector per operand (gamma, length
+ *      D) shared by all heads: u_d = x_d / sqrt(mean_e x_e^2 + eps) * gamma_d;
+ *   2. 3D rotary embedding with the token's voxel coordinates as positions: the head dimension
+ *      is cut into an x part, a y part and a z part (oracle_rope_split), and channel pair
+ *      (c, c+1) of the part for axis a, j-th pair of that part, is rotated by the angle
+ *      coords[a] * theta^(-2j / width_a):  (u, v) -> (u cos t - v sin t, u sin t + v cos t).
+ */
+
+/* Widths of the x, y and z parts: y and z get 2*floor(D/6) channels each, x the rest. */
+void oracle_rope_split(int32_t D, int32_t* wx, int32_t* wy, int32_t* wz) {
+    int32_t c = 2 * (D / 6);
+    *wy = c;
+    *wz = c;
+    *wx = D - 2 * c;
+}
+
+/* out[n, H, D] (double) = rotary(rmsnorm(X)) for every token and head; X of `dtype`. */
+int oracle_qk_prologue(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* X,
+                       const int32_t* coords, const float* gamma, double eps, double theta,
+                       double* out) {
+    if (D < 2 || (D & 1) || H < 1) return -1;
+    int32_t w[3];
+    oracle_rope_split(D, &w[0], &w[1], &w[2]);
+#pragma omp parallel for schedule(static)
+    for (int64_t ih = 0; ih < n * H; ++ih) {
+        int64_t i = ih / H;
+        double* o = out + ih * D;
+        double ss = 0.0;
+        for (int32_t d = 0; d < D; ++d) {
+            o[d] = load_elem(X, dtype, ih * D + d);
+            ss += o[d] * o[d];
+        }
+        double inv = 1.0 / sqrt(ss / (double)D + eps);
+        for (int32_t d = 0; d < D; ++d) o[d] = o[d] * inv * (double)gamma[d];
+        int32_t start = 0;
+        for (int32_t a = 0; a < 3; ++a) {
+            double pos = (double)coords[3 * i + a];
+            for (int32_t j = 0; j < w[a] / 2; ++j) {
+                double t = pos * pow(theta, -2.0 * (double)j / (double)w[a]);
+                double u = o[start + 2 * j], v = o[start + 2 * j + 1];
+                o[start + 2 * j] = u * cos(t) - v * sin(t);
+                o[start + 2 * j + 1] = u * sin(t) + v * cos(t);
+            }
+            start += w[a];
+        }
+    }
+    return 0;
+}

@@ -582,3 +582,105 @@ def test_backward_is_the_same_with_any_thread_count():
             subprocess.check_call([sys.executable, "-c", code, f], env=env)
             res.append(np.load(f))
     np.testing.assert_allclose(res[0], res[1], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# attention prologue: RMS normalisation of queries and keys, 3D rotary position embedding
+# ---------------------------------------------------------------------------------------------
+
+def test_prologue_rmsnorm_closed_forms():
+    # at the origin every rotation angle is 0, so only the normalisation acts: with eps = 0 and a
+    # unit weight the mean square over the head dimension is exactly 1; the result does not
+    # depend on the input's scale; a weight vector multiplies channel by channel
+    N, H, D = 40, 3, 32
+    x = _rand((N, H, D), 190)
+    zero = np.zeros((N, 3), np.int32)
+    ones = np.ones(D, np.float32)
+    u = oracle.qk_prologue(x, zero, ones, eps=0.0)
+    np.testing.assert_allclose((u ** 2).mean(axis=2), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(oracle.qk_prologue(3.7 * x, zero, ones, eps=0.0), u, rtol=1e-12)
+    gamma = np.random.default_rng(191).random(D).astype(np.float32) + 0.5
+    np.testing.assert_allclose(oracle.qk_prologue(x, zero, gamma, eps=0.0),
+                               u * gamma.astype(np.float64), rtol=1e-13)
+    # eps enters under the root: a constant row c gives c / sqrt(c^2 + eps)
+    c = np.full((1, 1, D), 0.01)
+    np.testing.assert_allclose(oracle.qk_prologue(c, zero[:1], ones, eps=1e-4),
+                               0.01 / np.sqrt(1e-4 + 1e-4), rtol=1e-13)
+
+
+@pytest.mark.parametrize("D", [32, 64, 96, 128])
+def test_prologue_rotation_angles(D):
+    # a unit vector on channel c (the first of a pair) normalises to sqrt(D) e_c; at position p
+    # along the part's axis the pair becomes sqrt(D) (cos t, sin t), t = p theta^(-2j / width),
+    # and the parts of the other two axes do not move
+    widths = oracle.rope_split(D)
+    assert sum(widths) == D and all(w % 2 == 0 for w in widths)
+    theta = 10000.0
+    starts = np.cumsum((0,) + widths[:2])
+    ones = np.ones(D, np.float32)
+    for a in range(3):
+        for j in (0, 1, widths[a] // 2 - 1):
+            c = starts[a] + 2 * j
+            x = np.zeros((1, 1, D))
+            x[0, 0, c] = 1.0
+            for p in (1, 5, 37):
+                pos = np.zeros((1, 3), np.int32)
+                pos[0, a] = p
+                u = oracle.qk_prologue(x, pos, ones, eps=0.0, theta=theta)[0, 0]
+                t = p * theta ** (-2.0 * j / widths[a])
+                exp = np.zeros(D)
+                exp[c], exp[c + 1] = np.sqrt(D) * np.cos(t), np.sqrt(D) * np.sin(t)
+                np.testing.assert_allclose(u, exp, atol=1e-12)
+
+
+def test_prologue_scores_depend_on_relative_position():
+    # rotations of both operands by their own positions: q.k depends only on the offset, so
+    # moving both tokens by the same vector keeps every score
+    D = 96
+    rng = np.random.default_rng(192)
+    q, k = rng.standard_normal((2, 1, 1, D))
+    gq, gk = (rng.random(D).astype(np.float32) + 0.5 for _ in range(2))
+    pq, pk = np.array([[3, 17, 40]], np.int32), np.array([[9, 2, 33]], np.int32)
+    shift = np.array([[11, 250, 7]], np.int32)
+    a = (oracle.qk_prologue(q, pq, gq) * oracle.qk_prologue(k, pk, gk)).sum()
+    b = (oracle.qk_prologue(q, pq + shift, gq) * oracle.qk_prologue(k, pk + shift, gk)).sum()
+    assert abs(a - b) <= 1e-10 * max(1.0, abs(a))
+    c = (oracle.qk_prologue(q, pq, gq) * oracle.qk_prologue(k, pq, gk)).sum()
+    assert abs(a - c) > 1e-3   # the offset itself does matter
+
+
+def test_forward_with_prologue_is_invariant_under_block_translation():
+    # the whole method with the prologue: moving every token by whole blocks keeps the blocks,
+    # the windows and (through the rotary embedding's relative form) every attention score. The
+    # compressed keys are block means of rotated keys times Wc, so a Wc that commutes with the
+    # rotations (a multiple of the identity) keeps the compressed scores relative as well.
+    c, q, k, v, _ = _tiny_inputs(seed=193)
+    g = _gates(len(c), 2, None, seed=15)
+    D = q.shape[2]
+    Wc = (0.7 * np.eye(D)).astype(np.float32)
+    rng = np.random.default_rng(194)
+    pro = dict(q_gamma=rng.random(D).astype(np.float32) + 0.5,
+               k_gamma=rng.random(D).astype(np.float32) + 0.5, eps=1e-6, theta=100.0)
+    a = run(c, q, k, v, g, Wc, 4, 2, prologue=pro)
+    b = run(c + np.array([8, 16, 24], np.int32), q, k, v, g, Wc, 4, 2, prologue=pro)
+    assert np.array_equal(a["sel"], b["sel"])
+    np.testing.assert_allclose(b["out"], a["out"], rtol=0, atol=1e-11)
+    # and the prologue changes the result (it is not silently skipped)
+    plain = run(c, q, k, v, g, Wc, 4, 2)
+    assert np.abs(plain["out"] - a["out"]).max() > 1e-2
+
+
+def test_prologue_normalises_and_scales_before_rotating():
+    # the rotation keeps the length of every channel pair, so each pair of the result has the
+    # length of the pair after normalisation and weighting (weighting after the rotation would
+    # not keep it, since the weights differ inside a pair)
+    N, H, D = 30, 2, 96
+    x = _rand((N, H, D), 195)
+    pos = np.random.default_rng(196).integers(0, 200, (N, 3)).astype(np.int32)
+    gamma = np.random.default_rng(197).random(D).astype(np.float32) * 2 + 0.1
+    u = oracle.qk_prologue(x, pos, gamma, eps=0.0)
+    rms = np.sqrt((x ** 2).mean(axis=2, keepdims=True))
+    y = x / rms * gamma.astype(np.float64)
+    pair = lambda a: np.sqrt(a[..., 0::2] ** 2 + a[..., 1::2] ** 2)
+    np.testing.assert_allclose(pair(u), pair(y), rtol=1e-12)
+    assert np.abs(u - y).max() > 1e-1   # and it does rotate

@@ -82,6 +82,8 @@ def lib():
             ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_i32p, c_f64p, c_i32p]
         L.oracle_rope_split.restype = None
         L.oracle_rope_split.argtypes = [ctypes.c_int32, c_i32p, c_i32p, c_i32p]
+        L.oracle_round_array.restype = None
+        L.oracle_round_array.argtypes = [c_f64p, ctypes.c_int64, ctypes.c_int32]
         L.oracle_qk_prologue.restype = ctypes.c_int
         L.oracle_qk_prologue.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                          ctypes.c_int32, c_vp, c_i32p, c_f32p, ctypes.c_double,
@@ -233,9 +235,11 @@ def rope_split(D: int):
     return a.value, b.value, c.value
 
 
-def qk_prologue(X, coords, gamma, eps: float = 1e-6, theta: float = 10000.0) -> np.ndarray:
+def qk_prologue(X, coords, gamma, eps: float = 1e-6, theta: float = 10000.0,
+                round_to_input: bool = False) -> np.ndarray:
     """RMS normalisation over the head dimension (weight gamma [D]) followed by the 3D rotary
-    embedding at the tokens' voxel coordinates; X [N, H, D] -> float64 [N, H, D]."""
+    embedding at the tokens' voxel coordinates; X [N, H, D] -> float64 [N, H, D]. With
+    round_to_input, the results are rounded to X's storage type (what the method then sees)."""
     x, dt = _raw(X)
     N, H, D = x.shape
     c = np.ascontiguousarray(coords, dtype=np.int32)
@@ -244,6 +248,8 @@ def qk_prologue(X, coords, gamma, eps: float = 1e-6, theta: float = 10000.0) -> 
     if lib().oracle_qk_prologue(N, H, D, dt, x.ctypes.data, _ptr(c, c_i32p), _ptr(g, c_f32p),
                                 float(eps), float(theta), _ptr(out, c_f64p)) != 0:
         raise ValueError("oracle_qk_prologue failed")
+    if round_to_input and dt != F64:
+        lib().oracle_round_array(_ptr(out, c_f64p), out.size, dt)
     return out
 
 
@@ -268,11 +274,12 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
     sel_in ([R, H, k] global block indices) replaces the selection of the rows. With
     branches=False only the compressed attention and the selection run: the result has o_cmp
     and sel, and out / o_sel / o_win are left at zero. prologue = dict(q_gamma, k_gamma, eps,
-    theta) first replaces Q and K by qk_prologue(Q), qk_prologue(K) (float64, unrounded).
+    theta) first replaces Q and K by qk_prologue(Q), qk_prologue(K), rounded to their input type
+    (the prologue's results are tensors of that type, as any layer's are).
     """
     if prologue is not None:
         pr = dict(prologue)
-        kw = dict(eps=pr.get("eps", 1e-6), theta=pr.get("theta", 10000.0))
+        kw = dict(eps=pr.get("eps", 1e-6), theta=pr.get("theta", 10000.0), round_to_input=True)
         Q = qk_prologue(Q, coords, pr["q_gamma"], **kw)
         K = qk_prologue(K, coords, pr["k_gamma"], **kw)
         V = _exact_f64(V)

@@ -831,6 +831,8 @@ int oracle_backward_dq_rows(int64_t n, int32_t H, int32_t D, int32_t dtype, cons
  *      is cut into an x part, a y part and a z part (oracle_rope_split), and channel pair
  *      (c, c+1) of the part for axis a, j-th pair of that part, is rotated by the angle
  *      coords[a] * theta^(-2j / width_a):  (u, v) -> (u cos t - v sin t, u sin t + v cos t).
+ * Like any layer of the model, the prologue hands its queries and keys on in the input type:
+ * the method runs on the results rounded to it (oracle_round_array, applied by the caller).
  */
 
 /* Widths of the x, y and z parts: y and z get 2*floor(D/6) channels each, x the rest. */
@@ -872,4 +874,10 @@ int oracle_qk_prologue(int64_t n, int32_t H, int32_t D, int32_t dtype, const voi
         }
     }
     return 0;
+}
+
+/* x[0..n) rounded in place to the storage type `dtype` (oracle_round_to, element by element). */
+void oracle_round_array(double* x, int64_t n, int32_t dtype) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) x[i] = oracle_round_to(x[i], dtype);
 }

@@ -684,3 +684,14 @@ def test_prologue_normalises_and_scales_before_rotating():
     pair = lambda a: np.sqrt(a[..., 0::2] ** 2 + a[..., 1::2] ** 2)
     np.testing.assert_allclose(pair(u), pair(y), rtol=1e-12)
     assert np.abs(u - y).max() > 1e-1   # and it does rotate
+
+
+def test_prologue_results_rounded_to_the_input_type():
+    # rounding the prologue's fp64 results to f16 equals numpy's f16 conversion of them
+    N, H, D = 50, 2, 64
+    x = _rand((N, H, D), 198).astype(np.float16)
+    pos = np.random.default_rng(199).integers(0, 100, (N, 3)).astype(np.int32)
+    g = np.random.default_rng(200).random(D).astype(np.float32) + 0.5
+    exact = oracle.qk_prologue(x, pos, g)
+    rounded = oracle.qk_prologue(x, pos, g, round_to_input=True)
+    np.testing.assert_array_equal(rounded, exact.astype(np.float16).astype(np.float64))

@@ -383,8 +383,9 @@ def cpu_baseline(cfg_name, target_s=20.0):
     t = workloads.make_tensors(cfg, len(coords))
     N = len(coords)
     oracle.lib()
-    fixed, per_row, _ = oracle_cost_model(cfg, coords, cu, t, 64, seed=4242)
-    n_rows = int(min(N, max(64, (target_s - fixed) / max(per_row, 1e-9))))
+    fixed, per_row, _ = oracle_cost_model(cfg, coords, cu, t, 256, seed=4242)
+    # second, larger sample sized to the time budget (bounded, whatever the first estimate says)
+    n_rows = int(min(N, 4096, max(256, (target_s - fixed) / max(per_row, 1e-6))))
     fixed, per_row, tn = oracle_cost_model(cfg, coords, cu, t, n_rows, seed=4243)
     step_s = fixed + per_row * N
     return {"value": N / step_s, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",

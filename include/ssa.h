@@ -180,6 +180,30 @@ SSA_API ssa_status_t ssa_forward_debug(ssa_plan_t plan, const void* q, const voi
                                void* stream);
 
 /*
+ * Forward pass with the attention prologue of the transformer that runs SSA (Hi3D v1.0 pipeline
+ * page, "Stage 3: sparse flow sampling": rotary position embeddings and RMS normalisation of the
+ * self-attention queries and keys). Before the method, q and k are each replaced, per token and
+ * head, by
+ *   u = x / sqrt(mean_d x_d^2 + eps) * gamma     (RMS normalisation over the head dimension)
+ * followed by a 3D rotary embedding at the token's voxel coordinates (x, y, z) from the plan: the
+ * head dimension is cut into an x part of D - 2c channels and y and z parts of c = 2*floor(D/6)
+ * channels each; channel pair (2p, 2p+1), the j-th pair of a part of width w along axis a, turns
+ * by the angle coords[a] * rope_theta^(-2j/w). V is not transformed.
+ *   q_gamma, k_gamma: device fp32 [D] weights of the normalisation (shared by all heads).
+ *   rope_theta: base of the rotary frequencies (> 1), e.g. 10000. eps: >= 0.
+ *   sel_out: optional device int32 [N, H, k], as in ssa_forward_debug (NULL = not written).
+ * Everything else as ssa_forward. bf16 / fp16: the transform runs inside the pooling kernel (keys)
+ * and on each query tile after its load (queries), with fp32 arithmetic and the transformed
+ * values rounded to the input type; fp32: a separate pass into workspace copies of q and k.
+ * Errors: as ssa_forward, and SSA_ERR_INVALID_ARG for a NULL weight, rope_theta <= 1 or eps < 0.
+ */
+SSA_API ssa_status_t ssa_forward_prologue(ssa_plan_t plan, const void* q, const void* k, const void* v,
+                                  const float* gates, const float* wc, const float* q_gamma,
+                                  const float* k_gamma, float rope_theta, float eps, int32_t heads,
+                                  int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
+                                  int32_t* sel_out, void* stream);
+
+/*
  * ssa_forward on HOST buffers: copies q, k, v, gates, wc (host) to plan-owned device buffers,
  * runs the forward and copies the result into out (host). Pinned host memory gives overlapped,
  * full-speed copies; pageable memory works but is slower. Waits for the device before returning.

@@ -48,6 +48,8 @@ _SIGS = {
     "ssa_forward_debug": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                           _vp, _vp],
     "ssa_forward_host": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp],
+    "ssa_forward_prologue": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float,
+                             _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "ssa_backward": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "ssa_last_device_status": [_vp, _vp],
     "ssa_plan_destroy": [_vp],
@@ -260,6 +262,25 @@ class Plan:
                                wc.data_ptr(), H, D, _DTYPE[dt], topk, out.data_ptr(), st),
                "ssa_forward")
         return out
+
+    def forward_prologue(self, q, k, v, gates, wc, topk: int, q_gamma, k_gamma,
+                         rope_theta: float = 10000.0, eps: float = 1e-6,
+                         out: Optional[torch.Tensor] = None, return_sel: bool = False):
+        """ssa_forward_prologue: RMS-normalised, rotary-embedded q and k, then the method.
+        q_gamma, k_gamma: fp32 CUDA tensors [D]."""
+        dt, H, D = self._args(q, k, v, gates, wc)
+        for gm in (q_gamma, k_gamma):
+            _dev(gm, torch.float32)
+            if gm.numel() != D:
+                raise ValueError("q_gamma and k_gamma must hold D values")
+        out = torch.empty_like(q) if out is None else _dev(out, dt)
+        sel = torch.empty(self.N, H, topk, dtype=torch.int32, device=q.device) if return_sel else None
+        _check(lib.ssa_forward_prologue(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                        gates.data_ptr(), wc.data_ptr(), q_gamma.data_ptr(),
+                                        k_gamma.data_ptr(), float(rope_theta), float(eps), H, D,
+                                        _DTYPE[dt], topk, out.data_ptr(), _ptr(sel),
+                                        _stream(self.stream)), "ssa_forward_prologue")
+        return (out, sel) if return_sel else out
 
     def forward_host(self, q, k, v, gates, wc, topk: int, out: torch.Tensor):
         """Forward on host (preferably pinned) CPU tensors; copies run inside the library."""

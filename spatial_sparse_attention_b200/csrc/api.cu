@@ -292,13 +292,31 @@ ssa_status_t check_forward_args(Plan* p, const void* q, const void* k, const voi
 ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, const float* gates,
                          const float* wc, int32_t H, int32_t D, ssa_dtype_t dt, int32_t topk,
                          void* out, int32_t* sel_out, cudaStream_t st,
-                         const BranchOut& bo = BranchOut()) {
+                         const BranchOut& bo = BranchOut(), const Prologue& pro = Prologue()) {
     ssa_status_t rc = ensure_workspace(p, H, D, dt, topk, st);
     if (rc != SSA_OK) return rc;
-    const Workspace& w = p->ws;
+    Workspace& w = p->ws;
+    if (pro.on() && dt == SSA_F32) {
+        // fp32 path: the prologue is a pass of its own into workspace copies of q and k
+        const size_t bytes = sizeof(float) * (size_t)p->N * H * D;
+        for (float** buf : {&w.qp, &w.kp}) {
+            if (*buf) continue;
+            *buf = (float*)p->alloc(bytes, st, p->alloc_ctx);
+            if (!*buf) return SSA_ERR_ALLOC;
+            w.owned.push_back(*buf);
+        }
+        {
+            ProfScope ps("prologue", st);
+            launch_qk_prologue_f32(p, (const float*)q, pro.q_gamma, pro, H, D, w.qp, st);
+            launch_qk_prologue_f32(p, (const float*)k, pro.k_gamma, pro, H, D, w.kp, st);
+        }
+        q = w.qp;
+        k = w.kp;
+    }
+    const Prologue fused = dt == SSA_F32 ? Prologue() : pro;   // 16-bit: inside pool and forward
     {
         ProfScope ps("pool", st);
-        launch_pool(p, w, k, v, wc, st);
+        launch_pool(p, w, k, v, wc, fused, st);
     }
     trace_step("pool", st);
     if (dt == SSA_F32) {
@@ -306,7 +324,11 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
         if ((rc = ensure_neighbours(p, st)) != SSA_OK) return rc;
         launch_forward_simt(p, w, q, k, v, gates, out, bo, st);
     }
-    else if ((rc = launch_forward_tc(p, w, q, gates, out, bo, st)) != SSA_OK) return rc;
+    else {
+        if ((rc = launch_select_tc(p, w, q, fused, st)) != SSA_OK) return rc;
+        trace_step("select", st);
+        if ((rc = launch_forward_tc(p, w, q, gates, out, bo, fused, st)) != SSA_OK) return rc;
+    }
     trace_step("forward", st);
     if (sel_out) launch_export_sel(p, w, sel_out, st);
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
@@ -444,6 +466,23 @@ ssa_status_t ssa_forward_debug(ssa_plan_t p, const void* q, const void* k, const
     bo.o[2] = o_win;
     return run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, sel_out,
                        (cudaStream_t)stream, bo);
+}
+
+ssa_status_t ssa_forward_prologue(ssa_plan_t p, const void* q, const void* k, const void* v,
+                                  const float* gates, const float* wc, const float* q_gamma,
+                                  const float* k_gamma, float rope_theta, float eps, int32_t heads,
+                                  int32_t head_dim, ssa_dtype_t dtype, int32_t topk, void* out,
+                                  int32_t* sel_out, void* stream) {
+    ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out);
+    if (rc != SSA_OK) return rc;
+    if (!q_gamma || !k_gamma || !(rope_theta > 1.0f) || !(eps >= 0.0f)) return SSA_ERR_INVALID_ARG;
+    Prologue pro;
+    pro.q_gamma = q_gamma;
+    pro.k_gamma = k_gamma;
+    pro.theta = rope_theta;
+    pro.eps = eps;
+    return run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, sel_out,
+                       (cudaStream_t)stream, BranchOut(), pro);
 }
 
 ssa_status_t ssa_forward_host(ssa_plan_t p, const void* q, const void* k, const void* v,

@@ -1,10 +1,10 @@
-// Device pieces of the tensor-core forward: the parameter block, 16-bit packing and the register
-// top-k list.
+// Device pieces of the tensor-core forward: the parameter block and 16-bit packing.
 #pragma once
 
 #include <type_traits>
 
 #include "common.cuh"
+#include "prologue.cuh"
 #include "tc.cuh"
 
 namespace ssa {
@@ -40,6 +40,11 @@ struct FwdParams {
     float* base;
     void* out;
     float* bout[3];   // optional per-branch outputs (fp32, token order), null when not wanted
+    // attention prologue on the query tiles (null q_gamma = off)
+    const float* q_gamma;
+    const int32_t* coords;
+    double theta;
+    float eps;
     int32_t* status;
     int64_t N, Nks, Mb, Mb8;
     int H, k, r;
@@ -68,26 +73,48 @@ __device__ __forceinline__ float unpack_hi(uint32_t v) {
     else return __uint_as_float(v & 0xffff0000u);
 }
 
+// Attention prologue on a query tile held in shared memory in the chunked, 64-byte-swizzled
+// operand order (32-column chunks `qreg` bytes apart): row `row` (token `tok`) is RMS-normalised
+// over the head dimension and turned by the 3D rotary embedding, in place, in fp32, and rounded
+// back to T. freq / axis: the rotary table of the D/2 channel pairs; gamma: [D] weights.
+template <typename T, int D>
+__device__ __forceinline__ void qtile_prologue(uint8_t* qtile, uint32_t qreg, int row, int32_t tok,
+                                               const int32_t* coords, const double* freq,
+                                               const int* axis, const float* gamma, float eps) {
+    const int32_t cx = coords[3 * tok], cy = coords[3 * tok + 1], cz = coords[3 * tok + 2];
+    float ss = 0.0f;
+#pragma unroll 1
+    for (int c16 = 0; c16 < D / 8; ++c16) {
+        const uint4 u = *reinterpret_cast<const uint4*>(qtile + (c16 >> 2) * qreg + tc::sw64(row, c16 & 3));
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float a = unpack_lo<T>(w[q]), b = unpack_hi<T>(w[q]);
+            ss = fmaf(a, a, fmaf(b, b, ss));
+        }
+    }
+    const float inv = rsqrtf(ss / (float)D + eps);
+#pragma unroll 1
+    for (int c16 = 0; c16 < D / 8; ++c16) {
+        uint4* up = reinterpret_cast<uint4*>(qtile + (c16 >> 2) * qreg + tc::sw64(row, c16 & 3));
+        uint4 u = *up;
+        uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int pr = c16 * 4 + q;
+            float c, sn;
+            rope_cos_sin(axis_coord(axis[pr], cx, cy, cz), freq[pr], c, sn);
+            const float a = unpack_lo<T>(w[q]) * inv * gamma[2 * pr];
+            const float b = unpack_hi<T>(w[q]) * inv * gamma[2 * pr + 1];
+            w[q] = pack2<T>(a * c - b * sn, a * sn + b * c);
+        }
+        *up = u;
+    }
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     uint32_t s = tc::smem_u32(p);
     return p + ((1024u - (s & 1023u)) & 1023u);
-}
-
-// Sorted top list (logit descending; among equal logits, lower block index first). Blocks are
-// offered in ascending index order, so a new entry goes after every entry whose logit is >= its
-// own. All positions are updated from the old list at once (no serial chain).
-template <int KM>
-__device__ __forceinline__ void topk_push(float (&tv)[KM], int32_t (&ti)[KM], float z, int32_t b) {
-    bool c[KM];
-#pragma unroll
-    for (int t = 0; t < KM; ++t) c[t] = z > tv[t];
-#pragma unroll
-    for (int t = KM - 1; t > 0; --t) {
-        tv[t] = c[t] ? (c[t - 1] ? tv[t - 1] : z) : tv[t];
-        ti[t] = c[t] ? (c[t - 1] ? ti[t - 1] : b) : ti[t];
-    }
-    tv[0] = c[0] ? z : tv[0];
-    ti[0] = c[0] ? b : ti[0];
 }
 
 }  // namespace attn

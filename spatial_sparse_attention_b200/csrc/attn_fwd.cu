@@ -5,8 +5,8 @@
 //
 // One CTA per (query tile of 128 tokens in block order, head). The CTA streams 64-key tiles
 // through three phases, each one softmax per row:
-//   C  the compressed tokens of the sequence (block mean . Wc). Each row keeps a running list of
-//      its top-(k-1) other blocks by compressed logit; the own block is slot 0.
+//   C  the compressed tokens of the sequence (block mean . Wc). The rows' selected blocks (own
+//      block plus the top-(k-1) others by compressed logit) come from the selection kernel.
 //   S  the selected tokens: the union over the tile's rows of their k selected blocks, each row
 //      masked to its own k blocks (a row's valid keys are k ranges of the union stream). Blocks
 //      of at most 7 tokens come from their sequence's packed pool instead when the tile selects
@@ -177,12 +177,32 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
     // masked keys (weight 0) never meet a non-finite V entry
     for (uint32_t o = tid * 16u; o < 4u * L::kTile; o += kThreads * 16u)
         *reinterpret_cast<uint4*>(g + L::kK + o) = make_uint4(0u, 0u, 0u, 0u);
+    // attention prologue: the rotary table (frequency and axis of each channel pair) and the
+    // query weights, in the union area (unused until phase C)
+    double* pro_freq = reinterpret_cast<double*>(g + L::kUnion);
+    int* pro_axis = reinterpret_cast<int*>(g + L::kUnion + 64 * 8);
+    float* pro_gamma = reinterpret_cast<float*>(g + L::kUnion + 64 * 12);
+    if (P.q_gamma) {
+        if (tid < D / 2) rope_pair(D, tid, P.theta, pro_axis[tid], pro_freq[tid]);
+        if (tid < D) pro_gamma[tid] = P.q_gamma[tid];
+    }
     tc::cp_async_wait_all();
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = (uint32_t)misc[M_TMEM];
+    if (P.q_gamma) {
+        // the query tile in place: RMS normalisation over the head dimension, then the 3D rotary
+        // embedding at the token's coordinates; each softmax thread takes its own row
+        if (tid >= 64 && tid - 64 < len)
+            qtile_prologue<T, D>(g + L::kQ, L::kQReg, tid - 64, P.perm[p0 + tid - 64], P.coords, pro_freq,
+                                 pro_axis, pro_gamma, P.eps);
+        tc::fence_proxy_async();   // generic-proxy writes of the tile, read next by the tensor cores
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    }
 
     if (warp == 0) {
         // ================================ producer ============================================
@@ -296,6 +316,13 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             for (int kk = 0; kk < kKT / 16; ++kk)
                 tc::mma_f16_ts(tmem + 128, tmem + b * kKT + kk * 8, tc::desc_mnmajor_g(vbase, kk, L::kCh),
                                idesc_o, (first && kk == 0) ? 0u : 1u);
+            if (kBf16) {
+                // bf16: P = P_hi + P_lo, the low part in the buffer's upper 32 columns
+#pragma unroll
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    tc::mma_f16_ts(tmem + 128, tmem + b * kKT + 32 + kk * 8,
+                                   tc::desc_mnmajor_g(vbase, kk, L::kCh), idesc_o, 1u);
+            }
             tc::mma_commit(&bar[PVD + b]);   // P V of tile i done: V stage, P buffer, O
             return true;
         };
@@ -352,13 +379,6 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             }
             return true;
         };
-        float tv[KM];
-        int32_t ti[KM];
-#pragma unroll
-        for (int u = 0; u < KM; ++u) {
-            tv[u] = -INFINITY;
-            ti[u] = -1;
-        }
         int ns = 0, nT = 1 << 30, ri = 0, nr = 0;
         int2 rcur = make_int2(0x7fffffff, 0x7fffffff);
         const uint64_t* wrow = P.wmask + (int64_t)wm0 * 128 + row;
@@ -420,13 +440,11 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             }
             if (j == nc) {
                 // ---- selection, union of the selected blocks, this row's key ranges ----------
-                if (ok && row_ok) {
-                    int32_t* srow = P.sel + ((int64_t)pos * H + h) * ksel;
-                    srow[0] = ob;
+                // this row's selection, written by the selection kernel (global block indices)
+                int32_t ti[KM];
+                const int32_t* srow = P.sel + ((int64_t)pos * H + h) * ksel;
 #pragma unroll
-                    for (int u = 0; u < KM; ++u)
-                        if (u + 1 < ksel) srow[u + 1] = ti[u];
-                }
+                for (int u = 0; u < KM; ++u) ti[u] = u + 1 < ksel ? srow[u + 1] : -1;
                 uint32_t* words = reinterpret_cast<uint32_t*>(g + L::kK);
                 const int W = (nblk + 31) >> 5;
                 int32_t* wpre = reinterpret_cast<int32_t*>(words + W);
@@ -604,29 +622,6 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             }
             const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            if (ph == 0 && ksel > 1 && tmax > tv[KM - 1]) {
-                // running top-(k-1) of the other blocks: candidates above the list's last entry,
-                // offered in ascending block order; the row's scores go to shared memory
-                // (quad q of row r at float4 index q * 128 + r) so a candidate is one load
-                const int32_t bbase = 8 * cg0 + kKT * j;
-                float4* srow4 = reinterpret_cast<float4*>(g + L::kUnion) + row;
-                const float* srow1 = reinterpret_cast<const float*>(srow4);
-                uint64_t cand = 0ull;
-                const float thr = tv[KM - 1];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    srow4[q * 128] = make_float4(s[4 * q], s[4 * q + 1], s[4 * q + 2], s[4 * q + 3]);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) cand |= (uint64_t)(s[4 * q + i] > thr) << (4 * q + i);
-                }
-                while (cand) {
-                    const int e = __ffsll((long long)cand) - 1;
-                    cand &= cand - 1;
-                    const int32_t bi = bbase + e;
-                    const float z = srow1[(e >> 2) * 512 + (e & 3)];
-                    if (bi != ob && z > tv[KM - 1]) topk_push<KM>(tv, ti, z, bi);
-                }
-            }
             // ---- running max, lazy rescale, P = 2^(s*sl - m) ------------------------------------
             const float tm = tmax * sl;
             bool resc = false;
@@ -658,15 +653,21 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float a0 = tc::ex2(fmaf(s[2 * i], sl, -mu));
-                const float a1 = tc::ex2(fmaf(s[2 * i + 1], sl, -mu));
-                pk[i] = pack2<T>(a0, a1);
-                // bf16 weights: the row sum uses the rounded weights the MMA multiplies V with
-                if (kBf16) ls[i & 3] += unpack_lo<T>(pk[i]) + unpack_hi<T>(pk[i]);
-                else ls[i & 3] += a0 + a1;
+                s[2 * i] = tc::ex2(fmaf(s[2 * i], sl, -mu));
+                s[2 * i + 1] = tc::ex2(fmaf(s[2 * i + 1], sl, -mu));
+                pk[i] = pack2<T>(s[2 * i], s[2 * i + 1]);
+                ls[i & 3] += s[2 * i] + s[2 * i + 1];
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             tc::tmem_st32(s_tm, pk);
+            if (kBf16) {
+                // bf16 keeps 8 significant bits: the weights go to the tensor cores as P_hi + P_lo
+                // (both bf16, the low part in the upper 32 columns), so P V carries ~16 bits of P
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    pk[i] = pack2<T>(s[2 * i] - unpack_lo<T>(pk[i]), s[2 * i + 1] - unpack_hi<T>(pk[i]));
+                tc::tmem_st32(s_tm + 32, pk);
+            }
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bar[PFULL + b]);
@@ -711,9 +712,10 @@ ssa_status_t run(const Plan* p, const FwdParams& P, int64_t max_seq_blocks, cuda
 
 template <typename T, int D>
 ssa_status_t run_km(const Plan* p, const FwdParams& P, int64_t mb, cudaStream_t st) {
-    if (P.k - 1 <= 8) return run<T, D, 8>(p, P, mb, st);
-    if (P.k - 1 <= 16) return run<T, D, 16>(p, P, mb, st);
-    return run<T, D, 32>(p, P, mb, st);
+    // KM: the other selected blocks per row, k - 1 rounded up to 7, 15 or 31 (k <= 32)
+    if (P.k <= 8) return run<T, D, 7>(p, P, mb, st);
+    if (P.k <= 16) return run<T, D, 15>(p, P, mb, st);
+    return run<T, D, 31>(p, P, mb, st);
 }
 
 template <typename T>
@@ -729,7 +731,7 @@ ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, int64_t mb, cudaStr
 }  // namespace
 
 ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
-                               void* out, const BranchOut& bo, cudaStream_t st) {
+                               void* out, const BranchOut& bo, const Prologue& pro, cudaStream_t st) {
     const bool bf16 = w.dtype == SSA_BF16;
     int64_t max_seq_blocks = 0;
     for (size_t s = 0; s + 1 < p->seq_blk.size(); ++s)
@@ -762,6 +764,10 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
     P.base = w.base;
     P.out = out;
     for (int b = 0; b < 3; ++b) P.bout[b] = bo.o[b];
+    P.q_gamma = pro.on() ? pro.q_gamma : nullptr;
+    P.coords = p->coords;
+    P.theta = pro.theta;
+    P.eps = pro.eps;
     P.status = p->d_status;
     P.N = p->N;
     P.Nks = p->Nks;

@@ -39,6 +39,17 @@ struct SeqInfo {
     int32_t gbx, gby, gbz;   // blocks per axis (ceil(g / 8))
 };
 
+// Attention prologue of a forward call: RMS normalisation of q and k over the head dimension
+// (weights q_gamma, k_gamma: device fp32 [D]) and the 3D rotary embedding with base theta at the
+// voxel coordinates (prologue.cuh). Off when q_gamma is null.
+struct Prologue {
+    const float* q_gamma = nullptr;
+    const float* k_gamma = nullptr;
+    double theta = 10000.0;
+    float eps = 1e-6f;
+    bool on() const { return q_gamma != nullptr; }
+};
+
 // Forward workspace, cached in the plan for one (H, D, dtype, k).
 struct Workspace {
     int32_t H = 0, D = 0, k = 0;
@@ -55,6 +66,9 @@ struct Workspace {
     int64_t Mb8 = 0;           // Mb rounded up to a multiple of 8
     float* base = nullptr;     // [query tiles, H, D/4, 128, 4] running g0*o_cmp + g1*o_sel
     int32_t* sel = nullptr;    // [N, H, k]        selected blocks, sorted token order
+    // fp32 path with the prologue: transformed q and k (allocated on first use)
+    float* qp = nullptr;       // [N, H, D]
+    float* kp = nullptr;       // [N, H, D]
     // host-buffer entry point staging (allocated on first use)
     void* h_q = nullptr; void* h_k = nullptr; void* h_v = nullptr; void* h_out = nullptr;
     float* h_gates = nullptr; float* h_wc = nullptr;
@@ -165,9 +179,13 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t s);
 ssa_status_t ensure_neighbour_counts(Plan* p, cudaStream_t s);
 ssa_status_t ensure_neighbours(Plan* p, cudaStream_t s);
 
-// pool.cu
+// pool.cu (with the prologue applied to k on the way when pro.on(), 16-bit types)
 void launch_pool(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,
-                 cudaStream_t s);
+                 const Prologue& pro, cudaStream_t s);
+
+// prologue.cu: out = prologue(x) for fp32 [N, H, D] rows (the fp32 path's stand-alone pass)
+void launch_qk_prologue_f32(const Plan* p, const float* x, const float* gamma, const Prologue& pro,
+                            int H, int D, float* out, cudaStream_t s);
 
 // Per-branch outputs of the forward, fp32 [N, H, D] in token order each: o_cmp, o_sel, o_win
 // (normalised branch attention outputs before the gates). Any entry may be null.
@@ -180,9 +198,15 @@ void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const
                          const void* v, const float* gates, void* out, const BranchOut& bo,
                          cudaStream_t s);
 
-// attn_fwd.cu (bf16 / fp16 path): the fused tensor-core forward
+// select.cu (bf16 / fp16 path): the selected blocks of every (token, head) into w.sel, sorted
+// token order (the prologue, when on, is applied to each query tile after it is loaded)
+ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
+                              cudaStream_t s);
+
+// attn_fwd.cu (bf16 / fp16 path): the fused tensor-core forward over w.sel (the prologue, when on, is
+// applied to each query tile after it is loaded)
 ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q, const float* gates,
-                               void* out, const BranchOut& bo, cudaStream_t s);
+                               void* out, const BranchOut& bo, const Prologue& pro, cudaStream_t s);
 
 // backward.cu
 ssa_status_t launch_backward(Plan* p, const Workspace& w, const void* q, const void* k,

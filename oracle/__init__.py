@@ -80,6 +80,16 @@ def lib():
             ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
             c_f32p, c_f32p, c_vp, ctypes.c_int32, ctypes.c_int32, c_i32p, c_i32p, c_i32p,
             ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_i32p, c_f64p, c_i32p]
+        L.oracle_forward_variant.restype = ctypes.c_int
+        L.oracle_forward_variant.argtypes = [
+            ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
+            c_f32p, c_f32p, c_i32p, c_f32p, c_f32p, ctypes.c_int32, c_i32p, c_i32p, c_i32p,
+            ctypes.c_int64, c_i64p, c_i32p, ctypes.c_int64, c_i64p, c_i32p,
+            c_f64p, c_f64p, c_f64p, c_f64p, c_i32p, c_f64p]
+        L.oracle_compress_conv.restype = ctypes.c_int
+        L.oracle_compress_conv.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, c_vp, c_vp, c_f32p, c_i32p, c_i32p,
+                                           c_i32p, c_f64p, c_f64p]
         L.oracle_rope_split.restype = None
         L.oracle_rope_split.argtypes = [ctypes.c_int32, c_i32p, c_i32p, c_i32p]
         L.oracle_round_array.restype = None
@@ -264,9 +274,20 @@ def _exact_f64(t) -> np.ndarray:
     return np.asarray(t, dtype=np.float64)
 
 
+def center_only_conv(Wc) -> np.ndarray:
+    """The convolution kernel [27, D, D] whose only nonzero tap is the centre one, Wc: the
+    convolution compression then equals the block mean times Wc."""
+    w = _f32(Wc)
+    D = w.shape[0]
+    W = np.zeros((27, D, D), np.float32)
+    W[13] = w
+    return W
+
+
 def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None,
             block: int = 8, round_compressed: bool = False, sel_in=None,
-            want_z: bool = False, branches: bool = True, prologue=None) -> Dict[str, object]:
+            want_z: bool = False, branches: bool = True, prologue=None, conv=None,
+            gate=None) -> Dict[str, object]:
     """Oracle forward for the query rows `rows` (global indices; None = all tokens).
 
     Returns out, o_cmp, o_sel, o_win ([R, H, D] float64), sel ([R, H, k] int32 global block
@@ -275,7 +296,10 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
     branches=False only the compressed attention and the selection run: the result has o_cmp
     and sel, and out / o_sel / o_win are left at zero. prologue = dict(q_gamma, k_gamma, eps,
     theta) first replaces Q and K by qk_prologue(Q), qk_prologue(K), rounded to their input type
-    (the prologue's results are tensors of that type, as any layer's are).
+    (the prologue's results are tensors of that type, as any layer's are). conv ([27, D, D]
+    fp32) compresses blocks by the sparse 3D convolution over the block grid instead of the
+    block mean times Wc; gate = dict(w=[D, 3], b=[3]) predicts the gates from each head's query
+    (sigmoid(q . w + b)) instead of reading `gates`.
     """
     if prologue is not None:
         pr = dict(prologue)
@@ -285,7 +309,7 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
         V = _exact_f64(V)
         return forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk, r, rows=rows, block=block,
                        round_compressed=round_compressed, sel_in=sel_in, want_z=want_z,
-                       branches=branches)
+                       branches=branches, conv=conv, gate=gate)
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     q, dt = _raw(Q)
@@ -294,6 +318,13 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
     g = _f32(gates)
     w = _f32(Wc)
     N, H, D = q.shape
+    wconv = wg = bg = None
+    if conv is not None or gate is not None:
+        wconv = np.ascontiguousarray(_f32(conv) if conv is not None else center_only_conv(w),
+                                     dtype=np.float32).reshape(27, D, D)
+        if gate is not None:
+            wg = np.ascontiguousarray(_f32(gate["w"]), dtype=np.float32).reshape(D, 3)
+            bg = np.ascontiguousarray(_f32(gate["b"]), dtype=np.float32).reshape(3)
     rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     R = len(rows)
     res = {name: np.zeros((R, H, D)) for name in ("out", "o_cmp", "o_sel", "o_win")}
@@ -316,6 +347,31 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
             if sel_in is not None:
                 sin = np.ascontiguousarray(np.asarray(sel_in, dtype=np.int64)[pick], dtype=np.int64)
                 sin = np.where(sin >= 0, sin - blk_base, -1).astype(np.int32)
+            outs_args = (
+                n_r, _ptr(local, c_i64p), _ptr(sin, c_i32p),
+                _ptr(outs["out"] if branches else None, c_f64p), _ptr(outs["o_cmp"], c_f64p),
+                _ptr(outs["o_sel"] if branches else None, c_f64p),
+                _ptr(outs["o_win"] if branches else None, c_f64p),
+                _ptr(sel, c_i32p), _ptr(zc, c_f64p))
+            if conv is not None or gate is not None:
+                bc = np.ascontiguousarray(partition(coords[lo:hi], block)[3], dtype=np.int32)
+                rc = L.oracle_forward_variant(
+                    hi - lo, H, D, dt,
+                    q[lo:hi].ctypes.data, k[lo:hi].ctypes.data, v[lo:hi].ctypes.data,
+                    _ptr(np.ascontiguousarray(g[lo:hi]), c_f32p), _ptr(wconv, c_f32p),
+                    _ptr(bc, c_i32p), _ptr(wg, c_f32p), _ptr(bg, c_f32p), topk,
+                    _ptr(perm, c_i32p), _ptr(tok_blk, c_i32p), _ptr(blk_off, c_i32p), mb,
+                    _ptr(no, c_i64p), _ptr(ni, c_i32p), *outs_args)
+                if rc != 0:
+                    raise RuntimeError("oracle_forward_variant failed")
+                for name in outs:
+                    res[name][pick] = outs[name]
+                res["sel"][pick] = np.where(sel >= 0, sel + blk_base, -1)
+                if want_z:
+                    for t_, p_ in enumerate(pick):
+                        zs[p_] = zc[t_, :, :mb].copy()
+                blk_base += mb
+                continue
             rc = L.oracle_forward(
                 hi - lo, H, D, dt,
                 q[lo:hi].ctypes.data, k[lo:hi].ctypes.data, v[lo:hi].ctypes.data,
@@ -439,6 +495,24 @@ def backward_dq_rows(coords, cu_seqlens, Q, K, V, gates, Wc, dO, topk: int, r: i
         sel_all[pick] = np.where(sel >= 0, sel + blk_base, -1)
         blk_base += mb
     return (dQ, sel_all) if return_sel else dQ
+
+
+def compress_conv(coords, K, V, W, block: int = 8):
+    """Compressed tokens (Kc, Vc) [Mb, H, D] of a single sequence by the sparse 3D convolution
+    over the block grid (W [27, D, D])."""
+    k, dt = _raw(K)
+    v, _ = _raw(V)
+    N, H, D = k.shape
+    Wf = np.ascontiguousarray(_f32(W), dtype=np.float32).reshape(27, D, D)
+    perm, tok_blk, blk_off, blk_coord = partition(coords, block)
+    mb = len(blk_coord)
+    Kc = np.zeros((mb, H, D))
+    Vc = np.zeros((mb, H, D))
+    bc = np.ascontiguousarray(blk_coord, dtype=np.int32)
+    lib().oracle_compress_conv(mb, H, D, dt, k.ctypes.data, v.ctypes.data, _ptr(Wf, c_f32p),
+                               _ptr(perm, c_i32p), _ptr(blk_off, c_i32p), _ptr(bc, c_i32p),
+                               _ptr(Kc, c_f64p), _ptr(Vc, c_f64p))
+    return Kc, Vc
 
 
 def compress(coords, K, V, Wc, block: int = 8, round_compressed: bool = False):

@@ -317,6 +317,97 @@ int oracle_compress(int64_t mb, int32_t H, int32_t D, int32_t dtype, const void*
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* 2b. compression by a sparse 3D convolution over the block grid                              */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * Direct3D-S2 summary page, "Technical principles of Direct3D-S2", SSA item: the compression
+ * module turns each block into a block-level token by sparse 3D convolution and pooling. The
+ * page gives no shapes; the plain reading taken here: pool first (the mean over the tokens
+ * present in the block, as in step 2), then one sparse 3D convolution over the grid of occupied
+ * blocks with a 3x3x3 kernel, stride 1, outputs at the occupied blocks only, an absent
+ * neighbour contributing nothing:
+ *   Kc_b = sum over offsets o in {-1,0,1}^3 with block b+o occupied of mean(K_{b+o}) . W_o
+ * W_o (D x D, row vector times W_o) is shared by K, V and all heads; offset (dx, dy, dz) is
+ * W[9*(dx+1) + 3*(dy+1) + (dz+1)]. With W_o = 0 except W_0 = Wc this is step 2.
+ */
+
+/* Index of the block of one sequence with block coordinates (x, y, z), or -1 (blk_coord holds
+ * the occupied blocks in lexicographic order). */
+static int64_t find_block(const int32_t* blk_coord, int64_t mb, int32_t x, int32_t y, int32_t z) {
+    int64_t lo = 0, hi = mb;
+    while (lo < hi) {
+        int64_t mid = lo + (hi - lo) / 2;
+        const int32_t* c = &blk_coord[3 * mid];
+        int less = c[0] < x || (c[0] == x && (c[1] < y || (c[1] == y && c[2] < z)));
+        if (less) lo = mid + 1; else hi = mid;
+    }
+    if (lo < mb && blk_coord[3 * lo] == x && blk_coord[3 * lo + 1] == y && blk_coord[3 * lo + 2] == z)
+        return lo;
+    return -1;
+}
+
+static void compress_conv(int64_t mb, int32_t H, int32_t D, int dtype, const void* K, const void* V,
+                          const float* W, const int32_t* perm, const int32_t* blk_off,
+                          const int32_t* blk_coord, double* Kc, double* Vc) {
+    double* km = (double*)calloc((size_t)(mb * H * D + 1), sizeof(double));
+    double* vm = (double*)calloc((size_t)(mb * H * D + 1), sizeof(double));
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t bh = 0; bh < mb * H; ++bh) {
+        int64_t b = bh / H;
+        int32_t h = (int32_t)(bh % H);
+        int64_t nb = blk_off[b + 1] - blk_off[b];
+        for (int64_t p = blk_off[b]; p < blk_off[b + 1]; ++p) {
+            int64_t j = perm[p];
+            for (int32_t d = 0; d < D; ++d) {
+                km[bh * D + d] += load_elem(K, dtype, (j * H + h) * D + d);
+                vm[bh * D + d] += load_elem(V, dtype, (j * H + h) * D + d);
+            }
+        }
+        for (int32_t d = 0; d < D; ++d) {
+            km[bh * D + d] /= (double)nb;
+            vm[bh * D + d] /= (double)nb;
+        }
+    }
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t bh = 0; bh < mb * H; ++bh) {
+        int64_t b = bh / H;
+        int32_t h = (int32_t)(bh % H);
+        for (int32_t e = 0; e < D; ++e) {
+            Kc[bh * D + e] = 0.0;
+            Vc[bh * D + e] = 0.0;
+        }
+        for (int32_t o = 0; o < 27; ++o) {
+            int64_t nb = find_block(blk_coord, mb, blk_coord[3 * b] + o / 9 - 1,
+                                    blk_coord[3 * b + 1] + (o / 3) % 3 - 1, blk_coord[3 * b + 2] + o % 3 - 1);
+            if (nb < 0) continue;
+            const double* mk = &km[(nb * H + h) * D];
+            const double* mv = &vm[(nb * H + h) * D];
+            const float* Wo = &W[(int64_t)o * D * D];
+            for (int32_t e = 0; e < D; ++e) {
+                double sk = 0.0, sv = 0.0;
+                for (int32_t d = 0; d < D; ++d) {
+                    sk += mk[d] * (double)Wo[d * D + e];
+                    sv += mv[d] * (double)Wo[d * D + e];
+                }
+                Kc[bh * D + e] += sk;
+                Vc[bh * D + e] += sv;
+            }
+        }
+    }
+    free(km);
+    free(vm);
+}
+
+/* Exported for tests: the convolution-compressed tokens of one sequence, [Mb, H, D] each. */
+int oracle_compress_conv(int64_t mb, int32_t H, int32_t D, int32_t dtype, const void* K, const void* V,
+                         const float* W, const int32_t* perm, const int32_t* blk_off,
+                         const int32_t* blk_coord, double* Kc, double* Vc) {
+    compress_conv(mb, H, D, dtype, K, V, W, perm, blk_off, blk_coord, Kc, Vc);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* 3-7. forward for a set of query rows                                                        */
 /* ------------------------------------------------------------------------------------------ */
 
@@ -375,19 +466,23 @@ static void select_blocks(int64_t mb, const double* z, int32_t own, int32_t k, i
  * When out, o_sel and o_win are all NULL only steps 3-4 run (compressed attention and the
  * selection), so the selection of many rows can be had at the cost of the compressed branch.
  */
-int oracle_forward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q, const void* K,
-                   const void* V, const float* gates, const float* Wc, int32_t topk,
-                   int32_t round_compressed, const int32_t* perm, const int32_t* tok_blk,
-                   const int32_t* blk_off, int64_t mb, const int64_t* nbr_off,
-                   const int32_t* nbr_idx, int64_t n_rows, const int64_t* rows,
-                   const int32_t* sel_in, double* out, double* o_cmp, double* o_sel,
-                   double* o_win, int32_t* sel, double* zc) {
+static int forward_impl(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q, const void* K,
+                        const void* V, const float* gates, const float* Wc, int32_t topk,
+                        int32_t round_compressed, const int32_t* perm, const int32_t* tok_blk,
+                        const int32_t* blk_off, int64_t mb, const int64_t* nbr_off,
+                        const int32_t* nbr_idx, int64_t n_rows, const int64_t* rows,
+                        const int32_t* sel_in, double* out, double* o_cmp, double* o_sel,
+                        double* o_win, int32_t* sel, double* zc, const float* Wconv,
+                        const int32_t* blk_coord, const float* Wg, const float* bg) {
     if (topk < 1 || D < 1 || H < 1) return -1;
     if (!rows) n_rows = n;
     double* Kc = (double*)malloc(sizeof(double) * (size_t)(mb * H * D + 1));
     double* Vc = (double*)malloc(sizeof(double) * (size_t)(mb * H * D + 1));
     if (!Kc || !Vc) return -1;
-    compress(mb, H, D, dtype, K, V, Wc, perm, blk_off, round_compressed, Kc, Vc);
+    if (Wconv)
+        compress_conv(mb, H, D, dtype, K, V, Wconv, perm, blk_off, blk_coord, Kc, Vc);
+    else
+        compress(mb, H, D, dtype, K, V, Wc, perm, blk_off, round_compressed, Kc, Vc);
     const double scale = 1.0 / sqrt((double)D);
     int64_t max_nb = 0;
     for (int64_t b = 0; b < mb; ++b)
@@ -482,14 +577,23 @@ int oracle_forward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q
             }
             attend(D, q, nk, kr, vr, scale, logits, ow);
 
-            /* 7. gated sum */
-            const float* g = &gates[(i * H + h) * 3];
+            /* 7. gated sum; with a gate predictor, g_c = sigmoid(bg_c + sum_d q_d Wg[d][c]) */
+            double g[3];
+            for (int32_t c = 0; c < 3; ++c) {
+                if (Wg) {
+                    double t = (double)bg[c];
+                    for (int32_t d = 0; d < D; ++d) t += q[d] * (double)Wg[d * 3 + c];
+                    g[c] = 1.0 / (1.0 + exp(-t));
+                } else {
+                    g[c] = (double)gates[(i * H + h) * 3 + c];
+                }
+            }
             for (int32_t d = 0; d < D; ++d) {
                 int64_t o = (ri * H + h) * D + d;
                 if (o_cmp) o_cmp[o] = oc[d];
                 if (o_sel) o_sel[o] = os[d];
                 if (o_win) o_win[o] = ow[d];
-                if (out) out[o] = (double)g[0] * oc[d] + (double)g[1] * os[d] + (double)g[2] * ow[d];
+                if (out) out[o] = g[0] * oc[d] + g[1] * os[d] + g[2] * ow[d];
             }
         }
         free(q); free(oc); free(os); free(ow); free(logits); free(z); free(s_loc);
@@ -498,6 +602,39 @@ int oracle_forward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q
     free(Kc);
     free(Vc);
     return 0;
+}
+
+int oracle_forward(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q, const void* K,
+                   const void* V, const float* gates, const float* Wc, int32_t topk,
+                   int32_t round_compressed, const int32_t* perm, const int32_t* tok_blk,
+                   const int32_t* blk_off, int64_t mb, const int64_t* nbr_off,
+                   const int32_t* nbr_idx, int64_t n_rows, const int64_t* rows,
+                   const int32_t* sel_in, double* out, double* o_cmp, double* o_sel,
+                   double* o_win, int32_t* sel, double* zc) {
+    return forward_impl(n, H, D, dtype, Q, K, V, gates, Wc, topk, round_compressed, perm, tok_blk,
+                        blk_off, mb, nbr_off, nbr_idx, n_rows, rows, sel_in, out, o_cmp, o_sel,
+                        o_win, sel, zc, NULL, NULL, NULL, NULL);
+}
+
+/*
+ * The forward with the compression by sparse 3D convolution (section 2b; Wconv [27, D, D],
+ * blk_coord [Mb, 3] of the sequence) and, when Wg is non-NULL, the gates predicted from each
+ * head's query (Direct3D-S2 summary page, "Technical principles", SSA item: the branches are
+ * aggregated with predicted gating scores): g = sigmoid(q . Wg + bg), Wg [D, 3], bg [3], shared
+ * by all heads, in the order (cmp, sel, win); `gates` is then not read. Other arguments as
+ * oracle_forward.
+ */
+int oracle_forward_variant(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q,
+                           const void* K, const void* V, const float* gates, const float* Wconv,
+                           const int32_t* blk_coord, const float* Wg, const float* bg, int32_t topk,
+                           const int32_t* perm, const int32_t* tok_blk, const int32_t* blk_off,
+                           int64_t mb, const int64_t* nbr_off, const int32_t* nbr_idx,
+                           int64_t n_rows, const int64_t* rows, const int32_t* sel_in, double* out,
+                           double* o_cmp, double* o_sel, double* o_win, int32_t* sel, double* zc) {
+    if (!Wconv || !blk_coord) return -1;
+    return forward_impl(n, H, D, dtype, Q, K, V, gates, NULL, topk, 0, perm, tok_blk, blk_off, mb,
+                        nbr_off, nbr_idx, n_rows, rows, sel_in, out, o_cmp, o_sel, o_win, sel, zc,
+                        Wconv, blk_coord, Wg, bg);
 }
 
 /* ------------------------------------------------------------------------------------------ */

@@ -695,3 +695,109 @@ def test_prologue_results_rounded_to_the_input_type():
     exact = oracle.qk_prologue(x, pos, g)
     rounded = oracle.qk_prologue(x, pos, g, round_to_input=True)
     np.testing.assert_array_equal(rounded, exact.astype(np.float16).astype(np.float64))
+
+
+# ---------------------------------------------------------------------------------------------
+# compression by sparse 3D convolution over the block grid; gates predicted from the queries
+# ---------------------------------------------------------------------------------------------
+
+def _conv_weights(D, seed, scale=None):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((27, D, D)) / np.sqrt(27 * D) if scale is None
+            else rng.standard_normal((27, D, D)) * scale).astype(np.float32)
+
+
+def test_conv_compression_with_only_the_centre_tap_is_mean_times_wc():
+    c, q, k, v, Wc = _tiny_inputs(seed=210)
+    Kc, Vc = oracle.compress(c, k, v, Wc)
+    Kc2, Vc2 = oracle.compress_conv(c, k, v, oracle.center_only_conv(Wc))
+    np.testing.assert_allclose(Kc2, Kc, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(Vc2, Vc, rtol=0, atol=1e-13)
+
+
+def test_conv_compression_matches_brute_force_over_block_neighbours():
+    # written out with dictionaries: the block means, then for every block the sum over the 27
+    # offsets of the neighbour's mean times that offset's matrix (absent neighbours skipped)
+    c, _ = _tiny_coords()
+    c = c[:500]
+    N, H, D = len(c), 2, 8
+    k, v = _rand((N, H, D), 211), _rand((N, H, D), 212)
+    W = _conv_weights(D, 213)
+    members = {}
+    for i, x in enumerate(c):
+        members.setdefault(tuple(int(t) // 8 for t in x), []).append(i)
+    blocks = sorted(members)
+    mk = {b: k[members[b]].mean(axis=0) for b in blocks}
+    mv = {b: v[members[b]].mean(axis=0) for b in blocks}
+    Kc, Vc = oracle.compress_conv(c, k, v, W)
+    for bi, b in enumerate(blocks):
+        ek = np.zeros((H, D))
+        ev = np.zeros((H, D))
+        for dx in (-1, 0, 1):
+            for dy in (-1, 0, 1):
+                for dz in (-1, 0, 1):
+                    nb = (b[0] + dx, b[1] + dy, b[2] + dz)
+                    if nb not in mk:
+                        continue
+                    Wo = W[9 * (dx + 1) + 3 * (dy + 1) + (dz + 1)].astype(np.float64)
+                    ek += mk[nb] @ Wo
+                    ev += mv[nb] @ Wo
+        np.testing.assert_allclose(Kc[bi], ek, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(Vc[bi], ev, rtol=0, atol=1e-12)
+
+
+def test_conv_compression_is_linear_in_the_kernel():
+    c, q, k, v, _ = _tiny_inputs(seed=214, D=16)
+    W1, W2 = _conv_weights(16, 215), _conv_weights(16, 216)
+    W1[13:] = 0.0   # disjoint taps: the fp32 sum W1 + W2 is exact
+    W2[:13] = 0.0
+    a = oracle.compress_conv(c, k, v, W1)
+    b = oracle.compress_conv(c, k, v, W2)
+    ab = oracle.compress_conv(c, k, v, W1 + W2)
+    for x, y, z in zip(a, b, ab):
+        np.testing.assert_allclose(z, x + y, rtol=0, atol=1e-12)
+
+
+def test_forward_with_centre_tap_and_explicit_gates_is_the_plain_forward():
+    c, q, k, v, Wc = _tiny_inputs(seed=217)
+    g = _gates(len(c), 2, None, seed=16)
+    plain = run(c, q, k, v, g, Wc, 4, 2)
+    conv = run(c, q, k, v, g, Wc, 4, 2, conv=oracle.center_only_conv(Wc))
+    assert np.array_equal(plain["sel"], conv["sel"])
+    for name in ("out", "o_cmp", "o_sel", "o_win"):
+        np.testing.assert_allclose(conv[name], plain[name], rtol=0, atol=1e-12)
+
+
+def test_predicted_gates():
+    c, q, k, v, Wc = _tiny_inputs(seed=218)
+    N, H, D = q.shape
+    W = _conv_weights(D, 219)
+    # a constant predictor (zero weights, bias logit(g)) is the constant gates g
+    gc = np.array([0.2, 0.5, 0.9])
+    const = run(c, q, k, v, None, Wc, 4, 2, conv=W,
+                gate=dict(w=np.zeros((D, 3), np.float32), b=np.log(gc / (1 - gc)).astype(np.float32)))
+    explicit = run(c, q, k, v, np.broadcast_to(gc.astype(np.float32), (N, H, 3)).copy(), Wc, 4, 2,
+                   conv=W)
+    np.testing.assert_allclose(const["out"], explicit["out"], rtol=0, atol=1e-6)
+    # a query-dependent predictor equals explicit gates holding sigmoid(q . Wg + bg) per head
+    rng = np.random.default_rng(220)
+    Wg = (rng.standard_normal((D, 3)) / np.sqrt(D)).astype(np.float32)
+    bg = rng.standard_normal(3).astype(np.float32)
+    pred = run(c, q, k, v, None, Wc, 4, 2, conv=W, gate=dict(w=Wg, b=bg))
+    logits = np.einsum("nhd,dc->nhc", q, Wg.astype(np.float64)) + bg.astype(np.float64)
+    gates = (1.0 / (1.0 + np.exp(-logits))).astype(np.float32)
+    ref = run(c, q, k, v, gates, Wc, 4, 2, conv=W)
+    np.testing.assert_allclose(pred["out"], ref["out"], rtol=0, atol=2e-7)   # gates rounded to f32
+    # the convolution changes the result (it is not silently the centre tap)
+    plain = run(c, q, k, v, gates, Wc, 4, 2)
+    assert np.abs(plain["out"] - ref["out"]).max() > 1e-2
+
+
+def test_conv_forward_is_invariant_under_block_translation():
+    c, q, k, v, Wc = _tiny_inputs(seed=221)
+    g = _gates(len(c), 2, None, seed=17)
+    W = _conv_weights(q.shape[2], 222)
+    a = run(c, q, k, v, g, Wc, 4, 2, conv=W)
+    b = run(c + np.array([16, 8, 24], np.int32), q, k, v, g, Wc, 4, 2, conv=W)
+    assert np.array_equal(a["sel"], b["sel"])
+    np.testing.assert_allclose(b["out"], a["out"], rtol=0, atol=1e-12)

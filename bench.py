@@ -345,6 +345,7 @@ def run_ours(args, rank, world, dist):
         "gpu_launches": int(launches),
         "clocks": clk,
     }
+    res["variants"] = measure_variants(plan, dev, cfg, pk.get("hbm_gbs", 6650.0))
     return res
 
 
@@ -371,6 +372,82 @@ def oracle_cost_model(cfg, coords, cu, t, n_rows, seed):
 
 def _cores():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def measure_variants(plan, dev, cfg, peak_hbm, steps=10, warmup=3):
+    """The forward with the options of ssa_forward_ex on the same workload: the attention prologue
+    (RMS normalisation and rotary embedding of q and k), and the compression by sparse 3D
+    convolution over the block grid with gates predicted from the queries. Per variant: ms per
+    forward (CUDA events) and the per-kernel breakdown; for the prologue's pooling kernel the HBM
+    rate of its bytes, for the convolution its fp32 FMA rate."""
+    import torch
+    import spatial_sparse_attention_b200 as ssa
+    D, H, N = cfg.D, cfg.H, dev["Q"].shape[0]
+    rng = np.random.default_rng(cfg.index * 1000 + 95)
+    w = {"q_gamma": (rng.random(D) + 0.5), "k_gamma": (rng.random(D) + 0.5),
+         "conv_w": rng.standard_normal((27, D, D)) / np.sqrt(27 * D),
+         "gate_w": rng.standard_normal((D, 3)) / np.sqrt(D), "gate_b": rng.standard_normal(3)}
+    w = {k: torch.from_numpy(v.astype(np.float32)).cuda() for k, v in w.items()}
+    variants = {
+        "prologue": dict(q_gamma=w["q_gamma"], k_gamma=w["k_gamma"], rope_theta=10000.0, eps=1e-6),
+        "conv_and_predicted_gates": dict(conv_w=w["conv_w"], gate_w=w["gate_w"], gate_b=w["gate_b"]),
+    }
+    out = torch.empty_like(dev["Q"])
+    res = {}
+    for name, kw in variants.items():
+        gates = None if "gate_w" in kw else dev["gates"]
+        wc = None if "conv_w" in kw else dev["Wc"]
+
+        def fwd():
+            plan.forward_ex(dev["Q"], dev["K"], dev["V"], gates, wc, cfg.topk, out=out, **kw)
+
+        for _ in range(warmup):
+            fwd()
+        torch.cuda.synchronize()
+        ssa.profile_reset()
+        ssa.profile_enable(True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fwd()
+        e1.record()
+        torch.cuda.synchronize()
+        ssa.profile_enable(False)
+        prof = ssa.profile_read()
+        if plan.status() != 0:
+            raise RuntimeError(f"device status set in variant {name}")
+        r = {"forward_ms": e0.elapsed_time(e1) / steps,
+             "breakdown_ms": {k: v[0] / steps for k, v in prof.items()}}
+        if name == "prologue":
+            # bytes of the pooling kernel with the prologue: K, V read; K_s, V_s written
+            byts = 4.0 * N * H * D * 2
+            pm = r["breakdown_ms"].get("pool")
+            if pm:
+                r["pool_hbm"] = {"bytes": byts, "achieved_gbs": byts / (pm * 1e-3) / 1e9,
+                                 "frac_of_measured_hbm": byts / (pm * 1e-3) / 1e9 / peak_hbm}
+        else:
+            cm = r["breakdown_ms"].get("conv")
+            if cm:
+                # FMAs: K and V, every head, D x D per (block, present neighbour)
+                flops = 2.0 * 2 * H * D * D * _present_neighbours(plan)
+                r["conv_fp32"] = {"flop": flops, "achieved_tflops": flops / (cm * 1e-3) / 1e12}
+        res[name] = r
+    return res
+
+
+def _present_neighbours(plan):
+    """Sum over occupied blocks of their occupied 3x3x3 neighbours (self included)."""
+    ex = plan.export()
+    bc = ex["blk_coord"].cpu().numpy().astype(np.int64)
+    bs = ex["blk_seq"].cpu().numpy().astype(np.int64)
+    keys = set(zip(bs.tolist(), bc[:, 0].tolist(), bc[:, 1].tolist(), bc[:, 2].tolist()))
+    n = 0
+    for s_, x, y, z in zip(bs.tolist(), bc[:, 0].tolist(), bc[:, 1].tolist(), bc[:, 2].tolist()):
+        for dx in (-1, 0, 1):
+            for dy in (-1, 0, 1):
+                for dz in (-1, 0, 1):
+                    n += (s_, x + dx, y + dy, z + dz) in keys
+    return n
 
 
 def cpu_baseline(cfg_name, target_s=20.0):

@@ -204,6 +204,45 @@ SSA_API ssa_status_t ssa_forward_prologue(ssa_plan_t plan, const void* q, const 
                                   int32_t* sel_out, void* stream);
 
 /*
+ * Options of ssa_forward_ex; a NULL pointer (or a zero-initialised struct) turns a part off.
+ *   q_gamma, k_gamma, rope_theta, rms_eps: the attention prologue of ssa_forward_prologue (both
+ *       weights set, or neither).
+ *   conv_w: device fp32 [27, D, D]. Compression by sparse 3D convolution over the block grid in
+ *       place of the block mean times Wc (Direct3D-S2 summary page, "Technical principles of
+ *       Direct3D-S2", SSA item: blocks become block-level tokens by sparse 3D convolution and
+ *       pooling). The block means of K and V go through one 3x3x3 convolution over the occupied
+ *       blocks of each sequence, stride 1, outputs at the occupied blocks only, an absent neighbour
+ *       contributing nothing: Kc_b = sum_o mean(K_{b+o}) . W_o, with W_o = conv_w[9(dx+1) +
+ *       3(dy+1) + (dz+1)] for the offset o = (dx, dy, dz), shared by K, V and all heads. The centre
+ *       tap alone (W_(0,0,0) = Wc, others zero) is the plain method.
+ *   gate_w, gate_b: device fp32 [D, 3] and [3]. Gates predicted from the queries (same item: the
+ *       branches are aggregated with predicted gating scores): g = sigmoid(q . gate_w + gate_b) per
+ *       token and head, q being the query as the attention sees it (after the prologue, in the
+ *       input type), order (cmp, sel, win). Both set, or neither.
+ */
+typedef struct {
+    const float* q_gamma;
+    const float* k_gamma;
+    float rope_theta;
+    float rms_eps;
+    const float* conv_w;
+    const float* gate_w;
+    const float* gate_b;
+} ssa_options_t;
+
+/*
+ * Forward pass with options (ssa_options_t; NULL = the plain ssa_forward). `gates` is not read,
+ * and may be NULL, when the gates are predicted; `wc` likewise with a convolution compression.
+ * sel_out: optional device int32 [N, H, k] (NULL = not written). Otherwise as ssa_forward; the
+ * first call with a convolution builds the plan's block neighbour table (27 per block).
+ * Errors: as ssa_forward, and SSA_ERR_INVALID_ARG for options set inconsistently.
+ */
+SSA_API ssa_status_t ssa_forward_ex(ssa_plan_t plan, const void* q, const void* k, const void* v,
+                            const float* gates, const float* wc, int32_t heads, int32_t head_dim,
+                            ssa_dtype_t dtype, int32_t topk, const ssa_options_t* options, void* out,
+                            int32_t* sel_out, void* stream);
+
+/*
  * ssa_forward on HOST buffers: copies q, k, v, gates, wc (host) to plan-owned device buffers,
  * runs the forward and copies the result into out (host). Pinned host memory gives overlapped,
  * full-speed copies; pageable memory works but is slower. Waits for the device before returning.
@@ -228,6 +267,16 @@ SSA_API ssa_status_t ssa_backward(ssa_plan_t plan, const void* q, const void* k,
 
 /* Wait for `stream`, then read and clear the plan's device status word. */
 SSA_API ssa_status_t ssa_last_device_status(ssa_plan_t plan, void* stream);
+
+/*
+ * Failure-detection check (measurement support, not part of the method): launches one warp that
+ * waits, with the same bounded mbarrier wait every kernel of this library uses, on a barrier that
+ * nothing arrives at, giving up after about max_cycles SM clock cycles (>= 1). The wait that runs
+ * out records a device timeout in the plan's status word: the next ssa_last_device_status (or any
+ * call that waits for the device) returns SSA_ERR_DEVICE_TIMEOUT and clears it; the context stays
+ * usable. Queues work on `stream` and returns without waiting.
+ */
+SSA_API ssa_status_t ssa_debug_wait_timeout(ssa_plan_t plan, int64_t max_cycles, void* stream);
 
 /* Release a plan and every buffer it owns (queued on the stream it was created on). */
 SSA_API ssa_status_t ssa_plan_destroy(ssa_plan_t plan);

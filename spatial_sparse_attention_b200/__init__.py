@@ -50,8 +50,10 @@ _SIGS = {
     "ssa_forward_host": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp],
     "ssa_forward_prologue": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float,
                              _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "ssa_forward_ex": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "ssa_backward": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp],
     "ssa_last_device_status": [_vp, _vp],
+    "ssa_debug_wait_timeout": [_vp, _i64, _vp],
     "ssa_plan_destroy": [_vp],
     "ssa_status_string": [_i32],
     "ssa_launch_count": [],
@@ -59,6 +61,12 @@ _SIGS = {
     "ssa_profile_reset": [],
     "ssa_profile_read": [_i32, _vp, _vp, _vp],
 }
+
+
+class Options(ctypes.Structure):
+    """ssa_options_t (include/ssa.h): the optional parts of ssa_forward_ex."""
+    _fields_ = [("q_gamma", _vp), ("k_gamma", _vp), ("rope_theta", ctypes.c_float),
+                ("rms_eps", ctypes.c_float), ("conv_w", _vp), ("gate_w", _vp), ("gate_b", _vp)]
 
 
 def _load():
@@ -282,6 +290,31 @@ class Plan:
                                         _stream(self.stream)), "ssa_forward_prologue")
         return (out, sel) if return_sel else out
 
+    def forward_ex(self, q, k, v, gates, wc, topk: int, q_gamma=None, k_gamma=None,
+                   rope_theta: float = 10000.0, eps: float = 1e-6, conv_w=None, gate_w=None,
+                   gate_b=None, out: Optional[torch.Tensor] = None, return_sel: bool = False):
+        """ssa_forward_ex: the prologue (q_gamma, k_gamma [D]), the compression by sparse 3D
+        convolution over the block grid (conv_w [27, D, D]) and gates predicted from the queries
+        (gate_w [D, 3], gate_b [3]), each optional (fp32 CUDA tensors). gates / wc may be None when
+        predicted / replaced by the convolution."""
+        dt = q.dtype
+        for t in (q, k, v):
+            _dev(t, dt)
+            if t.dim() != 3 or t.shape[0] != self.N:
+                raise ValueError("q, k, v must be [N, H, D]")
+        H, D = q.shape[1], q.shape[2]
+        for t in (gates, wc, q_gamma, k_gamma, conv_w, gate_w, gate_b):
+            if t is not None:
+                _dev(t, torch.float32)
+        opt = Options(_ptr(q_gamma), _ptr(k_gamma), float(rope_theta), float(eps), _ptr(conv_w),
+                      _ptr(gate_w), _ptr(gate_b))
+        out = torch.empty_like(q) if out is None else _dev(out, dt)
+        sel = torch.empty(self.N, H, topk, dtype=torch.int32, device=q.device) if return_sel else None
+        _check(lib.ssa_forward_ex(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(gates),
+                                  _ptr(wc), H, D, _DTYPE[dt], topk, ctypes.byref(opt),
+                                  out.data_ptr(), _ptr(sel), _stream(self.stream)), "ssa_forward_ex")
+        return (out, sel) if return_sel else out
+
     def forward_host(self, q, k, v, gates, wc, topk: int, out: torch.Tensor):
         """Forward on host (preferably pinned) CPU tensors; copies run inside the library."""
         for t in (q, k, v, gates, wc, out):
@@ -302,6 +335,11 @@ class Plan:
                                 _DTYPE[dt], topk, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                 _stream(self.stream)), "ssa_backward")
         return dq, dk, dv
+
+    def debug_wait_timeout(self, max_cycles: int):
+        """ssa_debug_wait_timeout: a bounded wait that runs out on purpose (failure detection)."""
+        _check(lib.ssa_debug_wait_timeout(self._h, int(max_cycles), _stream(self.stream)),
+               "ssa_debug_wait_timeout")
 
     def status(self):
         """Waits for the stream, returns and clears the device status (0 = ok)."""

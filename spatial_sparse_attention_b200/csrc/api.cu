@@ -289,22 +289,37 @@ ssa_status_t check_forward_args(Plan* p, const void* q, const void* k, const voi
     return SSA_OK;
 }
 
+// What a forward call computes beyond the plain method (everything off by default).
+struct Options {
+    Prologue pro;
+    const float* conv_w = nullptr;   // [27, D, D]: compression by sparse 3D convolution
+    const float* gate_w = nullptr;   // [D, 3] and [3]: gates predicted from the queries
+    const float* gate_b = nullptr;
+};
+
+// A workspace buffer of `bytes` allocated on first use (kept with the workspace).
+template <typename P>
+ssa_status_t ensure_buffer(Plan* p, Workspace& w, P*& buf, size_t bytes, cudaStream_t st) {
+    if (buf) return SSA_OK;
+    buf = (P*)p->alloc(std::max<size_t>(bytes, 16), st, p->alloc_ctx);
+    if (!buf) return SSA_ERR_ALLOC;
+    w.owned.push_back(buf);
+    return SSA_OK;
+}
+
 ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, const float* gates,
                          const float* wc, int32_t H, int32_t D, ssa_dtype_t dt, int32_t topk,
                          void* out, int32_t* sel_out, cudaStream_t st,
-                         const BranchOut& bo = BranchOut(), const Prologue& pro = Prologue()) {
+                         const BranchOut& bo = BranchOut(), const Options& opt = Options()) {
     ssa_status_t rc = ensure_workspace(p, H, D, dt, topk, st);
     if (rc != SSA_OK) return rc;
     Workspace& w = p->ws;
+    const Prologue& pro = opt.pro;
     if (pro.on() && dt == SSA_F32) {
         // fp32 path: the prologue is a pass of its own into workspace copies of q and k
         const size_t bytes = sizeof(float) * (size_t)p->N * H * D;
-        for (float** buf : {&w.qp, &w.kp}) {
-            if (*buf) continue;
-            *buf = (float*)p->alloc(bytes, st, p->alloc_ctx);
-            if (!*buf) return SSA_ERR_ALLOC;
-            w.owned.push_back(*buf);
-        }
+        if ((rc = ensure_buffer(p, w, w.qp, bytes, st)) != SSA_OK) return rc;
+        if ((rc = ensure_buffer(p, w, w.kp, bytes, st)) != SSA_OK) return rc;
         {
             ProfScope ps("prologue", st);
             launch_qk_prologue_f32(p, (const float*)q, pro.q_gamma, pro, H, D, w.qp, st);
@@ -314,18 +329,35 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
         k = w.kp;
     }
     const Prologue fused = dt == SSA_F32 ? Prologue() : pro;   // 16-bit: inside pool and forward
+    float* means = nullptr;
+    if (opt.conv_w) {
+        if ((rc = ensure_block_neighbours(p, st)) != SSA_OK) return rc;
+        if ((rc = ensure_buffer(p, w, w.means, sizeof(float) * 2 * (size_t)H * p->Mb * D, st)) != SSA_OK)
+            return rc;
+        means = w.means;
+    }
     {
         ProfScope ps("pool", st);
-        launch_pool(p, w, k, v, wc, fused, st);
+        launch_pool(p, w, k, v, wc, fused, means, st);
+    }
+    if (opt.conv_w) {
+        ProfScope ps("conv", st);
+        launch_conv_compress(p, w, means, opt.conv_w, st);
     }
     trace_step("pool", st);
+    if (opt.gate_w) {
+        if ((rc = ensure_buffer(p, w, w.gates, sizeof(float) * 3 * (size_t)p->N * H, st)) != SSA_OK) return rc;
+        gates = w.gates;
+        if (dt == SSA_F32) launch_gates_f32(p, (const float*)q, opt.gate_w, opt.gate_b, H, D, w.gates, st);
+    }
     if (dt == SSA_F32) {
         // the CUDA-core path walks the per-token neighbour lists
         if ((rc = ensure_neighbours(p, st)) != SSA_OK) return rc;
         launch_forward_simt(p, w, q, k, v, gates, out, bo, st);
-    }
-    else {
-        if ((rc = launch_select_tc(p, w, q, fused, st)) != SSA_OK) return rc;
+    } else {
+        if ((rc = launch_select_tc(p, w, q, fused, opt.gate_w, opt.gate_b, opt.gate_w ? w.gates : nullptr, st)) !=
+            SSA_OK)
+            return rc;
         trace_step("select", st);
         if ((rc = launch_forward_tc(p, w, q, gates, out, bo, fused, st)) != SSA_OK) return rc;
     }
@@ -476,13 +508,40 @@ ssa_status_t ssa_forward_prologue(ssa_plan_t p, const void* q, const void* k, co
     ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out);
     if (rc != SSA_OK) return rc;
     if (!q_gamma || !k_gamma || !(rope_theta > 1.0f) || !(eps >= 0.0f)) return SSA_ERR_INVALID_ARG;
-    Prologue pro;
-    pro.q_gamma = q_gamma;
-    pro.k_gamma = k_gamma;
-    pro.theta = rope_theta;
-    pro.eps = eps;
+    Options opt;
+    opt.pro.q_gamma = q_gamma;
+    opt.pro.k_gamma = k_gamma;
+    opt.pro.theta = rope_theta;
+    opt.pro.eps = eps;
     return run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, sel_out,
-                       (cudaStream_t)stream, BranchOut(), pro);
+                       (cudaStream_t)stream, BranchOut(), opt);
+}
+
+ssa_status_t ssa_forward_ex(ssa_plan_t p, const void* q, const void* k, const void* v,
+                            const float* gates, const float* wc, int32_t heads, int32_t head_dim,
+                            ssa_dtype_t dtype, int32_t topk, const ssa_options_t* options, void* out,
+                            int32_t* sel_out, void* stream) {
+    Options opt;
+    if (options) {
+        const ssa_options_t& o = *options;
+        if ((o.q_gamma == nullptr) != (o.k_gamma == nullptr)) return SSA_ERR_INVALID_ARG;
+        if (o.q_gamma && (!(o.rope_theta > 1.0f) || !(o.rms_eps >= 0.0f))) return SSA_ERR_INVALID_ARG;
+        if ((o.gate_w == nullptr) != (o.gate_b == nullptr)) return SSA_ERR_INVALID_ARG;
+        opt.pro.q_gamma = o.q_gamma;
+        opt.pro.k_gamma = o.k_gamma;
+        opt.pro.theta = o.rope_theta;
+        opt.pro.eps = o.rms_eps;
+        opt.conv_w = o.conv_w;
+        opt.gate_w = o.gate_w;
+        opt.gate_b = o.gate_b;
+    }
+    // the gates input is not read when they are predicted, nor wc with a convolution compression
+    static const float kUnused = 0.0f;
+    ssa_status_t rc = check_forward_args(p, q, k, v, opt.gate_w ? &kUnused : gates, opt.conv_w ? &kUnused : wc,
+                                         heads, head_dim, dtype, topk, out);
+    if (rc != SSA_OK) return rc;
+    return run_forward(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, sel_out,
+                       (cudaStream_t)stream, BranchOut(), opt);
 }
 
 ssa_status_t ssa_forward_host(ssa_plan_t p, const void* q, const void* k, const void* v,
@@ -555,6 +614,11 @@ ssa_status_t ssa_last_device_status(ssa_plan_t p, void* stream) {
         cudaMemsetAsync(p->d_status, 0, sizeof(int32_t), st) || cudaStreamSynchronize(st))
         return SSA_ERR_CUDA;
     return map_device_status(s);
+}
+
+ssa_status_t ssa_debug_wait_timeout(ssa_plan_t p, int64_t max_cycles, void* stream) {
+    if (!p || max_cycles < 1) return SSA_ERR_INVALID_ARG;
+    return launch_wait_timeout(p, max_cycles, (cudaStream_t)stream);
 }
 
 ssa_status_t ssa_plan_destroy(ssa_plan_t p) {

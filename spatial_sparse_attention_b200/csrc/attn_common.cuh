@@ -40,6 +40,10 @@ struct FwdParams {
     float* base;
     void* out;
     float* bout[3];   // optional per-branch outputs (fp32, token order), null when not wanted
+    // gates predicted from the queries (selection kernel; null gate_w = off)
+    const float* gate_w;
+    const float* gate_b;
+    float* gates_out;
     // attention prologue on the query tiles (null q_gamma = off)
     const float* q_gamma;
     const int32_t* coords;

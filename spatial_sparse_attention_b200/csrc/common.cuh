@@ -69,6 +69,9 @@ struct Workspace {
     // fp32 path with the prologue: transformed q and k (allocated on first use)
     float* qp = nullptr;       // [N, H, D]
     float* kp = nullptr;       // [N, H, D]
+    // convolution compression and predicted gates (allocated on first use)
+    float* means = nullptr;    // [2][H][Mb][D] block means of K and V
+    float* gates = nullptr;    // [N, H, 3] predicted gates
     // host-buffer entry point staging (allocated on first use)
     void* h_q = nullptr; void* h_k = nullptr; void* h_v = nullptr; void* h_out = nullptr;
     float* h_gates = nullptr; float* h_wc = nullptr;
@@ -118,6 +121,7 @@ struct Plan {
     int32_t* hvals = nullptr;
     uint64_t hmask = 0;
     int32_t nbr_cap = 32;        // per-warp sort buffer of the neighbour-list kernel
+    int32_t* blk_nbr = nullptr;  // [Mb][27] block at offset o of every block (-1 = none), first use
     int32_t* qt_pos = nullptr;   // [n_qtiles] first sorted position of each query tile
     int32_t* qt_len = nullptr;   // [n_qtiles]
     int32_t* qt_seq = nullptr;   // [n_qtiles]
@@ -179,9 +183,19 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t s);
 ssa_status_t ensure_neighbour_counts(Plan* p, cudaStream_t s);
 ssa_status_t ensure_neighbours(Plan* p, cudaStream_t s);
 
-// pool.cu (with the prologue applied to k on the way when pro.on(), 16-bit types)
+// pool.cu (with the prologue applied to k on the way when pro.on(), 16-bit types). With `means`
+// non-null: writes the fp32 block means [2][H][Mb][D] (K, then V) instead of the compressed tokens.
 void launch_pool(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,
-                 const Prologue& pro, cudaStream_t s);
+                 const Prologue& pro, float* means, cudaStream_t s);
+
+// conv.cu: compressed tokens by the sparse 3D convolution over the block grid from the block
+// means (w.kc/w.vc, and the grouped copies for 16-bit types); the 27 neighbours of every block.
+ssa_status_t ensure_block_neighbours(Plan* p, cudaStream_t s);
+void launch_conv_compress(const Plan* p, const Workspace& w, const float* means, const float* wconv,
+                          cudaStream_t s);
+// gates [N, H, 3] = sigmoid(q . wg + bg) for fp32 q (the 16-bit path predicts them in select.cu)
+void launch_gates_f32(const Plan* p, const float* q, const float* wg, const float* bg, int H, int D,
+                      float* gates, cudaStream_t s);
 
 // prologue.cu: out = prologue(x) for fp32 [N, H, D] rows (the fp32 path's stand-alone pass)
 void launch_qk_prologue_f32(const Plan* p, const float* x, const float* gamma, const Prologue& pro,
@@ -200,8 +214,10 @@ void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const
 
 // select.cu (bf16 / fp16 path): the selected blocks of every (token, head) into w.sel, sorted
 // token order (the prologue, when on, is applied to each query tile after it is loaded)
+// With gate_w non-null it also writes gates_out [N, H, 3] = sigmoid(q . gate_w + gate_b), q being the
+// query as the attention sees it (after the prologue).
 ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
-                              cudaStream_t s);
+                              const float* gate_w, const float* gate_b, float* gates_out, cudaStream_t s);
 
 // attn_fwd.cu (bf16 / fp16 path): the fused tensor-core forward over w.sel (the prologue, when on, is
 // applied to each query tile after it is loaded)
@@ -212,6 +228,9 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
 ssa_status_t launch_backward(Plan* p, const Workspace& w, const void* q, const void* k,
                              const void* v, const float* gates, const float* wc, const void* dout,
                              void* dq, void* dk, void* dv, cudaStream_t s);
+
+// selftest.cu: a bounded wait on an mbarrier nothing arrives at (records DEV_TIMEOUT)
+ssa_status_t launch_wait_timeout(Plan* p, int64_t max_cycles, cudaStream_t s);
 
 // selection export (attn_fwd.cu): sel_out [N,H,k] in token order from the sorted-order buffer.
 void launch_export_sel(const Plan* p, const Workspace& w, int32_t* sel_out, cudaStream_t s);
@@ -233,6 +252,16 @@ template <> struct Elem<__nv_bfloat16> {
     static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
     static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
 };
+
+// Byte offset of element column d (a multiple of 8) of row `row` of a grouped matrix with D
+// columns of a 16-bit type: rows go 8 at a time; a group stores its D/32 column chunks as 512-byte
+// atoms of 8 rows x 64 bytes whose 16-byte units of row i are permuted by unit ^= (i >> 1) & 3
+// (the tensor cores' shared-memory operand order with 64-byte swizzle).
+__device__ __forceinline__ int64_t grouped_off(int64_t row, int d, int D) {
+    const int64_t g = row >> 3;
+    const int i = (int)(row & 7), c = d >> 5, u = (d & 31) >> 3;
+    return g * (int64_t)(D / 32) * 512 + c * 512 + i * 64 + ((u ^ ((i >> 1) & 3)) << 4);
+}
 
 // Packed (sequence, x, y, z) key of the coordinate hash; each field < 2^16.
 __device__ __forceinline__ uint64_t pack_cell(int32_t s, int32_t x, int32_t y, int32_t z) {

@@ -724,6 +724,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     p->hmask = hsize - 1;
     p->nbr_cap = cap;
     p->nbr_idx = nullptr;
+    p->blk_nbr = nullptr;   // block neighbour table (convolution compression), built on first use
 
     // ---- query tiles and their window key unions (tensor-core window kernel) ----------------------
     std::vector<int32_t> qpos, qlen, qseq;

@@ -11,6 +11,9 @@
 // written twice: at its padded rows and, packed with the other small blocks of its sequence, in
 // that sequence's pool after all padded rows.
 //
+// With a convolution compression (`means` non-null) the block means go to `means` instead and
+// the compressed tokens are made by the convolution kernel (conv.cu).
+//
 // Grouped order (16-bit types): rows are taken 8 at a time; a group stores its D/32 column chunks
 // one after the other, each as a 512-byte atom of 8 rows x 64 bytes in which the four 16-byte
 // units of row i are permuted by unit ^= (i >> 1) & 3. This is the shared-memory operand order of
@@ -24,14 +27,6 @@
 namespace ssa {
 
 namespace {
-
-// byte offset of element column d of row `row` (16-byte unit granularity: d % 8 == 0) inside a
-// grouped matrix with D columns
-__device__ __forceinline__ int64_t grouped_off(int64_t row, int d, int D) {
-    const int64_t g = row >> 3;
-    const int i = (int)(row & 7), c = d >> 5, u = (d & 31) >> 3;
-    return g * (int64_t)(D / 32) * 512 + c * 512 + i * 64 + ((u ^ ((i >> 1) & 3)) << 4);
-}
 
 // Work split inside a block's CTA: a thread owns two adjacent 16-byte column units of the token
 // rows (32 bytes) and one of kLanes token lanes; lane L visits the block's tokens L, L + kLanes, ...
@@ -52,7 +47,8 @@ __global__ void __launch_bounds__(512) k_pool(const T* __restrict__ K, const T* 
                                                int H, int D, int64_t Nks, T* __restrict__ ks,
                                                T* __restrict__ vs, T* __restrict__ kc,
                                                T* __restrict__ vc, int64_t Mb8,
-                                               T* __restrict__ kcg, T* __restrict__ vcg) {
+                                               T* __restrict__ kcg, T* __restrict__ vcg,
+                                               float* __restrict__ means) {
     constexpr int kVec = 16 / sizeof(T);
     extern __shared__ float mean[];   // [2][H*D]: K means then V means
     __shared__ int32_t toks[kMaxBlockTokens];
@@ -132,6 +128,14 @@ __global__ void __launch_bounds__(512) k_pool(const T* __restrict__ K, const T* 
         }
     }
     __syncthreads();
+    if (means) {
+        // compression by convolution: the block means go out [2][H][Mb][D] (K, then V)
+        for (int o = threadIdx.x; o < 2 * HD; o += blockDim.x) {
+            const int which = o / HD, h = (o % HD) / D, e = o % D;
+            means[(((int64_t)which * H + h) * Mb + b) * D + e] = mean[o];
+        }
+        return;
+    }
     // Kc[h][b][e] = sum_d mean[h][d] * Wc[d][e]
     for (int o = threadIdx.x; o < HD; o += blockDim.x) {
         const int h = o / D, e = o % D;
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(512) k_pool_pro(const T* __restrict__ K, const
                                                    T* __restrict__ ks, T* __restrict__ vs,
                                                    T* __restrict__ kc, T* __restrict__ vc,
                                                    int64_t Mb8, T* __restrict__ kcg,
-                                                   T* __restrict__ vcg) {
+                                                   T* __restrict__ vcg, float* __restrict__ means) {
     constexpr int kVec = 8;
     extern __shared__ float part[];   // [kProLanes][2][H*D] per-lane sums, then the means
     __shared__ int32_t toks[kMaxBlockTokens];
@@ -280,6 +284,13 @@ __global__ void __launch_bounds__(512) k_pool_pro(const T* __restrict__ K, const
     }
     __syncthreads();
     const float* mean = part;
+    if (means) {
+        for (int o = threadIdx.x; o < 2 * HD; o += blockDim.x) {
+            const int which = o / HD, h = (o % HD) / D, e = o % D;
+            means[(((int64_t)which * H + h) * Mb + b) * D + e] = mean[o];
+        }
+        return;
+    }
     for (int o = threadIdx.x; o < HD; o += blockDim.x) {
         const int h = o / D, e = o % D;
         const float* mk = mean + h * D;
@@ -302,7 +313,7 @@ __global__ void __launch_bounds__(512) k_pool_pro(const T* __restrict__ K, const
 
 template <typename T>
 void run_pool_pro(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,
-                  const Prologue& pro, cudaStream_t st) {
+                  const Prologue& pro, float* means, cudaStream_t st) {
     // heads per pass: as few passes over the block's tokens as 512 threads allow, heads spread evenly
     const int max_hpp = 512 / (16 * kProLanes);
     const int hpp = (int)cdiv(w.H, cdiv(w.H, max_hpp));
@@ -313,13 +324,13 @@ void run_pool_pro(const Plan* p, const Workspace& w, const void* k, const void* 
     k_pool_pro<T><<<(unsigned)p->Mb, threads, smem, st>>>(
         (const T*)k, (const T*)v, wc, p->perm, p->blk_off, p->blk_poff, p->blk_tpool, p->blk_seq,
         p->seq_pool, p->coords, pro.k_gamma, pro.theta, pro.eps, p->Mb, w.H, w.D, p->Nks,
-        (T*)w.ks, (T*)w.vs, (T*)w.kc, (T*)w.vc, w.Mb8, (T*)w.kcg, (T*)w.vcg);
+        (T*)w.ks, (T*)w.vs, (T*)w.kc, (T*)w.vc, w.Mb8, (T*)w.kcg, (T*)w.vcg, means);
     note_launch();
 }
 
 template <typename T>
 void run_pool(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,
-              cudaStream_t st) {
+              float* means, cudaStream_t st) {
     constexpr int kVec = 16 / sizeof(T);
     const int HD = w.H * w.D;
     const int pairs = HD / (2 * kVec);
@@ -334,23 +345,23 @@ void run_pool(const Plan* p, const Workspace& w, const void* k, const void* v, c
     kern<<<(unsigned)p->Mb, threads, smem, st>>>(
         (const T*)k, (const T*)v, wc, p->perm, p->blk_off, p->blk_poff, p->blk_tpool, p->blk_seq,
         p->seq_pool, p->Mb, w.H, w.D, p->Nks,
-        (T*)w.ks, (T*)w.vs, (T*)w.kc, (T*)w.vc, w.Mb8, (T*)w.kcg, (T*)w.vcg);
+        (T*)w.ks, (T*)w.vs, (T*)w.kc, (T*)w.vc, w.Mb8, (T*)w.kcg, (T*)w.vcg, means);
     note_launch();
 }
 
 }  // namespace
 
 void launch_pool(const Plan* p, const Workspace& w, const void* k, const void* v, const float* wc,
-                 const Prologue& pro, cudaStream_t st) {
+                 const Prologue& pro, float* means, cudaStream_t st) {
     if (pro.on() && w.dtype != SSA_F32) {
-        if (w.dtype == SSA_BF16) run_pool_pro<__nv_bfloat16>(p, w, k, v, wc, pro, st);
-        else run_pool_pro<__half>(p, w, k, v, wc, pro, st);
+        if (w.dtype == SSA_BF16) run_pool_pro<__nv_bfloat16>(p, w, k, v, wc, pro, means, st);
+        else run_pool_pro<__half>(p, w, k, v, wc, pro, means, st);
         return;
     }
     switch (w.dtype) {
-    case SSA_F32: run_pool<float>(p, w, k, v, wc, st); break;
-    case SSA_BF16: run_pool<__nv_bfloat16>(p, w, k, v, wc, st); break;
-    default: run_pool<__half>(p, w, k, v, wc, st); break;
+    case SSA_F32: run_pool<float>(p, w, k, v, wc, means, st); break;
+    case SSA_BF16: run_pool<__nv_bfloat16>(p, w, k, v, wc, means, st); break;
+    default: run_pool<__half>(p, w, k, v, wc, means, st); break;
     }
 }
 

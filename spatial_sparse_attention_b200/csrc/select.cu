@@ -1,7 +1,9 @@
 // Block selection for the bf16 / fp16 path: for every (token, head), the own block plus the top
 // (k-1) other blocks of its sequence by compressed logit (Direct3D-S2 summary page, "Technical
 // principles", SSA item: the important blocks are chosen from the compression module's attention
-// scores). It runs before the fused attention kernel, which reads the selection back.
+// scores). It runs before the fused attention kernel, which reads the selection back. On request
+// it also predicts the gates from the query tile it holds (same item: the branches are
+// aggregated with predicted gating scores).
 //
 // One CTA per (query tile of 128 tokens in block order, head), 192 threads:
 //   warp 0     producer: the sequence's compressed keys, 64 per tile, into a two-stage ring by 1D
@@ -185,6 +187,30 @@ __global__ void __launch_bounds__(kThreads, 3) k_ssa_select(const __grid_constan
             for (int q = KM - 1; q > 0; --q) tk[q] = max(tk[q], min(tk[q - 1], key));
             tk[0] = max(tk[0], key);
         };
+        if (P.gate_w && row_ok) {
+            // gates predicted from this row's query (as the attention sees it, after the prologue):
+            // sigmoid(q . gate_w + gate_b), one per branch
+            float t0 = P.gate_b[0], t1 = P.gate_b[1], t2 = P.gate_b[2];
+#pragma unroll 1
+            for (int c16 = 0; c16 < D / 8; ++c16) {
+                const uint4 u = *reinterpret_cast<const uint4*>(g + L::kQ + (c16 >> 2) * L::kQReg +
+                                                                 tc::sw64(row, c16 & 3));
+                const uint32_t* wv = reinterpret_cast<const uint32_t*>(&u);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int d = c16 * 8 + 2 * q;
+                    const float a = unpack_lo<T>(wv[q]), bq = unpack_hi<T>(wv[q]);
+                    const float* w0 = P.gate_w + d * 3;
+                    t0 = fmaf(a, w0[0], fmaf(bq, w0[3], t0));
+                    t1 = fmaf(a, w0[1], fmaf(bq, w0[4], t1));
+                    t2 = fmaf(a, w0[2], fmaf(bq, w0[5], t2));
+                }
+            }
+            float* go = P.gates_out + ((int64_t)tok * H + h) * 3;
+            go[0] = 1.0f / (1.0f + __expf(-t0));
+            go[1] = 1.0f / (1.0f + __expf(-t1));
+            go[2] = 1.0f / (1.0f + __expf(-t2));
+        }
         float4* stage4 = reinterpret_cast<float4*>(g + L::kStage) + row;
         const float* stage1 = reinterpret_cast<const float*>(stage4);
         bool ok = true;
@@ -311,7 +337,7 @@ ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, cudaStream_t st) {
 }  // namespace
 
 ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
-                              cudaStream_t st) {
+                              const float* gate_w, const float* gate_b, float* gates_out, cudaStream_t st) {
     FwdParams P = FwdParams();
     P.q = q;
     P.kcg = w.kcg;
@@ -327,6 +353,9 @@ ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, 
     P.coords = p->coords;
     P.theta = pro.theta;
     P.eps = pro.eps;
+    P.gate_w = gate_w;
+    P.gate_b = gate_b;
+    P.gates_out = gates_out;
     P.N = p->N;
     P.Mb = p->Mb;
     P.Mb8 = w.Mb8;

@@ -142,7 +142,7 @@ def head_slice(t: dict, heads):
 
 
 def validate_gpu_selection(coords, cu, t, topk, r, gpu_sel, blk_seq, dtype, rows=None,
-                           heads=None, prologue=None):
+                           heads=None, prologue=None, conv=None, gate=None):
     """Check the GPU's selection of `rows` (None = all) and `heads` (None = all) against the
     oracle's own: equal sets, or near ties within the stated gap. Returns (the GPU selection of
     those rows and heads, report)."""
@@ -152,14 +152,15 @@ def validate_gpu_selection(coords, cu, t, topk, r, gpu_sel, blk_seq, dtype, rows
     gs = gpu_sel[rows] if heads is None else gpu_sel[rows][:, list(heads)]
     # the oracle's own selection (compressed branch only), then the rows whose set differs
     own = oracle.forward(coords, cu, th["Q"], th["K"], th["V"], th["gates"], th["Wc"], topk, r,
-                         rows=rows, branches=False, prologue=prologue)["sel"]
+                         rows=rows, branches=False, prologue=prologue, conv=conv, gate=gate)["sel"]
     same = np.all(np.sort(gs, axis=2) == np.sort(own, axis=2), axis=2)
     assert np.array_equal(gs[:, :, 0], own[:, :, 0]), "slot 0 must be the own block"
     bad = np.nonzero(~same.all(axis=1))[0]
     worst = 0.0
     if len(bad):
         zr = oracle.forward(coords, cu, th["Q"], th["K"], th["V"], th["gates"], th["Wc"], topk, r,
-                            rows=rows[bad], branches=False, want_z=True, prologue=prologue)
+                            rows=rows[bad], branches=False, want_z=True, prologue=prologue,
+                            conv=conv, gate=gate)
         _, worst = selection_agreement(gs[bad], zr["sel"], zr["z"],
                                        blk_base_of_rows(cu, rows[bad], blk_seq), dtype)
     report = dict(pairs=int(same.size), mismatched=int((~same).sum()), worst_logit_gap=worst)
@@ -168,17 +169,17 @@ def validate_gpu_selection(coords, cu, t, topk, r, gpu_sel, blk_seq, dtype, rows
 
 
 def oracle_on_gpu_selection(coords, cu, t, topk, r, gpu_sel, blk_seq, dtype, rows=None,
-                            heads=None, prologue=None):
+                            heads=None, prologue=None, conv=None, gate=None):
     """The fp64 oracle's forward for `rows` (None = all) and `heads` (None = all), evaluated with
     the GPU's selection once that selection has been validated against the oracle's own.
 
     Returns (reference dict with out / o_cmp / o_sel / o_win [R, H', D] and rows, report)."""
     rows = np.arange(len(coords)) if rows is None else np.asarray(rows)
     gs, report = validate_gpu_selection(coords, cu, t, topk, r, gpu_sel, blk_seq, dtype, rows,
-                                        heads, prologue)
+                                        heads, prologue, conv, gate)
     th = head_slice(t, heads)
     ref = oracle.forward(coords, cu, th["Q"], th["K"], th["V"], th["gates"], th["Wc"], topk, r,
-                         rows=rows, sel_in=gs, prologue=prologue)
+                         rows=rows, sel_in=gs, prologue=prologue, conv=conv, gate=gate)
     return ref, report
 
 

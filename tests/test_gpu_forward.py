@@ -243,3 +243,19 @@ def test_too_many_blocks_in_a_sequence_is_unsupported():
     with pytest.raises(ssa.SSAError) as e:
         plan.forward(q, q, q, gates, torch.eye(32, device="cuda"), 2)
     assert e.value.name == "SSA_ERR_UNSUPPORTED"
+
+
+def test_bounded_wait_timeout_is_reported_and_the_next_call_is_clean():
+    """A bounded mbarrier wait that runs out (nothing ever arrives) is reported as
+    SSA_ERR_DEVICE_TIMEOUT by the next status read; the plan and the context stay usable."""
+    cfg = workloads.CONFIGS["small"]
+    c, cu, g = coords_of("small")
+    plan = make_plan(c, cu, g, cfg.radius)
+    plan.debug_wait_timeout(2_000_000)   # about a millisecond at the SM clock
+    assert plan.status() == 7             # SSA_ERR_DEVICE_TIMEOUT, and cleared by the read
+    assert plan.status() == 0
+    t = tensors_of("small")
+    out, sel, _ = gpu_forward(plan, t, cfg.topk)
+    bs = plan.export()["blk_seq"].cpu().numpy()
+    ref, _ = oracle_on_gpu_selection(c, cu, t, cfg.topk, cfg.radius, sel.cpu().numpy(), bs, cfg.dtype)
+    check_close(_pick(out, ref["rows"], None), ref["out"], cfg.dtype, "after timeout")

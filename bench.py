@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(workloads.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the timing of the forward's options (prologue, convolution, gates)")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of the config's "
                          "(a smaller cut for profiling; 0 = the config's own)")
@@ -345,7 +347,8 @@ def run_ours(args, rank, world, dist):
         "gpu_launches": int(launches),
         "clocks": clk,
     }
-    res["variants"] = measure_variants(plan, dev, cfg, pk.get("hbm_gbs", 6650.0))
+    if not args.no_variants:
+        res["variants"] = measure_variants(plan, dev, cfg, pk.get("hbm_gbs", 6650.0))
     return res
 
 

@@ -614,14 +614,14 @@ __global__ void __launch_bounds__(kThreads, FL<D, KM>::kMinBlocks) k_ssa_fwd(con
             if (__any_sync(0xffffffffu, vm != ~0ull)) apply_bits(s, vm);
             float mx[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[i], s[i + 8]);
-#pragma unroll
-            for (int e = 16; e < 64; e += 8) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[e + i]);
+            for (int i = 0; i < 8; ++i) {
+                mx[i] = tc::fmax3(s[i], s[i + 8], s[i + 16]);
+                mx[i] = tc::fmax3(mx[i], s[i + 24], s[i + 32]);
+                mx[i] = tc::fmax3(mx[i], s[i + 40], s[i + 48]);
+                mx[i] = fmaxf(mx[i], s[i + 56]);
             }
-            const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float tmax = tc::fmax3(tc::fmax3(mx[0], mx[1], mx[2]), tc::fmax3(mx[3], mx[4], mx[5]),
+                                         fmaxf(mx[6], mx[7]));
             // ---- running max, lazy rescale, P = 2^(s*sl - m) ------------------------------------
             const float tm = tmax * sl;
             bool resc = false;

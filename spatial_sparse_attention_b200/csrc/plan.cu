@@ -288,7 +288,9 @@ __global__ void k_fill_int4(int4* __restrict__ a, int64_t n, int4 v) {
 // neighbourhoods of its tokens, as ascending padded rows. Candidates are the tokens of the blocks
 // in the 3x3x3 block neighbourhood of every block the tile touches (r <= 8 keeps every window
 // inside it); a candidate is kept if it lies within Chebyshev distance r of some tile token.
-// kFill == false writes counts, kFill == true writes the rows at wt_off.
+// kFill == false writes counts, and the first spill_cap rows of every tile to spill[tile];
+// kFill == true writes the rows at wt_off for the tiles that held more than spill_cap rows (the
+// others are copied from spill by k_copy_union).
 template <bool kFill>
 __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t* __restrict__ qt_len,
                                const int32_t* __restrict__ qt_seq, const int32_t* __restrict__ perm,
@@ -298,7 +300,8 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
                                const int32_t* __restrict__ key2blk, const SeqInfo* __restrict__ seqs,
                                const int4* __restrict__ scoord, int r,
                                int32_t* __restrict__ wt_cnt, const int32_t* __restrict__ wt_off,
-                               int32_t* __restrict__ wt_keys) {
+                               int32_t* __restrict__ wt_keys, int32_t* __restrict__ spill, int spill_cap) {
+    if (kFill && wt_off[blockIdx.x + 1] - wt_off[blockIdx.x] <= spill_cap) return;   // copied instead
     constexpr int kCandCap = 4096;     // 27 neighbours x up to 128 distinct tile blocks, padded
     __shared__ int4 qc[kQTile];
     __shared__ int32_t cand[kCandCap];
@@ -510,7 +513,9 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
             before += u < wid ? wsum[u] : 0;
             all += wsum[u];
         }
-        if (kFill && keep) wt_keys[out_base + total + before + __popc(m & ((1u << lane) - 1))] = row;
+        const int at = total + before + __popc(m & ((1u << lane) - 1));
+        if (kFill && keep) wt_keys[out_base + at] = row;
+        if (!kFill && keep && at < spill_cap) spill[(int64_t)t * spill_cap + at] = row;
         total += all;
         __syncthreads();
     }
@@ -522,6 +527,15 @@ __global__ void k_window_union(const int32_t* __restrict__ qt_pos, const int32_t
 // a row opens a group when its group differs from the previous row's, and a group opens a run
 // when it does not follow the previous group. kFill == false writes the run and group counts;
 // kFill == true writes each run (first group, groups) at wr_off.
+// The window key unions that fit their tile's spill slot, from the slot to wt_keys.
+__global__ void k_copy_union(const int32_t* __restrict__ wt_off, const int32_t* __restrict__ spill,
+                             int spill_cap, int32_t* __restrict__ wt_keys) {
+    const int t = blockIdx.x;
+    const int32_t a = wt_off[t], n = wt_off[t + 1] - a;
+    if (n > spill_cap) return;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) wt_keys[a + i] = spill[(int64_t)t * spill_cap + i];
+}
+
 template <bool kFill>
 __global__ void k_window_runs(int64_t T, const int32_t* __restrict__ wt_off,
                               const int32_t* __restrict__ wt_keys, int32_t* __restrict__ wr_cnt,
@@ -745,11 +759,17 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         cudaMemcpyAsync(p->qt_len, qlen.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st) ||
         cudaMemcpyAsync(p->qt_seq, qseq.data(), sizeof(int32_t) * T, cudaMemcpyHostToDevice, st))
         return SSA_ERR_CUDA;
-    int32_t* wt_cnt;
+    int32_t *wt_cnt, *spill;
     SSA_ALLOC(wt_cnt, int32_t, T + 1);
+    // One pass finds each tile's window union; unions of up to spill_cap rows are kept in a slot
+    // per tile (at most 256 MB in all) and copied once their offsets are known, larger ones are
+    // found again by a second pass that skips every other tile.
+    int spill_cap = (int)std::min<int64_t>(4096, ((int64_t)64 << 20) / std::max<int64_t>(T, 1));
+    spill_cap = spill_cap >= 256 ? spill_cap & ~31 : 0;
+    SSA_ALLOC(spill, int32_t, (int64_t)T * std::max(spill_cap, 1));
     k_window_union<false><<<(unsigned)T, 128, 0, st>>>(
         p->qt_pos, p->qt_len, p->qt_seq, p->perm, p->tok_blk, p->coords, p->blk_coord, p->blk_poff,
-        p->blk_off, key2blk, p->d_seqs, p->scoord, r, wt_cnt, nullptr, nullptr);
+        p->blk_off, key2blk, p->d_seqs, p->scoord, r, wt_cnt, nullptr, nullptr, spill, spill_cap);
     note_launch();
     trace_step("plan neighbour lists + window union counts", st);
     scan_exclusive(wt_cnt, p->wt_off, T, tmp, st);
@@ -759,10 +779,11 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
         return SSA_ERR_CUDA;
     if (n_wkeys < 0) return SSA_ERR_UNSUPPORTED;
     SSA_ALLOC(p->wt_keys, int32_t, n_wkeys);
+    k_copy_union<<<(unsigned)T, 128, 0, st>>>(p->wt_off, spill, spill_cap, p->wt_keys);
     k_window_union<true><<<(unsigned)T, 128, 0, st>>>(
         p->qt_pos, p->qt_len, p->qt_seq, p->perm, p->tok_blk, p->coords, p->blk_coord, p->blk_poff,
-        p->blk_off, key2blk, p->d_seqs, p->scoord, r, nullptr, p->wt_off, p->wt_keys);
-    note_launch();
+        p->blk_off, key2blk, p->d_seqs, p->scoord, r, nullptr, p->wt_off, p->wt_keys, nullptr, spill_cap);
+    note_launch(2);
     trace_step("plan window unions", st);
     int32_t *wr_cnt, *wm_cnt;
     SSA_ALLOC(wr_cnt, int32_t, T + 1);
@@ -830,7 +851,7 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
 
     // scratch of the plan build is released now
     void* scratch[] = {tok_key, key_cnt, bidx, key2blk, blk_cnt, blk_pcnt, blk_fill,
-                       tmp, wt_cnt, wr_cnt, wm_cnt, ptok};
+                       tmp, wt_cnt, wr_cnt, wm_cnt, ptok, spill};
     for (void* ptr : scratch) {
         auto it = std::find(p->owned.begin(), p->owned.end(), ptr);
         if (it != p->owned.end()) {

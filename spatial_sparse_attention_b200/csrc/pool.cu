@@ -36,7 +36,7 @@ constexpr int kLanes = 4;
 constexpr int kMaxBlockTokens = 512;   // 8^3 cells
 
 template <typename T, bool kSorted>
-__global__ void __launch_bounds__(512) k_pool(const T* __restrict__ K, const T* __restrict__ V,
+__global__ void __launch_bounds__(512, 2) k_pool(const T* __restrict__ K, const T* __restrict__ V,
                                                const float* __restrict__ Wc,
                                                const int32_t* __restrict__ perm,
                                                const int32_t* __restrict__ blk_off,
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(512) k_pool(const T* __restrict__ K, const T* 
 constexpr int kProLanes = 2;
 
 template <typename T>
-__global__ void __launch_bounds__(512) k_pool_pro(const T* __restrict__ K, const T* __restrict__ V,
+__global__ void __launch_bounds__(512, 2) k_pool_pro(const T* __restrict__ K, const T* __restrict__ V,
                                                    const float* __restrict__ Wc,
                                                    const int32_t* __restrict__ perm,
                                                    const int32_t* __restrict__ blk_off,

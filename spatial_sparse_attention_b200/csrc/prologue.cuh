@@ -33,12 +33,12 @@ __device__ __forceinline__ int32_t axis_coord(int axis, int32_t x, int32_t y, in
     return axis == 0 ? x : (axis == 1 ? y : z);
 }
 
-// cos and sin of coordinate * freq: the angle is formed and reduced to [-pi, pi] in double, so
-// the result keeps fp32 accuracy at any coordinate of the supported grids.
+// cos and sin of coordinate * freq: the angle is formed in turns (freq / 2pi, exact enough in
+// double) and reduced to [-1/2, 1/2] of a turn in double, so the result keeps fp32 accuracy at any
+// coordinate of the supported grids.
 __device__ __forceinline__ void rope_cos_sin(int32_t coord, double freq, float& c, float& s) {
-    const double t = (double)coord * freq;
-    const double two_pi = 6.283185307179586476925286766559;
-    const float r = (float)(t - two_pi * rint(t / two_pi));
+    const double turns = (double)coord * (freq * 0.15915494309189533577);   // freq / (2 pi)
+    const float r = (float)(turns - rint(turns)) * 6.2831853071795864769f;
     __sincosf(r, &s, &c);
 }
 

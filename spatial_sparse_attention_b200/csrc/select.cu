@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_ssa_select(const __grid_constan
             float glo = INFINITY, tmax = -INFINITY;
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-                const float gq = fmaxf(fmaxf(s[4 * q], s[4 * q + 1]), fmaxf(s[4 * q + 2], s[4 * q + 3]));
+                const float gq = fmaxf(tc::fmax3(s[4 * q], s[4 * q + 1], s[4 * q + 2]), s[4 * q + 3]);
                 glo = fminf(glo, gq);
                 tmax = fmaxf(tmax, gq);
             }

@@ -90,6 +90,11 @@ def lib():
         L.oracle_compress_conv.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                            ctypes.c_int32, c_vp, c_vp, c_f32p, c_i32p, c_i32p,
                                            c_i32p, c_f64p, c_f64p]
+        L.oracle_select_subblock.restype = ctypes.c_int
+        L.oracle_select_subblock.argtypes = [
+            ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_vp, c_vp, c_vp,
+            c_f32p, c_f32p, c_i32p, ctypes.c_int32, c_i32p, c_i32p, c_i32p, c_i32p,
+            ctypes.c_int64, ctypes.c_int64, c_i64p, c_i32p, c_f64p]
         L.oracle_rope_split.restype = None
         L.oracle_rope_split.argtypes = [ctypes.c_int32, c_i32p, c_i32p, c_i32p]
         L.oracle_round_array.restype = None
@@ -287,7 +292,7 @@ def center_only_conv(Wc) -> np.ndarray:
 def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None,
             block: int = 8, round_compressed: bool = False, sel_in=None,
             want_z: bool = False, branches: bool = True, prologue=None, conv=None,
-            gate=None) -> Dict[str, object]:
+            gate=None, share=None) -> Dict[str, object]:
     """Oracle forward for the query rows `rows` (global indices; None = all tokens).
 
     Returns out, o_cmp, o_sel, o_win ([R, H, D] float64), sel ([R, H, k] int32 global block
@@ -299,9 +304,12 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
     (the prologue's results are tensors of that type, as any layer's are). conv ([27, D, D]
     fp32) compresses blocks by the sparse 3D convolution over the block grid instead of the
     block mean times Wc; gate = dict(w=[D, 3], b=[3]) predicts the gates from each head's query
-    (sigmoid(q . w + b)) instead of reading `gates`.
+    (sigmoid(q . w + b)) instead of reading `gates`. share="subblock" selects the blocks once per
+    4x4x4 sub-block of cells from the summed compressed-attention weights of its queries
+    (select_subblock) instead of once per query.
     """
-    if prologue is not None:
+    if share not in (None, "subblock"):
+        raise ValueError(f"unknown selection sharing {share!r}")
         pr = dict(prologue)
         kw = dict(eps=pr.get("eps", 1e-6), theta=pr.get("theta", 10000.0), round_to_input=True)
         Q = qk_prologue(Q, coords, pr["q_gamma"], **kw)
@@ -309,6 +317,11 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
         V = _exact_f64(V)
         return forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk, r, rows=rows, block=block,
                        round_compressed=round_compressed, sel_in=sel_in, want_z=want_z,
+                       branches=branches, conv=conv, gate=gate, share=share)
+    if share == "subblock" and sel_in is None:
+        sh = select_subblock(coords, cu_seqlens, Q, K, V, Wc, topk, rows=rows, block=block, conv=conv)
+        return forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk, r, rows=rows, block=block,
+                       round_compressed=round_compressed, sel_in=sh["sel"], want_z=want_z,
                        branches=branches, conv=conv, gate=gate)
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
@@ -395,6 +408,62 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
     if want_z:
         res["z"] = zs
     res["rows"] = rows
+    return res
+
+
+def select_subblock(coords, cu_seqlens, Q, K, V, Wc, topk: int, rows=None, block: int = 8,
+                    conv=None, want_score: bool = False) -> Dict[str, object]:
+    """Selection shared by the queries of each 4x4x4 sub-block of cells (oracle_select_subblock):
+    the own block plus the top (k-1) other blocks by the sum over the sub-block's queries of
+    their compressed-attention weights. Q and K are taken as given (apply qk_prologue first for
+    the prologue). Returns sel ([R, H, k] global block indices, -1 = empty slot) for the rows
+    (global indices; None = all tokens) and, if want_score, score: list of [H, Mb_seq] summed
+    weights of each row's sub-block."""
+    if block != 8:
+        raise ValueError("sub-blocks of 4 cells are defined for blocks of 8 cells")
+    coords = np.ascontiguousarray(coords, dtype=np.int32)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    q, dt = _raw(Q)
+    k, _ = _raw(K)
+    v, _ = _raw(V)
+    w = _f32(Wc)
+    N, H, D = q.shape
+    wconv = None
+    if conv is not None:
+        wconv = np.ascontiguousarray(_f32(conv), dtype=np.float32).reshape(27, D, D)
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    R = len(rows)
+    out_sel = np.full((R, H, topk), -1, np.int32)
+    scores = [None] * R
+    seq_of = np.searchsorted(cu, rows, side="right") - 1
+    blk_base = 0
+    L = lib()
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        perm, tok_blk, blk_off, blk_coord = partition(coords[lo:hi], block)
+        mb = len(blk_off) - 1
+        pick = np.nonzero(seq_of == s)[0]
+        if len(pick) and mb > 0:
+            local = np.ascontiguousarray(rows[pick] - lo)
+            sel = np.zeros((len(pick), H, topk), np.int32)
+            sc = np.zeros((len(pick), H, mb)) if want_score else None
+            rc = L.oracle_select_subblock(
+                hi - lo, H, D, dt, q[lo:hi].ctypes.data, k[lo:hi].ctypes.data, v[lo:hi].ctypes.data,
+                _ptr(w, c_f32p), _ptr(wconv, c_f32p),
+                _ptr(np.ascontiguousarray(blk_coord, dtype=np.int32), c_i32p), topk,
+                _ptr(np.ascontiguousarray(coords[lo:hi]), c_i32p), _ptr(perm, c_i32p),
+                _ptr(tok_blk, c_i32p), _ptr(blk_off, c_i32p), mb, len(local), _ptr(local, c_i64p),
+                _ptr(sel, c_i32p), _ptr(sc, c_f64p))
+            if rc != 0:
+                raise RuntimeError("oracle_select_subblock failed")
+            out_sel[pick] = np.where(sel >= 0, sel + blk_base, -1)
+            if want_score:
+                for t, p in enumerate(pick):
+                    scores[p] = sc[t].copy()
+        blk_base += mb
+    res = {"sel": out_sel, "rows": rows}
+    if want_score:
+        res["score"] = scores
     return res
 
 

@@ -454,6 +454,118 @@ static void select_blocks(int64_t mb, const double* z, int32_t own, int32_t k, i
 }
 
 /*
+ * 4b. Selection shared by the queries of one 4x4x4 sub-block of cells.
+ * The pages choose the important blocks from the compression module's attention scores and
+ * leave open whose scores (Direct3D-S2 summary page, "Technical principles", SSA item). This
+ * variant pools them over a sub-block G = the tokens of the sequence with the same
+ * (floor(x/4), floor(y/4), floor(z/4)); as 4 divides 8, G lies in one block, its members' own
+ * block. Per head:
+ *   score_G(b) = sum_{i in G} p_i(b),  p_i = softmax_b(scale * q_i . Kc_b)  (step 3's weights);
+ *   every member of G takes S_G = {own} + the top (k-1) other blocks by score_G (descending,
+ *   equal scores -> lower block index), ranked by select_blocks.
+ * coords: [n, 3] of the sequence (non-negative). Compression as the forward: Kc from Wconv
+ * (section 2b) when non-NULL, else mean . Wc, unrounded. Outputs for the `n_rows` rows (local
+ * indices in `rows`; NULL = all n): sel [n_rows, H, k] local block indices (-1 = empty slot),
+ * and score (may be NULL) [n_rows, H, mb] = score_G of the row's sub-block.
+ */
+static int32_t subblock_of(const int32_t* c) {
+    return (((c[0] >> 2) & 1) << 2) | (((c[1] >> 2) & 1) << 1) | ((c[2] >> 2) & 1);
+}
+
+int oracle_select_subblock(int64_t n, int32_t H, int32_t D, int32_t dtype, const void* Q,
+                           const void* K, const void* V, const float* Wc, const float* Wconv,
+                           const int32_t* blk_coord, int32_t topk, const int32_t* coords,
+                           const int32_t* perm, const int32_t* tok_blk, const int32_t* blk_off,
+                           int64_t mb, int64_t n_rows, const int64_t* rows, int32_t* sel,
+                           double* score) {
+    if (topk < 1 || D < 1 || H < 1 || mb < 1) return -1;
+    if (!rows) n_rows = n;
+    const int64_t ng = mb * 8; /* group id = 8 * block + sub-block of the block */
+    int64_t* g_off = (int64_t*)calloc((size_t)(ng + 1), sizeof(int64_t));
+    int64_t* g_mem = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n + 1));
+    int64_t* g_slot = (int64_t*)malloc(sizeof(int64_t) * (size_t)(ng + 1)); /* needed group -> slot */
+    double* Kc = (double*)malloc(sizeof(double) * (size_t)(mb * H * D + 1));
+    double* Vc = (double*)malloc(sizeof(double) * (size_t)(mb * H * D + 1));
+    if (!g_off || !g_mem || !g_slot || !Kc || !Vc) return -1;
+    if (Wconv)
+        compress_conv(mb, H, D, dtype, K, V, Wconv, perm, blk_off, blk_coord, Kc, Vc);
+    else
+        compress(mb, H, D, dtype, K, V, Wc, perm, blk_off, 0, Kc, Vc);
+    /* members of every group, in ascending token index */
+    for (int64_t i = 0; i < n; ++i) g_off[8 * (int64_t)tok_blk[i] + subblock_of(&coords[3 * i]) + 1] += 1;
+    for (int64_t g = 0; g < ng; ++g) g_off[g + 1] += g_off[g];
+    {
+        int64_t* fill = (int64_t*)malloc(sizeof(int64_t) * (size_t)(ng + 1));
+        if (!fill) return -1;
+        memcpy(fill, g_off, sizeof(int64_t) * (size_t)ng);
+        for (int64_t i = 0; i < n; ++i) g_mem[fill[8 * (int64_t)tok_blk[i] + subblock_of(&coords[3 * i])]++] = i;
+        free(fill);
+    }
+    /* the groups the requested rows belong to */
+    for (int64_t g = 0; g < ng; ++g) g_slot[g] = -1;
+    int64_t n_need = 0;
+    for (int64_t ri = 0; ri < n_rows; ++ri) {
+        int64_t i = rows ? rows[ri] : ri;
+        int64_t g = 8 * (int64_t)tok_blk[i] + subblock_of(&coords[3 * i]);
+        if (g_slot[g] < 0) g_slot[g] = n_need++;
+    }
+    int64_t* need = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_need + 1));
+    int32_t* gsel = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n_need * H * topk + 1));
+    double* gscore = score ? (double*)malloc(sizeof(double) * (size_t)(n_need * H * mb + 1)) : NULL;
+    if (!need || !gsel || (score && !gscore)) return -1;
+    for (int64_t g = 0; g < ng; ++g)
+        if (g_slot[g] >= 0) need[g_slot[g]] = g;
+    const double scale = 1.0 / sqrt((double)D);
+
+#pragma omp parallel
+    {
+        double* q = (double*)malloc(sizeof(double) * (size_t)D);
+        double* z = (double*)malloc(sizeof(double) * (size_t)mb);
+        double* acc = (double*)malloc(sizeof(double) * (size_t)mb);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t gh = 0; gh < n_need * H; ++gh) {
+            const int64_t slot = gh / H, g = need[slot];
+            const int32_t h = (int32_t)(gh % H);
+            for (int64_t b = 0; b < mb; ++b) acc[b] = 0.0;
+            for (int64_t t = g_off[g]; t < g_off[g + 1]; ++t) {
+                const int64_t i = g_mem[t];
+                for (int32_t d = 0; d < D; ++d) q[d] = load_elem(Q, dtype, (i * H + h) * D + d);
+                /* this member's compressed-attention weights, as in step 3 */
+                double m = -INFINITY;
+                for (int64_t b = 0; b < mb; ++b) {
+                    double t2 = 0.0;
+                    for (int32_t d = 0; d < D; ++d) t2 += q[d] * Kc[(b * H + h) * D + d];
+                    z[b] = scale * t2;
+                    if (z[b] > m) m = z[b];
+                }
+                double l = 0.0;
+                for (int64_t b = 0; b < mb; ++b) {
+                    z[b] = exp(z[b] - m);
+                    l += z[b];
+                }
+                for (int64_t b = 0; b < mb; ++b) acc[b] += z[b] / l;
+            }
+            select_blocks(mb, acc, (int32_t)(g / 8), topk, &gsel[gh * topk]);
+            if (gscore)
+                for (int64_t b = 0; b < mb; ++b) gscore[gh * mb + b] = acc[b];
+        }
+        free(q); free(z); free(acc);
+    }
+    for (int64_t ri = 0; ri < n_rows; ++ri) {
+        int64_t i = rows ? rows[ri] : ri;
+        int64_t slot = g_slot[8 * (int64_t)tok_blk[i] + subblock_of(&coords[3 * i])];
+        for (int32_t h = 0; h < H; ++h) {
+            for (int32_t s2 = 0; s2 < topk; ++s2)
+                sel[(ri * H + h) * topk + s2] = gsel[(slot * H + h) * topk + s2];
+            if (score)
+                for (int64_t b = 0; b < mb; ++b) score[(ri * H + h) * mb + b] = gscore[(slot * H + h) * mb + b];
+        }
+    }
+    free(g_off); free(g_mem); free(g_slot); free(need); free(gsel); free(gscore); free(Kc); free(Vc);
+    return 0;
+}
+
+/*
  * Forward pass of one sequence for `n_rows` query rows (local indices in `rows`; NULL = all n).
  * Q, K, V: [n, H, D] of `dtype`; gates: [n, H, 3] (cmp, sel, win); Wc: [D, D].
  * Plan arrays come from oracle_partition / oracle_window of the same sequence.

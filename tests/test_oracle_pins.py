@@ -801,3 +801,93 @@ def test_conv_forward_is_invariant_under_block_translation():
     b = run(c + np.array([16, 8, 24], np.int32), q, k, v, g, Wc, 4, 2, conv=W)
     assert np.array_equal(a["sel"], b["sel"])
     np.testing.assert_allclose(b["out"], a["out"], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# selection shared by the queries of a 4x4x4 sub-block (the pages leave open whose compression
+# scores choose the blocks; this variant sums them over a sub-block's queries)
+# ---------------------------------------------------------------------------------------------
+
+def test_subblock_selection_with_one_query_per_subblock_is_the_per_query_selection():
+    """Cells on a lattice of spacing 4: every 4x4x4 sub-block holds one query, and the sum of
+    its weights ranks blocks as that query's logits do (softmax is increasing)."""
+    rng = np.random.default_rng(21)
+    lat = np.stack(np.meshgrid(*(np.arange(0, 48, 4),) * 3, indexing="ij"), -1).reshape(-1, 3)
+    c = lat[np.sort(rng.choice(len(lat), 700, replace=False))].astype(np.int32)
+    N, H, D = len(c), 2, 16
+    q, k, v = (_rand((N, H, D), 22 + i) for i in range(3))
+    g = _gates(N, H, None, 25)
+    Wc = _rand((D, D), 26) / np.sqrt(D)
+    a = run(c, q, k, v, g, Wc, 5, 2)
+    b = run(c, q, k, v, g, Wc, 5, 2, share="subblock")
+    np.testing.assert_array_equal(a["sel"], b["sel"])
+    np.testing.assert_allclose(b["out"], a["out"], rtol=0, atol=1e-13)
+
+
+def test_subblock_selection_matches_brute_force_on_tiny_input():
+    """numpy restatement: blocks by np.unique of the 8-cell keys, Kc = block mean . Wc, each
+    query's softmax, sums per (block, 4-cell sub-block) by np.add.at, ranking by lexsort."""
+    c, _ = _tiny_coords()
+    N, H, D, topk = len(c), 2, 8, 4
+    q, k, v = (_rand((N, H, D), 31 + i) for i in range(3))
+    Wc = (_rand((D, D), 34) / np.sqrt(D)).astype(np.float32)   # the oracle takes Wc in fp32
+    ours = oracle.select_subblock(c, [0, N], q, k, v, Wc, topk, want_score=True)
+    ukeys, tok_blk = np.unique(c // 8, axis=0, return_inverse=True)
+    tok_blk = tok_blk.reshape(-1)
+    mb = len(ukeys)
+    cnt = np.bincount(tok_blk, minlength=mb)
+    sub = ((c[:, 0] >> 2) & 1) * 4 + ((c[:, 1] >> 2) & 1) * 2 + ((c[:, 2] >> 2) & 1)
+    grp = tok_blk * 8 + sub
+    for h in range(H):
+        kbar = np.zeros((mb, D))
+        np.add.at(kbar, tok_blk, k[:, h])
+        kc = (kbar / cnt[:, None]) @ Wc.astype(np.float64)
+        z = q[:, h] @ kc.T / np.sqrt(D)
+        p = np.exp(z - z.max(1, keepdims=True))
+        p /= p.sum(1, keepdims=True)
+        score = np.zeros((mb * 8, mb))
+        np.add.at(score, grp, p)
+        for i in range(N):
+            s = score[grp[i]]
+            np.testing.assert_allclose(ours["score"][i][h], s, rtol=1e-12, atol=1e-15)
+            own = tok_blk[i]
+            order = [b for b in np.lexsort((np.arange(mb), -s)) if b != own][:topk - 1]
+            want = [own] + order + [-1] * (topk - 1 - len(order))
+            assert list(ours["sel"][i, h]) == want, (i, h)
+
+
+def test_subblock_selection_sums_weights_over_the_subblock():
+    """Planted: three queries of one sub-block each rank another block first (A or C), but B is a
+    close second for all three, so the summed weights pick B for every one of them; a query of a
+    neighbouring sub-block of the same block keeps its own choice. Per-query selection differs."""
+    D = 4
+    c = np.array([[0, 0, 0], [1, 0, 0], [2, 0, 0], [5, 0, 0],    # own block (0,0,0)
+                  [8, 0, 0], [16, 0, 0], [24, 0, 0]], np.int32)   # blocks A, B, C: one cell each
+    alpha = 4.0
+    k = np.zeros((7, 1, D))
+    k[4, 0, 0] = k[5, 0, 1] = k[6, 0, 2] = alpha                 # Kc_A, Kc_B, Kc_C with Wc = I
+    want_z = np.array([[5.0, 4.9, 0.0], [0.0, 4.0, 4.1], [0.0, 4.0, 4.1], [6.0, 0.0, 0.0]])
+    q = np.zeros((7, 1, D))
+    q[:4, 0, :3] = want_z * np.sqrt(D) / alpha                    # z_b = q . Kc_b / sqrt(D)
+    v = _rand((7, 1, D), 40)
+    g = _gates(7, 1, [0.0, 1.0, 0.0])
+    Wc = np.eye(D)
+    shared = run(c, q, k, v, g, Wc, 2, 1, share="subblock", rows=np.arange(4))
+    alone = run(c, q, k, v, g, Wc, 2, 1, rows=np.arange(4))
+    assert shared["sel"][:, 0].tolist() == [[0, 2], [0, 2], [0, 2], [0, 1]]
+    assert alone["sel"][:, 0].tolist() == [[0, 1], [0, 3], [0, 3], [0, 1]]
+
+
+def test_subblock_selection_is_shared_by_all_queries_of_a_subblock():
+    c, _ = _tiny_coords()
+    N, H, D = len(c), 2, 8
+    q, k, v = (_rand((N, H, D), 51 + i) for i in range(3))
+    Wc = _rand((D, D), 54) / np.sqrt(D)
+    sel = oracle.select_subblock(c, [0, N], q, k, v, Wc, 4)["sel"]
+    key = np.concatenate([c // 4, np.zeros((N, 1), np.int32)], 1)
+    _, grp = np.unique(key, axis=0, return_inverse=True)
+    grp = grp.reshape(-1)
+    for gi in np.unique(grp):
+        m = np.nonzero(grp == gi)[0]
+        assert (sel[m] == sel[m[0]]).all()
+    assert len(np.unique(grp)) < N   # the tiny shell has sub-blocks with several cells

@@ -310,6 +310,7 @@ def forward(coords, cu_seqlens, Q, K, V, gates, Wc, topk: int, r: int, rows=None
     """
     if share not in (None, "subblock"):
         raise ValueError(f"unknown selection sharing {share!r}")
+    if prologue is not None:
         pr = dict(prologue)
         kw = dict(eps=pr.get("eps", 1e-6), theta=pr.get("theta", 10000.0), round_to_input=True)
         Q = qk_prologue(Q, coords, pr["q_gamma"], **kw)

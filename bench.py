@@ -60,8 +60,8 @@ def config_of(args):
 # capture of the kernel (dram__bytes_read.sum + dram__bytes_write.sum of the 4-head cut, divided
 # by 4; the launch's traffic grows in proportion to the heads). Valid only for the kernel sources
 # the capture was taken with.
-KERNEL_TRAFFIC = {"sources_sha256": "0e28bab05d86fcb8e98190cc10159222927ac684dd26f4f99db12c35d2f0d10e",
-                  "config": "pass3", "bytes_per_head": 632926208.0 / 4}
+KERNEL_TRAFFIC = {"sources_sha256": "c622e7fa5a59592e7904318c205eba5bb9542a596bed6933c1a00d409a63683f",
+                  "config": "pass3", "bytes_per_head": (441356544.0 + 226973184.0) / 4}
 KERNEL_SOURCES = ("attn_fwd.cu", "attn_common.cuh", "tc.cuh")
 
 
@@ -379,8 +379,9 @@ def _cores():
 
 def measure_variants(plan, dev, cfg, peak_hbm, steps=10, warmup=3):
     """The forward with the options of ssa_forward_ex on the same workload: the attention prologue
-    (RMS normalisation and rotary embedding of q and k), and the compression by sparse 3D
-    convolution over the block grid with gates predicted from the queries. Per variant: ms per
+    (RMS normalisation and rotary embedding of q and k), the compression by sparse 3D convolution
+    over the block grid with gates predicted from the queries, and the selection shared by each
+    4x4x4 sub-block (a different method: fewer distinct blocks per query tile). Per variant: ms per
     forward (CUDA events) and the per-kernel breakdown; for the prologue's pooling kernel the HBM
     rate of its bytes, for the convolution its fp32 FMA rate."""
     import torch
@@ -394,6 +395,7 @@ def measure_variants(plan, dev, cfg, peak_hbm, steps=10, warmup=3):
     variants = {
         "prologue": dict(q_gamma=w["q_gamma"], k_gamma=w["k_gamma"], rope_theta=10000.0, eps=1e-6),
         "conv_and_predicted_gates": dict(conv_w=w["conv_w"], gate_w=w["gate_w"], gate_b=w["gate_b"]),
+        "shared_selection": dict(share_selection=True),
     }
     out = torch.empty_like(dev["Q"])
     res = {}
@@ -428,7 +430,7 @@ def measure_variants(plan, dev, cfg, peak_hbm, steps=10, warmup=3):
             if pm:
                 r["pool_hbm"] = {"bytes": byts, "achieved_gbs": byts / (pm * 1e-3) / 1e9,
                                  "frac_of_measured_hbm": byts / (pm * 1e-3) / 1e9 / peak_hbm}
-        else:
+        elif name == "conv_and_predicted_gates":
             cm = r["breakdown_ms"].get("conv")
             if cm:
                 # FMAs: K and V, every head, D x D per (block, present neighbour)

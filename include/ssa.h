@@ -219,6 +219,16 @@ SSA_API ssa_status_t ssa_forward_prologue(ssa_plan_t plan, const void* q, const 
  *       branches are aggregated with predicted gating scores): g = sigmoid(q . gate_w + gate_b) per
  *       token and head, q being the query as the attention sees it (after the prologue, in the
  *       input type), order (cmp, sel, win). Both set, or neither.
+ *   select_share: 0 = every query selects its own blocks (the plain method); 1 = the queries of
+ *       each 4x4x4 sub-block of cells (same (floor(x/4), floor(y/4), floor(z/4)) in one sequence;
+ *       it lies in one 8x8x8 block) share one selection: their own block plus the top (k-1)
+ *       other blocks by the sum over the sub-block's queries of their compressed-attention
+ *       weights (softmax of the compressed logits), equal sums to the lower block index. The
+ *       pages choose the blocks from the compression module's attention scores (same item)
+ *       without saying whose; this pools them over neighbouring queries. bf16 / fp16 only
+ *       (SSA_ERR_UNSUPPORTED for fp32). The first call builds the plan's sub-block order and
+ *       its selection tiles (whole sub-blocks of a sequence, at most 128 rows and 32 sub-blocks
+ *       each, packed on the host: the call waits for the stream twice).
  */
 typedef struct {
     const float* q_gamma;
@@ -228,6 +238,7 @@ typedef struct {
     const float* conv_w;
     const float* gate_w;
     const float* gate_b;
+    int32_t select_share;
 } ssa_options_t;
 
 /*

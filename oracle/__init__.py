@@ -425,8 +425,10 @@ def select_subblock(coords, cu_seqlens, Q, K, V, Wc, topk: int, rows=None, block
     coords = np.ascontiguousarray(coords, dtype=np.int32)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     q, dt = _raw(Q)
-    k, _ = _raw(K)
-    v, _ = _raw(V)
+    k, dk = _raw(K)
+    v, dv = _raw(V)
+    if dk != dt or dv != dt:
+        raise ValueError("Q, K and V must have one storage type")
     w = _f32(Wc)
     N, H, D = q.shape
     wconv = None

@@ -66,7 +66,8 @@ _SIGS = {
 class Options(ctypes.Structure):
     """ssa_options_t (include/ssa.h): the optional parts of ssa_forward_ex."""
     _fields_ = [("q_gamma", _vp), ("k_gamma", _vp), ("rope_theta", ctypes.c_float),
-                ("rms_eps", ctypes.c_float), ("conv_w", _vp), ("gate_w", _vp), ("gate_b", _vp)]
+                ("rms_eps", ctypes.c_float), ("conv_w", _vp), ("gate_w", _vp), ("gate_b", _vp),
+                ("select_share", ctypes.c_int32)]
 
 
 def _load():
@@ -292,11 +293,13 @@ class Plan:
 
     def forward_ex(self, q, k, v, gates, wc, topk: int, q_gamma=None, k_gamma=None,
                    rope_theta: float = 10000.0, eps: float = 1e-6, conv_w=None, gate_w=None,
-                   gate_b=None, out: Optional[torch.Tensor] = None, return_sel: bool = False):
+                   gate_b=None, out: Optional[torch.Tensor] = None, return_sel: bool = False,
+                   share_selection: bool = False):
         """ssa_forward_ex: the prologue (q_gamma, k_gamma [D]), the compression by sparse 3D
         convolution over the block grid (conv_w [27, D, D]) and gates predicted from the queries
         (gate_w [D, 3], gate_b [3]), each optional (fp32 CUDA tensors). gates / wc may be None when
-        predicted / replaced by the convolution."""
+        predicted / replaced by the convolution. share_selection: one selection per 4x4x4
+        sub-block of cells, from the summed compressed-attention weights of its queries."""
         dt = q.dtype
         for t in (q, k, v):
             _dev(t, dt)
@@ -307,7 +310,7 @@ class Plan:
             if t is not None:
                 _dev(t, torch.float32)
         opt = Options(_ptr(q_gamma), _ptr(k_gamma), float(rope_theta), float(eps), _ptr(conv_w),
-                      _ptr(gate_w), _ptr(gate_b))
+                      _ptr(gate_w), _ptr(gate_b), int(bool(share_selection)))
         out = torch.empty_like(q) if out is None else _dev(out, dt)
         sel = torch.empty(self.N, H, topk, dtype=torch.int32, device=q.device) if return_sel else None
         _check(lib.ssa_forward_ex(self._h, q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(gates),

@@ -295,6 +295,7 @@ struct Options {
     const float* conv_w = nullptr;   // [27, D, D]: compression by sparse 3D convolution
     const float* gate_w = nullptr;   // [D, 3] and [3]: gates predicted from the queries
     const float* gate_b = nullptr;
+    bool share = false;              // one selection per 4x4x4 sub-block (16-bit types)
 };
 
 // A workspace buffer of `bytes` allocated on first use (kept with the workspace).
@@ -355,9 +356,13 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
         if ((rc = ensure_neighbours(p, st)) != SSA_OK) return rc;
         launch_forward_simt(p, w, q, k, v, gates, out, bo, st);
     } else {
-        if ((rc = launch_select_tc(p, w, q, fused, opt.gate_w, opt.gate_b, opt.gate_w ? w.gates : nullptr, st)) !=
-            SSA_OK)
-            return rc;
+        if (opt.share) {
+            if ((rc = ensure_subblock_tiles(p, st)) != SSA_OK) return rc;
+            rc = launch_select_shared(p, w, q, fused, opt.gate_w, opt.gate_b, opt.gate_w ? w.gates : nullptr, st);
+        } else {
+            rc = launch_select_tc(p, w, q, fused, opt.gate_w, opt.gate_b, opt.gate_w ? w.gates : nullptr, st);
+        }
+        if (rc != SSA_OK) return rc;
         trace_step("select", st);
         if ((rc = launch_forward_tc(p, w, q, gates, out, bo, fused, st)) != SSA_OK) return rc;
     }
@@ -534,6 +539,9 @@ ssa_status_t ssa_forward_ex(ssa_plan_t p, const void* q, const void* k, const vo
         opt.conv_w = o.conv_w;
         opt.gate_w = o.gate_w;
         opt.gate_b = o.gate_b;
+        if (o.select_share != 0 && o.select_share != 1) return SSA_ERR_INVALID_ARG;
+        opt.share = o.select_share == 1;
+        if (opt.share && dtype == SSA_F32) return SSA_ERR_UNSUPPORTED;
     }
     // the gates input is not read when they are predicted, nor wc with a convolution compression
     static const float kUnused = 0.0f;

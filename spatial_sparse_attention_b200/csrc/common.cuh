@@ -122,6 +122,11 @@ struct Plan {
     uint64_t hmask = 0;
     int32_t nbr_cap = 32;        // per-warp sort buffer of the neighbour-list kernel
     int32_t* blk_nbr = nullptr;  // [Mb][27] block at offset o of every block (-1 = none), first use
+    int32_t* sb_rows = nullptr;  // [N] sorted positions, each block's tokens in 4x4x4 sub-block
+                                 //      order (then ascending position); first use of shared selection
+    int4* sst = nullptr;         // [n_sst] selection tiles of whole sub-blocks of one sequence:
+                                 //      (first index into sb_rows, rows <= 128, sequence, sub-blocks <= 32)
+    int64_t n_sst = 0;
     int32_t* qt_pos = nullptr;   // [n_qtiles] first sorted position of each query tile
     int32_t* qt_len = nullptr;   // [n_qtiles]
     int32_t* qt_seq = nullptr;   // [n_qtiles]
@@ -216,6 +221,10 @@ void launch_forward_simt(const Plan* p, const Workspace& w, const void* q, const
 // token order (the prologue, when on, is applied to each query tile after it is loaded)
 // With gate_w non-null it also writes gates_out [N, H, 3] = sigmoid(q . gate_w + gate_b), q being the
 // query as the attention sees it (after the prologue).
+ssa_status_t ensure_subblock_tiles(Plan* p, cudaStream_t st);
+ssa_status_t launch_select_shared(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
+                                  const float* gate_w, const float* gate_b, float* gates_out,
+                                  cudaStream_t st);
 ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
                               const float* gate_w, const float* gate_b, float* gates_out, cudaStream_t s);
 

@@ -739,6 +739,9 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
     p->nbr_cap = cap;
     p->nbr_idx = nullptr;
     p->blk_nbr = nullptr;   // block neighbour table (convolution compression), built on first use
+    p->sb_rows = nullptr;   // sub-block order and selection tiles (shared selection), first use
+    p->sst = nullptr;
+    p->n_sst = 0;
 
     // ---- query tiles and their window key unions (tensor-core window kernel) ----------------------
     std::vector<int32_t> qpos, qlen, qseq;
@@ -858,6 +861,104 @@ ssa_status_t build_plan(Plan* p, const int32_t* coords, cudaStream_t st) {
             p->release(ptr, st, p->alloc_ctx);
             p->owned.erase(it);
         }
+    }
+    return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+// ---- sub-block order and selection tiles (selection shared by a 4x4x4 sub-block) ----------------
+// One warp per block. A token's sub-block within its block is the 3-bit index of
+// ((x >> 2) & 1, (y >> 2) & 1, (z >> 2) & 1) (4 divides 8, so a sub-block never leaves its block).
+// Writes the block's sorted positions grouped by sub-block (stable) to sb_rows, and the tokens of
+// each of its 8 sub-blocks to sbc[8 b + s].
+__global__ void k_subblock_order(const int32_t* __restrict__ perm, const int32_t* __restrict__ coords,
+                                 const int32_t* __restrict__ blk_off, int32_t* __restrict__ sb_rows,
+                                 int32_t* __restrict__ sbc) {
+    const int b = blockIdx.x, lane = threadIdx.x;
+    const int32_t a0 = blk_off[b], n = blk_off[b + 1] - a0;
+    auto sub_of = [&](int32_t pos) {
+        const int32_t* c = coords + 3 * (int64_t)perm[pos];
+        return (((c[0] >> 2) & 1) << 2) | (((c[1] >> 2) & 1) << 1) | ((c[2] >> 2) & 1);
+    };
+    int mine = 0;   // lane s < 8: tokens of sub-block s
+    for (int i = 0; i < n; i += 32) {
+        const int s = i + lane < n ? sub_of(a0 + i + lane) : -1;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const unsigned bal = __ballot_sync(0xffffffffu, s == q);
+            if (lane == q) mine += __popc(bal);
+        }
+    }
+    int base = mine;   // exclusive prefix over lanes 0..7
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, base, d);
+        if (lane >= d) base += t;
+    }
+    base -= mine;
+    if (lane < 8) sbc[8 * (int64_t)b + lane] = mine;
+    for (int i = 0; i < n; i += 32) {
+        const int s = i + lane < n ? sub_of(a0 + i + lane) : -1;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const unsigned bal = __ballot_sync(0xffffffffu, s == q);
+            const int bq = __shfl_sync(0xffffffffu, base, q);
+            if (s == q) sb_rows[a0 + bq + __popc(bal & ((1u << lane) - 1u))] = a0 + i + lane;
+            if (lane == q) base += __popc(bal);
+        }
+    }
+}
+
+ssa_status_t ensure_subblock_tiles(Plan* p, cudaStream_t st) {
+    if (p->sst) return SSA_OK;
+    if (p->Mb == 0) {
+        SSA_ALLOC(p->sst, int4, 1);
+        p->n_sst = 0;
+        return SSA_OK;
+    }
+    int32_t* sbc;
+    SSA_ALLOC(p->sb_rows, int32_t, p->N);
+    SSA_ALLOC(sbc, int32_t, 8 * p->Mb);
+    k_subblock_order<<<(unsigned)p->Mb, 32, 0, st>>>(p->perm, p->coords, p->blk_off, p->sb_rows, sbc);
+    note_launch();
+    std::vector<int32_t> cnt((size_t)(8 * p->Mb)), off((size_t)(p->Mb + 1));
+    if (cudaMemcpyAsync(cnt.data(), sbc, sizeof(int32_t) * cnt.size(), cudaMemcpyDeviceToHost, st) ||
+        cudaMemcpyAsync(off.data(), p->blk_off, sizeof(int32_t) * off.size(), cudaMemcpyDeviceToHost, st) ||
+        cudaStreamSynchronize(st))
+        return SSA_ERR_CUDA;
+    // Tiles take the sub-blocks of a sequence in order (blocks in order, sub-blocks within), a new
+    // tile whenever the next sub-block would pass 128 rows or 32 sub-blocks (a sub-block has at
+    // most 64 rows). Tile = (first index into sb_rows, rows, sequence, sub-blocks).
+    std::vector<int4> tiles;
+    for (int32_t s = 0; s < p->B; ++s) {
+        int32_t first = 0, rows = 0, nsub = 0;
+        for (int64_t b = p->seq_blk[s]; b < p->seq_blk[s + 1]; ++b) {
+            int32_t at = off[b];
+            for (int q = 0; q < 8; ++q) {
+                const int32_t c = cnt[8 * b + q];
+                if (c == 0) continue;
+                if (rows > 0 && (rows + c > 128 || nsub == 32)) {
+                    tiles.push_back(make_int4(first, rows, s, nsub));
+                    rows = 0;
+                    nsub = 0;
+                }
+                if (rows == 0) first = at;
+                rows += c;
+                nsub += 1;
+                at += c;
+            }
+        }
+        if (rows > 0) tiles.push_back(make_int4(first, rows, s, nsub));
+    }
+    p->n_sst = (int64_t)tiles.size();
+    SSA_ALLOC(p->sst, int4, std::max<int64_t>(p->n_sst, 1));
+    if (p->n_sst > 0 &&
+        (cudaMemcpyAsync(p->sst, tiles.data(), sizeof(int4) * tiles.size(), cudaMemcpyHostToDevice, st) ||
+         cudaStreamSynchronize(st)))
+        return SSA_ERR_CUDA;
+    auto it = std::find(p->owned.begin(), p->owned.end(), (void*)sbc);
+    if (it != p->owned.end()) {
+        p->release(sbc, st, p->alloc_ctx);
+        p->owned.erase(it);
     }
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }

@@ -300,6 +300,382 @@ __global__ void __launch_bounds__(kThreads, 3) k_ssa_select(const __grid_constan
     }
 }
 
+// ---- selection shared by the queries of a 4x4x4 sub-block --------------------------------------
+// One CTA per (selection tile, head), 192 threads in the roles of k_ssa_select. A tile holds whole
+// sub-blocks of one sequence (at most 128 rows and 32 sub-blocks), its rows grouped by sub-block.
+// The compressed keys stream twice. Pass 1 gives each row the base-2 log-sum-exp of its scaled
+// compressed logits; pass 2 its weights p = 2^(z sl - lse2), staged in shared memory and summed
+// per (sub-block, column) in a fixed order over the sub-block's rows. The thread that forms a sum
+// also tests it against its sub-block's current entry threshold and marks the column; the thread
+// that owns the sub-block's list then inserts the marked columns only. Lists hold 64-bit keys: the
+// fp32 sum's bits, then the block index complemented, so equal sums go to the lower block index
+// and the ranking of the fp32 sums is exact.
+constexpr int kMaxSub = 32;   // sub-blocks per selection tile
+
+template <int D>
+struct SLS {
+    static constexpr uint32_t kCh = D / 32;
+    static constexpr uint32_t kQReg = 128 * 64;
+    static constexpr uint32_t kGB = kCh * 512;
+    static constexpr uint32_t kTile = 8 * kGB;
+    static constexpr uint32_t kQ = 0;
+    static constexpr uint32_t kK = kQ + kCh * kQReg;
+    static constexpr uint32_t kPS = 68;                          // floats per staged row (padded)
+    static constexpr uint32_t kStage = kK + 2 * kTile;           // float [128][kPS]; after the loop
+                                                                 // int32 [kMaxSub][32]: the lists
+    static constexpr uint32_t kSum = kStage + 128 * kPS * 4;     // float [kMaxSub][64]
+    static constexpr uint32_t kThr = kSum + kMaxSub * 64 * 4;    // uint64 [kMaxSub]: entry keys
+    static constexpr uint32_t kCand = kThr + kMaxSub * 8;        // uint32 [kMaxSub][2]: marked columns
+    static constexpr uint32_t kSeg = kCand + kMaxSub * 8;        // int32 [3][kMaxSub] first, rows, own; count
+    static constexpr uint32_t kRowKey = kSeg + (3 * kMaxSub + 4) * 4;   // int32 [128]
+    static constexpr uint32_t kPro = kRowKey + 128 * 4;          // rotary table and weights
+    static constexpr uint32_t kBar = kPro + 64 * 12 + 128 * 4;
+    static constexpr uint32_t kMisc = kBar + 16 * 8;
+    static constexpr uint32_t kBytes = kMisc + 64;
+    static constexpr uint32_t kAlloc = kBytes + 1024;
+};
+
+// Named barrier that also returns the AND of `v` over the `count` threads (whole warps).
+__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t count, bool v) {
+    __syncwarp();
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(count)
+        : "memory");
+    return r != 0u;
+}
+
+// selection tiles, their rows in sub-block order
+struct SubParams {
+    FwdParams f;
+    const int4* sst;
+    const int32_t* sb_rows;
+};
+
+template <typename T, int D, int KM>
+__global__ void __launch_bounds__(kThreads, 2) k_ssa_select_sub(const __grid_constant__ SubParams S) {
+    using L = SLS<D>;
+    const FwdParams& P = S.f;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* g = align1024(smem_raw);
+    const uint32_t sb = tc::smem_u32(g);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(g + L::kBar);
+    int* misc = reinterpret_cast<int*>(g + L::kMisc);
+    volatile int* abort_flag = misc + M_ABORT;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y, H = P.H;
+
+    const int4 tl = S.sst[blockIdx.x];   // (first index into sb_rows, rows, sequence, sub-blocks)
+    const int32_t r0 = tl.x, len = tl.y, seq = tl.z;
+    const int32_t bl = P.seq_blk[seq], nblk = P.seq_blk[seq + 1] - bl;
+    const int32_t cg0 = bl >> 3, ng = ((bl + nblk + 7) >> 3) - cg0;
+    const int nc = P.k > 1 ? (ng + 7) >> 3 : 0;   // k = 1: the own block alone, nothing to rank
+
+    // ---- setup: TMEM, barriers, Q tile, zeroed K stages, prologue table, sub-blocks ------------
+    if (warp == 1) {
+        tc::tmem_alloc(reinterpret_cast<uint32_t*>(misc + M_TMEM), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], (i == SFREE || i == SFREE + 1) ? 4u : 1u);
+        misc[M_ABORT] = 0;
+        tc::fence_mbar_init();
+    }
+    const T* Q = reinterpret_cast<const T*>(P.q);
+    for (int e = tid; e < 128 * (D / 8); e += kThreads) {
+        const int row = e / (D / 8), c16 = e % (D / 8);
+        const bool ok = row < len;
+        const T* src = ok ? Q + ((int64_t)P.perm[S.sb_rows[r0 + row]] * H + h) * D + c16 * 8 : Q;
+        tc::cp_async16(sb + L::kQ + (c16 >> 2) * L::kQReg + tc::sw64(row, c16 & 3), src, ok ? 16u : 0u);
+    }
+    for (uint32_t o = tid * 16u; o < 2u * L::kTile; o += kThreads * 16u)
+        *reinterpret_cast<uint4*>(g + L::kK + o) = make_uint4(0u, 0u, 0u, 0u);
+    double* pro_freq = reinterpret_cast<double*>(g + L::kPro);
+    int* pro_axis = reinterpret_cast<int*>(g + L::kPro + 64 * 8);
+    float* pro_gamma = reinterpret_cast<float*>(g + L::kPro + 64 * 12);
+    if (P.q_gamma) {
+        if (tid < D / 2) rope_pair(D, tid, P.theta, pro_axis[tid], pro_freq[tid]);
+        if (tid < D) pro_gamma[tid] = P.q_gamma[tid];
+    }
+    // (block, sub-block) key of every row; rows come grouped by it
+    int* row_key = reinterpret_cast<int*>(g + L::kRowKey);
+    int* seg = reinterpret_cast<int*>(g + L::kSeg);   // first row | rows | own block (global) | count
+    uint64_t* thr = reinterpret_cast<uint64_t*>(g + L::kThr);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(g + L::kCand);
+    if (tid < 128) {
+        int key = -1;
+        if (tid < len) {
+            const int32_t tok = P.perm[S.sb_rows[r0 + tid]];
+            const int32_t* c = P.coords + 3 * (int64_t)tok;
+            key = 8 * P.tok_blk[tok] + ((((c[0] >> 2) & 1) << 2) | (((c[1] >> 2) & 1) << 1) | ((c[2] >> 2) & 1));
+        }
+        row_key[tid] = key;
+    }
+    if (tid < kMaxSub) {
+        thr[tid] = 0ull;
+        cand[2 * tid] = 0u;
+        cand[2 * tid + 1] = 0u;
+    }
+    tc::cp_async_wait_all();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = (uint32_t)misc[M_TMEM];
+    if (tid == 0) {
+        int n = 0;
+        for (int r = 0; r < len && n <= kMaxSub; ++r) {
+            if (r == 0 || row_key[r] != row_key[r - 1]) {
+                if (n == kMaxSub) {   // more sub-blocks than the plan packs: give up on the tile
+                    n = kMaxSub + 1;
+                    break;
+                }
+                seg[n] = r;
+                seg[kMaxSub + n] = 0;
+                seg[2 * kMaxSub + n] = row_key[r] >> 3;
+                ++n;
+            }
+            seg[kMaxSub + n - 1] += 1;
+        }
+        if (n > kMaxSub) {
+            atomicOr(P.status, DEV_BAD_INDEX);
+            n = 0;
+        }
+        seg[3 * kMaxSub] = n;
+    }
+    if (P.q_gamma && tid >= 64 && tid - 64 < len)
+        qtile_prologue<T, D>(g + L::kQ, L::kQReg, tid - 64, P.perm[S.sb_rows[r0 + tid - 64]], P.coords, pro_freq,
+                             pro_axis, pro_gamma, P.eps);
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const int nseg = seg[3 * kMaxSub];
+
+    if (warp == 0) {
+        // ================================ producer: the compressed keys, twice ================
+        const uint8_t* kch = static_cast<const uint8_t*>(P.kcg) + (int64_t)h * P.Mb8 * D * 2;
+        int last = -1;
+        for (int j = 0; j < 2 * nc && nseg > 0; ++j) {
+            const int s = j & 1, jt = j < nc ? j : j - nc;
+            if (j >= 2 && !wait_or_flag(&bar[KEMPTY + s], (uint32_t)((j >> 1) - 1) & 1u, P.status, abort_flag))
+                break;
+            const uint32_t n = (uint32_t)min(8, ng - 8 * jt);
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(&bar[KFULL + s], n * L::kGB);
+                tc::bulk_load(sb + L::kK + s * L::kTile, kch + (int64_t)(cg0 + 8 * jt) * L::kGB, n * L::kGB,
+                              &bar[KFULL + s]);
+            }
+            last = j;
+        }
+        if (lane == 0)
+            for (int j = max(last - 1, 0); j <= last; ++j)
+                tc::mbar_wait(&bar[KFULL + (j & 1)], (uint32_t)(j >> 1) & 1u, kWaitCycles);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ================================ MMA issuer ==========================================
+        if (lane == 0) {
+            const uint32_t idesc_s = tc::idesc_f16(kBf16, 128, kKT, false);
+            for (int j = 0; j < 2 * nc && nseg > 0; ++j) {
+                const int b = j & 1;
+                if (!wait_or_flag(&bar[KFULL + b], (uint32_t)(j >> 1) & 1u, P.status, abort_flag)) break;
+                if (j >= 2 && !wait_or_flag(&bar[SFREE + b], (uint32_t)((j >> 1) - 1) & 1u, P.status, abort_flag))
+                    break;
+                tc::fence_after_sync();
+                const uint32_t kbase = sb + L::kK + b * L::kTile;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_f16_ss(tmem + b * kKT, tc::desc_kmajor_r(sb + L::kQ, kk, L::kQReg),
+                                   tc::desc_kmajor_g(kbase, kk, L::kCh), idesc_s, kk > 0 ? 1u : 0u);
+                tc::mma_commit(&bar[SFULL + b]);
+                tc::mma_commit(&bar[KEMPTY + b]);
+            }
+            tc::mma_commit(&bar[FIN]);
+            tc::mbar_wait(&bar[FIN], 0u, kWaitCycles);
+        }
+        __syncwarp();
+    } else {
+        // ================================ rows: softmax statistics, weights, sums ==============
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int t128 = tid - 64;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const bool row_ok = row < len;
+        const int32_t pos = row_ok ? S.sb_rows[r0 + row] : 0;
+        const int32_t tok = P.perm[pos];
+        const int ksel = P.k;
+        const float sl = P.sl;
+        if (P.gate_w && row_ok) {
+            float t0 = P.gate_b[0], t1 = P.gate_b[1], t2 = P.gate_b[2];
+#pragma unroll 1
+            for (int c16 = 0; c16 < D / 8; ++c16) {
+                const uint4 u = *reinterpret_cast<const uint4*>(g + L::kQ + (c16 >> 2) * L::kQReg +
+                                                                 tc::sw64(row, c16 & 3));
+                const uint32_t* wv = reinterpret_cast<const uint32_t*>(&u);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int d = c16 * 8 + 2 * q;
+                    const float a = unpack_lo<T>(wv[q]), bq = unpack_hi<T>(wv[q]);
+                    const float* w0 = P.gate_w + d * 3;
+                    t0 = fmaf(a, w0[0], fmaf(bq, w0[3], t0));
+                    t1 = fmaf(a, w0[1], fmaf(bq, w0[4], t1));
+                    t2 = fmaf(a, w0[2], fmaf(bq, w0[5], t2));
+                }
+            }
+            float* go = P.gates_out + ((int64_t)tok * H + h) * 3;
+            go[0] = 1.0f / (1.0f + __expf(-t0));
+            go[1] = 1.0f / (1.0f + __expf(-t1));
+            go[2] = 1.0f / (1.0f + __expf(-t2));
+        }
+        float* stage = reinterpret_cast<float*>(g + L::kStage);
+        float* sums = reinterpret_cast<float*>(g + L::kSum);
+        uint64_t tk[KM];   // the list of sub-block t128 (t128 < nseg), best first; 0 = empty
+#pragma unroll
+        for (int u = 0; u < KM; ++u) tk[u] = 0ull;
+        float m = -INFINITY, l = 0.0f, lse = 0.0f;
+        bool ok = nseg > 0;
+        for (int j = 0; j < 2 * nc && ok; ++j) {
+            const int b = j & 1, jt = j < nc ? j : j - nc;
+            // one decision for all four row warps, so that they meet the same named barriers
+            ok = named_sync_and(1, 128, wait_or_flag(&bar[SFULL + b], (uint32_t)(j >> 1) & 1u, P.status,
+                                                     abort_flag));
+            if (!ok) break;
+            tc::fence_after_sync();
+            float s[64];
+            tc::tmem_ld64(tmem + lane_base + b * kKT, s);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bar[SFREE + b]);
+            const int32_t cbase = 8 * cg0 + kKT * jt - bl;   // local block index of column 0
+            if (cbase < 0 || cbase + kKT > nblk) {
+#pragma unroll
+                for (int e = 0; e < 64; ++e) s[e] = (cbase + e >= 0 && cbase + e < nblk) ? s[e] : -INFINITY;
+            }
+            if (j < nc) {
+                // pass 1: running maximum and sum of 2^(z sl)
+                float tmax = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 64; e += 4) tmax = fmaxf(tmax, tc::fmax3(s[e], s[e + 1], fmaxf(s[e + 2], s[e + 3])));
+                const float tm = tmax * sl;
+                if (tm > m) {
+                    l *= tc::ex2(m - tm);
+                    m = tm;
+                }
+                float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int e = 0; e < 64; ++e) ls[e & 3] += tc::ex2(fmaf(s[e], sl, -m));
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                if (j == nc - 1) lse = m + __log2f(l);
+                continue;
+            }
+            // pass 2: this row's weights into the stage
+            float4* srow = reinterpret_cast<float4*>(stage + row * L::kPS);
+#pragma unroll
+            for (int e = 0; e < 64; e += 4)
+                srow[e >> 2] = make_float4(tc::ex2(fmaf(s[e], sl, -lse)), tc::ex2(fmaf(s[e + 1], sl, -lse)),
+                                           tc::ex2(fmaf(s[e + 2], sl, -lse)), tc::ex2(fmaf(s[e + 3], sl, -lse)));
+            tc::named_sync(1, 128);
+            // sum of column c over the rows of sub-blocks q = t128 / 64, + 2, ... (four partial sums
+            // in a fixed pattern), and a mark where it can enter the sub-block's list
+            {
+                const int c = t128 & 63;
+                const int32_t blk = cbase + c;
+                const bool col_ok = blk >= 0 && blk < nblk;
+                for (int q = t128 >> 6; q < nseg; q += 2) {
+                    const int a = seg[q], n = seg[kMaxSub + q];
+                    const float* sc = stage + a * L::kPS + c;
+                    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+                    int r = 0;
+                    for (; r + 4 <= n; r += 4) {
+                        a0 += sc[r * L::kPS];
+                        a1 += sc[(r + 1) * L::kPS];
+                        a2 += sc[(r + 2) * L::kPS];
+                        a3 += sc[(r + 3) * L::kPS];
+                    }
+                    for (; r < n; ++r) a0 += sc[r * L::kPS];
+                    const float acc = (a0 + a1) + (a2 + a3);
+                    sums[q * 64 + c] = acc;
+                    const uint64_t key = ((uint64_t)__float_as_uint(acc) << 32) | (uint32_t)(0x7fffffff - blk);
+                    if (col_ok && blk != seg[2 * kMaxSub + q] - bl && key > thr[q])
+                        atomicOr(&cand[2 * q + (c >> 5)], 1u << (c & 31));
+                }
+            }
+            tc::named_sync(1, 128);
+            if (t128 < nseg) {
+                const float* sq = sums + t128 * 64;
+#pragma unroll 1
+                for (int hw = 0; hw < 2; ++hw) {
+                    uint32_t mk = cand[2 * t128 + hw];
+                    while (mk) {
+                        const int e = 32 * hw + __ffs(mk) - 1;
+                        mk &= mk - 1;
+                        const int32_t blk = cbase + e;
+                        const uint64_t key = ((uint64_t)__float_as_uint(sq[e]) << 32) | (uint32_t)(0x7fffffff - blk);
+                        if (key > tk[KM - 1]) {
+#pragma unroll
+                            for (int q = KM - 1; q > 0; --q) tk[q] = max(tk[q], min(tk[q - 1], key));
+                            tk[0] = max(tk[0], key);
+                        }
+                    }
+                    cand[2 * t128 + hw] = 0u;
+                }
+                thr[t128] = tk[KM - 1];
+            }
+        }
+        tc::named_sync(1, 128);   // the stage is free: the lists go there
+        int32_t* lists = reinterpret_cast<int32_t*>(g + L::kStage);
+        if (t128 < nseg) {
+#pragma unroll
+            for (int u = 0; u < KM; ++u)
+                lists[t128 * 32 + u] = tk[u] ? bl + (0x7fffffff - (int32_t)(uint32_t)(tk[u] & 0xffffffffull)) : -1;
+        }
+        tc::named_sync(1, 128);
+        if (row_ok && nseg > 0 && !*abort_flag) {
+            int q = 0;
+            while (q + 1 < nseg && row >= seg[q + 1]) ++q;
+            int32_t* so = P.sel + ((int64_t)pos * H + h) * ksel;
+            so[0] = seg[2 * kMaxSub + q];
+#pragma unroll
+            for (int u = 0; u < KM; ++u)
+                if (u + 1 < ksel) so[u + 1] = nc > 0 ? lists[q * 32 + u] : -1;
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <typename T, int D, int KM>
+ssa_status_t run_sub(const Plan* p, const FwdParams& P, cudaStream_t st) {
+    SubParams S;
+    S.f = P;
+    S.sst = p->sst;
+    S.sb_rows = p->sb_rows;
+    using L = SLS<D>;
+    static_assert(L::kAlloc <= 113u * 1024u, "at least two CTAs per SM");
+    static bool configured = false;
+    if (!configured) {
+        if (cudaFuncSetAttribute(k_ssa_select_sub<T, D, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)L::kAlloc) != cudaSuccess)
+            return SSA_ERR_CUDA;
+        configured = true;
+    }
+    if (p->n_sst == 0) return SSA_OK;
+    k_ssa_select_sub<T, D, KM><<<dim3((unsigned)p->n_sst, (unsigned)P.H), kThreads, L::kAlloc, st>>>(S);
+    note_launch();
+    return cudaPeekAtLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
 template <typename T, int D, int KM>
 ssa_status_t run(const Plan* p, const FwdParams& P, cudaStream_t st) {
     using L = SL<D>;
@@ -317,27 +693,30 @@ ssa_status_t run(const Plan* p, const FwdParams& P, cudaStream_t st) {
 }
 
 template <typename T, int D>
-ssa_status_t run_km(const Plan* p, const FwdParams& P, cudaStream_t st) {
+ssa_status_t run_km(const Plan* p, const FwdParams& P, bool shared, cudaStream_t st) {
     // KM: the list length, k - 1 rounded up to 7, 15 or 31 (k <= 32)
+    if (shared) {
+        if (P.k <= 8) return run_sub<T, D, 7>(p, P, st);
+        if (P.k <= 16) return run_sub<T, D, 15>(p, P, st);
+        return run_sub<T, D, 31>(p, P, st);
+    }
     if (P.k <= 8) return run<T, D, 7>(p, P, st);
     if (P.k <= 16) return run<T, D, 15>(p, P, st);
     return run<T, D, 31>(p, P, st);
 }
 
 template <typename T>
-ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, cudaStream_t st) {
+ssa_status_t run_d(const Plan* p, const FwdParams& P, int D, bool shared, cudaStream_t st) {
     switch (D) {
-    case 32: return run_km<T, 32>(p, P, st);
-    case 64: return run_km<T, 64>(p, P, st);
-    case 96: return run_km<T, 96>(p, P, st);
-    default: return run_km<T, 128>(p, P, st);
+    case 32: return run_km<T, 32>(p, P, shared, st);
+    case 64: return run_km<T, 64>(p, P, shared, st);
+    case 96: return run_km<T, 96>(p, P, shared, st);
+    default: return run_km<T, 128>(p, P, shared, st);
     }
 }
 
-}  // namespace
-
-ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
-                              const float* gate_w, const float* gate_b, float* gates_out, cudaStream_t st) {
+FwdParams select_params(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
+                        const float* gate_w, const float* gate_b, float* gates_out) {
     FwdParams P = FwdParams();
     P.q = q;
     P.kcg = w.kcg;
@@ -361,9 +740,27 @@ ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, 
     P.Mb8 = w.Mb8;
     P.H = w.H;
     P.k = w.k;
+    P.sl = (float)(1.4426950408889634 / sqrt((double)w.D));
+    return P;
+}
+
+}  // namespace
+
+ssa_status_t launch_select_tc(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
+                              const float* gate_w, const float* gate_b, float* gates_out, cudaStream_t st) {
+    const FwdParams P = select_params(p, w, q, pro, gate_w, gate_b, gates_out);
     ProfScope ps("k_ssa_select", st);
-    if (w.dtype == SSA_BF16) return run_d<__nv_bfloat16>(p, P, w.D, st);
-    return run_d<__half>(p, P, w.D, st);
+    if (w.dtype == SSA_BF16) return run_d<__nv_bfloat16>(p, P, w.D, false, st);
+    return run_d<__half>(p, P, w.D, false, st);
+}
+
+ssa_status_t launch_select_shared(const Plan* p, const Workspace& w, const void* q, const Prologue& pro,
+                                  const float* gate_w, const float* gate_b, float* gates_out,
+                                  cudaStream_t st) {
+    const FwdParams P = select_params(p, w, q, pro, gate_w, gate_b, gates_out);
+    ProfScope ps("k_ssa_select_sub", st);
+    if (w.dtype == SSA_BF16) return run_d<__nv_bfloat16>(p, P, w.D, true, st);
+    return run_d<__half>(p, P, w.D, true, st);
 }
 
 }  // namespace ssa

@@ -153,10 +153,25 @@ bool check_device(ssa_status_t* st) {
 
 size_t elem_size(ssa_dtype_t t) { return t == SSA_F32 ? 4 : 2; }
 
+void free_host_pipe(Plan* p) {
+    HostPipe& hp = p->hp;
+    if (hp.s_in) cudaStreamSynchronize(hp.s_in);
+    if (hp.s_out) cudaStreamSynchronize(hp.s_out);
+    plan_free_all(p, hp.owned);
+    for (cudaEvent_t e : {hp.e_in[0], hp.e_in[1], hp.e_comp[0], hp.e_comp[1], hp.e_out[0], hp.e_out[1],
+                          hp.e_par, hp.e_start})
+        if (e) cudaEventDestroy(e);
+    if (hp.s_in) cudaStreamDestroy(hp.s_in);
+    if (hp.s_out) cudaStreamDestroy(hp.s_out);
+    hp = HostPipe();
+}
+
 void destroy(Plan* p) {
     ssa_plan_s* h = static_cast<ssa_plan_s*>(p);
     if (!p) return;
     plan_free_all(p, p->ws.owned);
+    plan_free_all(p, p->ws_chunk.owned);
+    free_host_pipe(p);
     plan_free_all(p, p->owned);
     if (p->ws.h_q) cudaStreamSynchronize(p->stream);
     delete h;
@@ -236,9 +251,8 @@ ssa_status_t make_plan(const int32_t* coords, const int64_t* cu, int32_t B, cons
 }
 
 // (Re)allocates the forward workspace for (H, D, dtype, k) if the cached one does not match.
-ssa_status_t ensure_workspace(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int32_t k,
+ssa_status_t ensure_workspace(Plan* p, Workspace& w, int32_t H, int32_t D, ssa_dtype_t dt, int32_t k,
                               cudaStream_t st) {
-    Workspace& w = p->ws;
     if (w.H == H && w.D == D && w.dtype == dt && w.k == k && w.kc) return SSA_OK;
     plan_free_all(p, w.owned);
     w = Workspace();
@@ -311,10 +325,11 @@ ssa_status_t ensure_buffer(Plan* p, Workspace& w, P*& buf, size_t bytes, cudaStr
 ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, const float* gates,
                          const float* wc, int32_t H, int32_t D, ssa_dtype_t dt, int32_t topk,
                          void* out, int32_t* sel_out, cudaStream_t st,
-                         const BranchOut& bo = BranchOut(), const Options& opt = Options()) {
-    ssa_status_t rc = ensure_workspace(p, H, D, dt, topk, st);
+                         const BranchOut& bo = BranchOut(), const Options& opt = Options(),
+                         Workspace* wsp = nullptr) {
+    Workspace& w = wsp ? *wsp : p->ws;
+    ssa_status_t rc = ensure_workspace(p, w, H, D, dt, topk, st);
     if (rc != SSA_OK) return rc;
-    Workspace& w = p->ws;
     const Prologue& pro = opt.pro;
     if (pro.on() && dt == SSA_F32) {
         // fp32 path: the prologue is a pass of its own into workspace copies of q and k
@@ -369,6 +384,118 @@ ssa_status_t run_forward(Plan* p, const void* q, const void* k, const void* v, c
     trace_step("forward", st);
     if (sel_out) launch_export_sel(p, w, sel_out, st);
     return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+// Gates of heads [h0, h0 + hc) of [N, H, 3] into [N, hc, 3].
+__global__ void k_gather_gates(const float* __restrict__ in, int64_t N, int H, int h0, int hc,
+                               float* __restrict__ out) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= N * hc * 3) return;
+    const int64_t n = e / (hc * 3), r = e % (hc * 3);
+    out[e] = in[(n * H + h0) * 3 + r];
+}
+
+// Heads per chunk of the host-buffer path: the smallest divisor of H whose rows of one token are
+// at least 256 bytes (efficient strided copies); H itself (no chunking) if there is none below H.
+int32_t host_chunk_heads(int32_t H, int32_t D, ssa_dtype_t dt) {
+    const size_t es = elem_size(dt);
+    for (int32_t d = 1; d < H; ++d)
+        if (H % d == 0 && (size_t)d * D * es >= 256) return d;
+    return H;
+}
+
+ssa_status_t ensure_host_pipe(Plan* p, int32_t H, int32_t D, ssa_dtype_t dt, int32_t hc, cudaStream_t st) {
+    HostPipe& hp = p->hp;
+    if (hp.hc == hc && hp.H == H && hp.D == D && hp.dtype == dt) return SSA_OK;
+    free_host_pipe(p);
+    if (cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) ||
+        cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking))
+        return SSA_ERR_CUDA;
+    for (cudaEvent_t* e : {&hp.e_in[0], &hp.e_in[1], &hp.e_comp[0], &hp.e_comp[1], &hp.e_out[0], &hp.e_out[1],
+                           &hp.e_par, &hp.e_start})
+        if (cudaEventCreateWithFlags(e, cudaEventDisableTiming)) return SSA_ERR_CUDA;
+    const size_t cb = elem_size(dt) * (size_t)p->N * hc * D;
+    auto A = [&](size_t bytes) -> void* {
+        void* ptr = p->alloc(std::max<size_t>(bytes, 16), st, p->alloc_ctx);
+        if (ptr) hp.owned.push_back(ptr);
+        return ptr;
+    };
+    for (int s = 0; s < 2; ++s) {
+        hp.q[s] = A(cb);
+        hp.k[s] = A(cb);
+        hp.v[s] = A(cb);
+        hp.o[s] = A(cb);
+        hp.g[s] = (float*)A(sizeof(float) * 3 * (size_t)p->N * hc);
+        if (!hp.q[s] || !hp.k[s] || !hp.v[s] || !hp.o[s] || !hp.g[s]) return SSA_ERR_ALLOC;
+    }
+    hp.gates = (float*)A(sizeof(float) * 3 * (size_t)p->N * H);
+    hp.wc = (float*)A(sizeof(float) * (size_t)D * D);
+    if (!hp.gates || !hp.wc) return SSA_ERR_ALLOC;
+    // the buffers come from the caller's stream: the side streams wait for their allocation
+    if (cudaEventRecord(hp.e_start, st) || cudaStreamWaitEvent(hp.s_in, hp.e_start, 0) ||
+        cudaStreamWaitEvent(hp.s_out, hp.e_start, 0))
+        return SSA_ERR_CUDA;
+    hp.hc = hc;
+    hp.H = H;
+    hp.D = D;
+    hp.dtype = dt;
+    return SSA_OK;
+}
+
+// The host-buffer forward, heads in chunks of hc: chunk c's inputs are copied in on s_in (strided
+// rows of the [N, H, D] host tensors) while chunk c - 1 runs on the caller's stream and chunk
+// c - 2's output is copied out on s_out. Two slots of buffers; events order their reuse.
+ssa_status_t forward_host_chunked(Plan* p, const void* q, const void* k, const void* v, const float* gates,
+                                  const float* wc, int32_t H, int32_t D, ssa_dtype_t dt, int32_t topk,
+                                  void* out, int32_t hc, cudaStream_t st) {
+    ssa_status_t rc = ensure_host_pipe(p, H, D, dt, hc, st);
+    if (rc != SSA_OK) return rc;
+    HostPipe& hp = p->hp;
+    const size_t es = elem_size(dt), row = es * (size_t)H * D, crow = es * (size_t)hc * D;
+    const int64_t N = p->N;
+    const int nch = H / hc;
+    const auto H2D = cudaMemcpyHostToDevice, D2H = cudaMemcpyDeviceToHost;
+    // work the caller queued before this call (a plan rebuild) comes first on every stream
+    if (cudaEventRecord(hp.e_start, st) || cudaStreamWaitEvent(hp.s_in, hp.e_start, 0) ||
+        cudaStreamWaitEvent(hp.s_out, hp.e_start, 0))
+        return SSA_ERR_CUDA;
+    if (cudaMemcpyAsync(hp.gates, gates, sizeof(float) * 3 * (size_t)N * H, H2D, hp.s_in) ||
+        cudaMemcpyAsync(hp.wc, wc, sizeof(float) * (size_t)D * D, H2D, hp.s_in) ||
+        cudaEventRecord(hp.e_par, hp.s_in))
+        return SSA_ERR_CUDA;
+    for (int c = 0; c < nch; ++c) {
+        const int s = c & 1;
+        const size_t h0 = (size_t)c * hc * D * es;
+        // copies in: the slot's previous chunk must be done with its inputs
+        if (c >= 2 && cudaStreamWaitEvent(hp.s_in, hp.e_comp[s], 0)) return SSA_ERR_CUDA;
+        if (cudaMemcpy2DAsync(hp.q[s], crow, (const uint8_t*)q + h0, row, crow, (size_t)N, H2D, hp.s_in) ||
+            cudaMemcpy2DAsync(hp.k[s], crow, (const uint8_t*)k + h0, row, crow, (size_t)N, H2D, hp.s_in) ||
+            cudaMemcpy2DAsync(hp.v[s], crow, (const uint8_t*)v + h0, row, crow, (size_t)N, H2D, hp.s_in) ||
+            cudaEventRecord(hp.e_in[s], hp.s_in))
+            return SSA_ERR_CUDA;
+        // the forward of the chunk: its inputs are in, the slot's previous output is out
+        if (cudaStreamWaitEvent(st, hp.e_in[s], 0) || (c == 0 && cudaStreamWaitEvent(st, hp.e_par, 0)) ||
+            (c >= 2 && cudaStreamWaitEvent(st, hp.e_out[s], 0)))
+            return SSA_ERR_CUDA;
+        const int64_t ng = N * hc * 3;
+        if (ng > 0) {
+            k_gather_gates<<<(unsigned)cdiv(ng, 256), 256, 0, st>>>(hp.gates, N, H, c * hc, hc, hp.g[s]);
+            note_launch();
+        }
+        rc = run_forward(p, hp.q[s], hp.k[s], hp.v[s], hp.g[s], hp.wc, hc, D, dt, topk, hp.o[s], nullptr, st,
+                         BranchOut(), Options(), &p->ws_chunk);
+        if (rc != SSA_OK) return rc;
+        if (cudaEventRecord(hp.e_comp[s], st)) return SSA_ERR_CUDA;
+        // copies out
+        if (cudaStreamWaitEvent(hp.s_out, hp.e_comp[s], 0) ||
+            cudaMemcpy2DAsync((uint8_t*)out + h0, row, hp.o[s], crow, crow, (size_t)N, D2H, hp.s_out) ||
+            cudaEventRecord(hp.e_out[s], hp.s_out))
+            return SSA_ERR_CUDA;
+    }
+    // the caller's stream completes after the last copies out
+    for (int s = 0; s < 2 && s < nch; ++s)
+        if (cudaStreamWaitEvent(st, hp.e_out[s], 0)) return SSA_ERR_CUDA;
+    return SSA_OK;
 }
 
 }  // namespace
@@ -429,11 +556,15 @@ ssa_status_t ssa_plan_rebuild(ssa_plan_t p, const int32_t* coords, void* stream)
         plan_free_all(p, p->owned);
         plan_free_all(p, p->ws.owned);
         p->ws = Workspace();
+        plan_free_all(p, p->ws_chunk.owned);
+        p->ws_chunk = Workspace();
         return rc;
     }
     if (p->Mb != old_mb || p->Nks != old_nks) {
         plan_free_all(p, p->ws.owned);
         p->ws = Workspace();
+        plan_free_all(p, p->ws_chunk.owned);
+        p->ws_chunk = Workspace();
     }
     return SSA_OK;
 }
@@ -559,37 +690,43 @@ ssa_status_t ssa_forward_host(ssa_plan_t p, const void* q, const void* k, const 
     ssa_status_t rc = check_forward_args(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out);
     if (rc != SSA_OK) return rc;
     cudaStream_t st = (cudaStream_t)stream;
-    Workspace& w = p->ws;
-    const size_t tb = elem_size(dtype) * (size_t)p->N * heads * head_dim;
-    const size_t gb = sizeof(float) * (size_t)p->N * heads * 3;
-    const size_t wb = sizeof(float) * (size_t)head_dim * head_dim;
-    rc = ensure_workspace(p, heads, head_dim, dtype, topk, st);
-    if (rc != SSA_OK) return rc;
-    if (!w.h_q) {
-        void* bufs[6];
-        const size_t sizes[6] = {tb, tb, tb, tb, gb, wb};
-        for (int i = 0; i < 6; ++i) {
-            bufs[i] = p->alloc(sizes[i], st, p->alloc_ctx);
-            if (!bufs[i]) return SSA_ERR_ALLOC;
-            w.owned.push_back(bufs[i]);
+    const int32_t hc = host_chunk_heads(heads, head_dim, dtype);
+    if (hc < heads) {
+        if ((rc = forward_host_chunked(p, q, k, v, gates, wc, heads, head_dim, dtype, topk, out, hc, st)) != SSA_OK)
+            return rc;
+    } else {
+        Workspace& w = p->ws;
+        const size_t tb = elem_size(dtype) * (size_t)p->N * heads * head_dim;
+        const size_t gb = sizeof(float) * (size_t)p->N * heads * 3;
+        const size_t wb = sizeof(float) * (size_t)head_dim * head_dim;
+        rc = ensure_workspace(p, w, heads, head_dim, dtype, topk, st);
+        if (rc != SSA_OK) return rc;
+        if (!w.h_q) {
+            void* bufs[6];
+            const size_t sizes[6] = {tb, tb, tb, tb, gb, wb};
+            for (int i = 0; i < 6; ++i) {
+                bufs[i] = p->alloc(sizes[i], st, p->alloc_ctx);
+                if (!bufs[i]) return SSA_ERR_ALLOC;
+                w.owned.push_back(bufs[i]);
+            }
+            w.h_q = bufs[0];
+            w.h_k = bufs[1];
+            w.h_v = bufs[2];
+            w.h_out = bufs[3];
+            w.h_gates = (float*)bufs[4];
+            w.h_wc = (float*)bufs[5];
         }
-        w.h_q = bufs[0];
-        w.h_k = bufs[1];
-        w.h_v = bufs[2];
-        w.h_out = bufs[3];
-        w.h_gates = (float*)bufs[4];
-        w.h_wc = (float*)bufs[5];
+        const auto H2D = cudaMemcpyHostToDevice;
+        if (cudaMemcpyAsync(w.h_q, q, tb, H2D, st) || cudaMemcpyAsync(w.h_k, k, tb, H2D, st) ||
+            cudaMemcpyAsync(w.h_v, v, tb, H2D, st) || cudaMemcpyAsync(w.h_gates, gates, gb, H2D, st) ||
+            cudaMemcpyAsync(w.h_wc, wc, wb, H2D, st))
+            return SSA_ERR_CUDA;
+        rc = run_forward(p, w.h_q, w.h_k, w.h_v, w.h_gates, w.h_wc, heads, head_dim, dtype, topk,
+                         w.h_out, nullptr, st);
+        if (rc != SSA_OK) return rc;
+        if (cudaMemcpyAsync(out, w.h_out, tb, cudaMemcpyDeviceToHost, st)) return SSA_ERR_CUDA;
     }
-    const auto H2D = cudaMemcpyHostToDevice;
-    if (cudaMemcpyAsync(w.h_q, q, tb, H2D, st) || cudaMemcpyAsync(w.h_k, k, tb, H2D, st) ||
-        cudaMemcpyAsync(w.h_v, v, tb, H2D, st) || cudaMemcpyAsync(w.h_gates, gates, gb, H2D, st) ||
-        cudaMemcpyAsync(w.h_wc, wc, wb, H2D, st))
-        return SSA_ERR_CUDA;
-    rc = run_forward(p, w.h_q, w.h_k, w.h_v, w.h_gates, w.h_wc, heads, head_dim, dtype, topk,
-                     w.h_out, nullptr, st);
-    if (rc != SSA_OK) return rc;
-    if (cudaMemcpyAsync(out, w.h_out, tb, cudaMemcpyDeviceToHost, st) || cudaStreamSynchronize(st))
-        return SSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st)) return SSA_ERR_CUDA;
     int32_t s = 0;
     if (cudaMemcpy(&s, p->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost)) return SSA_ERR_CUDA;
     return map_device_status(s);
@@ -603,7 +740,7 @@ ssa_status_t ssa_backward(ssa_plan_t p, const void* q, const void* k, const void
     if (rc != SSA_OK) return rc;
     if (!dout || !dk || !dv) return SSA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    rc = ensure_workspace(p, heads, head_dim, dtype, topk, st);
+    rc = ensure_workspace(p, p->ws, heads, head_dim, dtype, topk, st);
     if (rc != SSA_OK) return rc;
     // the selection is the forward's: run the forward path to produce it (output goes to dq,
     // which the backward overwrites)

@@ -78,6 +78,26 @@ struct Workspace {
     std::vector<void*> owned;
 };
 
+// Host-buffer entry point, heads in chunks: copies in (s_in), the forward of a chunk (the
+// caller's stream) and copies out (s_out) overlap; two slots of device buffers.
+struct HostPipe {
+    int32_t hc = 0;                 // heads per chunk the buffers are sized for (0 = none yet)
+    int32_t H = 0, D = 0;
+    ssa_dtype_t dtype = SSA_F32;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t e_in[2] = {nullptr, nullptr}, e_comp[2] = {nullptr, nullptr}, e_out[2] = {nullptr, nullptr};
+    cudaEvent_t e_par = nullptr;    // gates and Wc copied
+    cudaEvent_t e_start = nullptr;  // the caller's stream at entry
+    void* q[2] = {nullptr, nullptr};
+    void* k[2] = {nullptr, nullptr};
+    void* v[2] = {nullptr, nullptr};
+    void* o[2] = {nullptr, nullptr};
+    float* g[2] = {nullptr, nullptr};
+    float* gates = nullptr;         // [N, H, 3] all heads
+    float* wc = nullptr;            // [D, D]
+    std::vector<void*> owned;
+};
+
 struct Plan {
     int device = 0;
     cudaStream_t stream = nullptr;  // creation stream (frees are queued here)
@@ -139,6 +159,8 @@ struct Plan {
     uint64_t* wmask = nullptr;   // [wm_off[T]][128] window mask: bit c of row i = key c within r
     std::vector<void*> owned;
     Workspace ws;
+    Workspace ws_chunk;   // workspace of the chunked host-buffer path (its heads per chunk)
+    HostPipe hp;
 };
 
 extern std::atomic<int64_t> g_launches;

@@ -213,6 +213,25 @@ def test_repeat_calls_are_bitwise_identical_and_host_entry_matches():
     assert torch.equal(a.cpu(), out_h)
 
 
+@pytest.mark.parametrize("H,D,dtype", [(6, 32, "f32"), (22, 96, "f16"), (4, 64, "bf16")])
+def test_host_entry_in_head_chunks_matches_the_device_forward(H, D, dtype):
+    """The host-buffer entry point copies and computes the heads in chunks (6 x 32 fp32 in 3
+    chunks of 2, 22 x 96 fp16 in 11, 4 x 64 bf16 in 2): every element equals the device forward."""
+    c, cu, g = coords_of("small")
+    cfg = workloads.WorkloadConfig("chunks", 17, (), H=H, D=D, dtype=dtype, topk=8, radius=2)
+    t = workloads.make_tensors(cfg, len(c))
+    plan = make_plan(c, cu, g, 2)
+    dev = to_gpu(t)
+    a = plan.forward(dev["Q"], dev["K"], dev["V"], dev["gates"], dev["Wc"], 8)
+    host = {k: v.pin_memory() for k, v in t.items()}
+    out_h = torch.empty_like(host["Q"]).pin_memory()
+    for _ in range(2):   # the second call reuses the chunk buffers
+        out_h.zero_()
+        plan.forward_host(host["Q"], host["K"], host["V"], host["gates"], host["Wc"], 8, out_h)
+        torch.cuda.synchronize()
+        assert torch.equal(a.cpu(), out_h)
+
+
 def test_forward_argument_errors():
     import spatial_sparse_attention_b200 as ssa
     c, cu, g = coords_of("tiny")

@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the timing of the forward's options (prologue, convolution, gates)")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the timing of the backward (ssa_backward) on the same workload")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the workload with this many heads instead of the config's "
                          "(a smaller cut for profiling; 0 = the config's own)")
@@ -349,7 +351,51 @@ def run_ours(args, rank, world, dist):
     }
     if not args.no_variants:
         res["variants"] = measure_variants(plan, dev, cfg, pk.get("hbm_gbs", 6650.0))
+    if not args.no_backward:
+        res["backward"] = measure_backward(plan, dev, cfg, work, peak)
     return res
+
+
+def measure_backward(plan, dev, cfg, work, peak, steps=3, warmup=1):
+    """ssa_backward on the same workload with a seeded dO ~ N(0, 1): ms per call (CUDA events; the
+    call runs the forward that fixes the selection first), the split between that forward and the
+    backward kernels, and the backward's algorithmic rate: 10 D FLOP per credited (query, key)
+    pair (recomputed q.k and dO.v, and the dq, dk, dv products), 2.5 times the forward's."""
+    import torch
+    import spatial_sparse_attention_b200 as ssa
+    g = torch.Generator(device="cuda").manual_seed(cfg.index * 1000 + 6)
+    dO = torch.randn(dev["Q"].shape, generator=g, device="cuda", dtype=torch.float32).to(dev["Q"].dtype)
+
+    def bwd():
+        return plan.backward(dev["Q"], dev["K"], dev["V"], dev["gates"], dev["Wc"], dO, cfg.topk)
+
+    for _ in range(warmup):
+        bwd()
+    torch.cuda.synchronize()
+    ssa.profile_reset()
+    ssa.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        bwd()
+    e1.record()
+    torch.cuda.synchronize()
+    ssa.profile_enable(False)
+    prof = ssa.profile_read()
+    if plan.status() != 0:
+        raise RuntimeError("device status set during the backward")
+    ms = e0.elapsed_time(e1) / steps
+    flop = 2.5 * work["total"]
+    bk = prof.get("backward", (0.0, 1))[0] / steps
+    r = {"ms": ms, "tokens_per_s": dev["Q"].shape[0] / (ms * 1e-3),
+         "breakdown_ms": {k: v[0] / steps for k, v in prof.items()},
+         "algorithmic_tflop": flop / 1e12,
+         "backward_kernels_tflops": flop / (bk * 1e-3) / 1e12 if bk > 0 else None,
+         "note": "CUDA-core kernels for the selected and window branches (query side, key side), "
+                 "cuBLAS TF32 GEMMs for the compressed branch; the call includes its forward"}
+    if peak and bk > 0:
+        r["frac_of_fp16_peak"] = flop / (bk * 1e-3) / 1e12 / peak
+    return r
 
 
 def oracle_cost_model(cfg, coords, cu, t, n_rows, seed):

@@ -51,8 +51,10 @@ def build(verbose: bool = False, jobs: int = 8) -> str:
         objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
     if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
         tmp = LIB + ".tmp%d" % os.getpid()
+        cuda_lib = os.path.join(os.path.dirname(os.path.dirname(NVCC)), "lib64")
         subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
-                        "-cudart", "static", "-o", tmp, *objs], check=True)
+                        "-cudart", "static", "-o", tmp, *objs, "-L", cuda_lib, "-lcublas",
+                        "-Xlinker", "-rpath", "-Xlinker", cuda_lib], check=True)
         os.replace(tmp, LIB)
     return LIB
 

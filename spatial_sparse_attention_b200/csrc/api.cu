@@ -172,6 +172,7 @@ void destroy(Plan* p) {
     plan_free_all(p, p->ws.owned);
     plan_free_all(p, p->ws_chunk.owned);
     free_host_pipe(p);
+    destroy_blas(p);
     plan_free_all(p, p->owned);
     if (p->ws.h_q) cudaStreamSynchronize(p->stream);
     delete h;

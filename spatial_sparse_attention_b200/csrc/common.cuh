@@ -161,6 +161,7 @@ struct Plan {
     Workspace ws;
     Workspace ws_chunk;   // workspace of the chunked host-buffer path (its heads per chunk)
     HostPipe hp;
+    void* cublas = nullptr;   // cuBLAS handle of the backward's compressed-branch GEMMs (first use)
 };
 
 extern std::atomic<int64_t> g_launches;
@@ -256,6 +257,7 @@ ssa_status_t launch_forward_tc(const Plan* p, const Workspace& w, const void* q,
                                void* out, const BranchOut& bo, const Prologue& pro, cudaStream_t s);
 
 // backward.cu
+void destroy_blas(Plan* p);
 ssa_status_t launch_backward(Plan* p, const Workspace& w, const void* q, const void* k,
                              const void* v, const float* gates, const float* wc, const void* dout,
                              void* dq, void* dk, void* dv, cudaStream_t s);

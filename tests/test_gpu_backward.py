@@ -89,3 +89,24 @@ def test_backward_varlen_rows_one_head_in_full_and_sums():
         exp = (np.einsum("nh,nhd->hd", gates[lo:hi, :, 0], dO[lo:hi]) @ Wc.T
                + np.einsum("nh,nhd->hd", gates[lo:hi, :, 1] + gates[lo:hi, :, 2], dO[lo:hi]))
         assert rel_l2(dv[lo:hi].sum(0), exp) <= 5e-3
+
+
+def test_backward_head_dims_and_ragged_varlen():
+    """Every element of dQ, dK, dV on a ragged batch (an empty and a one-token sequence among two
+    shells) for head dims 32-128 in each input type: the compressed branch's GEMMs meet sequences
+    of one row and one block, and batches of heads of every size."""
+    a, _, _ = coords_of("tiny")
+    b = np.array([[5, 6, 7]], np.int32)
+    c = np.concatenate([a[:700], b, a[700:1333]])
+    cu = np.array([0, 700, 700, 701, len(c)])
+    grids = np.array([[32, 32, 32], [16, 16, 16], [9, 9, 9], [32, 32, 32]], np.int32)
+    for D, dtype, k in ((128, "f16", 5), (96, "bf16", 3), (32, "f32", 4)):
+        cfg = workloads.WorkloadConfig("bwd", 19, (), H=3, D=D, dtype=dtype, topk=k, radius=2)
+        t = workloads.make_tensors(cfg, len(c), with_grad_out=True)
+        plan = make_plan(c, cu, grids, 2)
+        dq, dk, dv, sel = gpu_backward(plan, t, k)
+        bs = plan.export()["blk_seq"].cpu().numpy()
+        gs, _ = validate_gpu_selection(c, cu, t, k, 2, sel, bs, dtype)
+        ref = oracle.backward(c, cu, t["Q"], t["K"], t["V"], t["gates"], t["Wc"], t["dO"], k, 2, sel=gs)
+        for x, r, nm in zip((dq, dk, dv), ref, ("dQ", "dK", "dV")):
+            check_grad_close(_np(x), r, dtype, f"D={D} {dtype} {nm}")

@@ -255,8 +255,13 @@ SSA_API ssa_status_t ssa_forward_ex(ssa_plan_t plan, const void* q, const void* 
 
 /*
  * ssa_forward on HOST buffers: copies q, k, v, gates, wc (host) to plan-owned device buffers,
- * runs the forward and copies the result into out (host). Pinned host memory gives overlapped,
- * full-speed copies; pageable memory works but is slower. Waits for the device before returning.
+ * runs the forward and copies the result into out (host). When H has a divisor h < H whose token
+ * rows are at least 256 bytes (h D element size), the heads go in chunks of the smallest such h:
+ * the copies of one chunk in, the forward of the previous one and the copy of the one before
+ * that out overlap on two plan-owned side streams (first call: streams, events and two slots of
+ * chunk buffers are created). Results equal the device forward's bit for bit. Pinned host memory
+ * gives overlapped, full-speed copies; pageable memory works but is slower. The side streams
+ * start after the work queued on `stream` before the call. Waits for the device before returning.
  */
 SSA_API ssa_status_t ssa_forward_host(ssa_plan_t plan, const void* q, const void* k, const void* v,
                               const float* gates, const float* wc, int32_t heads,
@@ -268,8 +273,13 @@ SSA_API ssa_status_t ssa_forward_host(ssa_plan_t plan, const void* q, const void
  * method trains through SSA, with a faster backward than baseline sparse attention): gradients
  * of sum(dO * out) with respect to q, k, v, with the block
  * selection held fixed (it is not differentiable) and the compressed tokens' rounding treated as
- * identity. dq, dk, dv: device [N, H, D] of dtype. Accumulates in fp32 (CUDA cores); intended for
- * correctness, not speed. Queues work and returns without waiting.
+ * identity. dq, dk, dv: device [N, H, D] of dtype. Runs the forward first (for the selection).
+ * The compressed branch goes through cuBLAS strided-batched GEMMs per sequence (TF32 tensor cores
+ * for bf16 / fp16, fp32 for fp32; the first call creates the plan's cuBLAS handle) with fp32
+ * buffers of rows x blocks per head (up to 16 GB each, two of them); the selected and window
+ * branches through CUDA-core kernels for the query side and, over inverted selection lists and
+ * the window lists, the key side, with fp32 accumulation and no atomics. Queues work and returns
+ * without waiting (the buffers are allocated and freed stream-ordered through the allocator).
  */
 SSA_API ssa_status_t ssa_backward(ssa_plan_t plan, const void* q, const void* k, const void* v,
                           const float* gates, const float* wc, const void* dout, int32_t heads,

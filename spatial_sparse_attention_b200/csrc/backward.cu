@@ -68,13 +68,28 @@ __device__ __forceinline__ float warp_sum(float s) {
     return s;
 }
 
+// Lane L holds elements [4L, 4L + 4) of a D-vector (D <= 128, a multiple of 32): one 8-byte
+// (16-bit types) or 16-byte (fp32) load per row.
+template <typename T>
+__device__ __forceinline__ void load4(const T* base, int64_t row, int D, int lane, float (&x)[4]) {
+    if (4 * lane >= D) {
+        x[0] = x[1] = x[2] = x[3] = 0.0f;
+        return;
+    }
+    if constexpr (std::is_same<T, float>::value) {
+        const float4 v = *reinterpret_cast<const float4*>(base + row + 4 * lane);
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(base + row + 4 * lane);
+        const T* e = reinterpret_cast<const T*>(&v);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) x[c] = Elem<T>::to_f(e[c]);
+    }
+}
+
 template <typename T>
 __device__ __forceinline__ void load_row(const void* base, int64_t row, int D, int lane, float (&x)[4]) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int d = lane + 32 * t;
-        x[t] = d < D ? ld<T>(base, row + d) : 0.0f;
-    }
+    load4<T>(reinterpret_cast<const T*>(base), row, D, lane, x);
 }
 
 // Keys are visited four at a time (independent loads and reductions in flight). A visitor gets
@@ -140,17 +155,16 @@ __device__ void branch_rows(const BwdParams& P, Visit visit, float g, const floa
     visit([&](const Rows4& bt) {
         float zq[4], zv[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) zq[u] = zv[u] = 0.0f;
+        for (int u = 0; u < 4; ++u) {
+            zq[u] = zv[u] = 0.0f;
+            if (u < bt.n) {
+                float kx[4], vx[4];
+                load4<T>(K, bt.r[u], D, lane, kx);
+                load4<T>(V, bt.r[u], D, lane, vx);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const int d = lane + 32 * t;
-            if (d < D) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (u < bt.n) {
-                        zq[u] = fmaf(q[t], Elem<T>::to_f(K[bt.r[u] + d]), zq[u]);
-                        zv[u] = fmaf(go[t], Elem<T>::to_f(V[bt.r[u] + d]), zv[u]);
-                    }
+                for (int c = 0; c < 4; ++c) {
+                    zq[u] = fmaf(q[c], kx[c], zq[u]);
+                    zv[u] = fmaf(go[c], vx[c], zv[u]);
                 }
             }
         }
@@ -179,18 +193,20 @@ __device__ void branch_rows(const BwdParams& P, Visit visit, float g, const floa
     visit([&](const Rows4& bt) {
         float zq[4], zv[4], kv[4][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) zq[u] = zv[u] = 0.0f;
+        for (int u = 0; u < 4; ++u) {
+            zq[u] = zv[u] = 0.0f;
+            float vx[4];
+            if (u < bt.n) {
+                load4<T>(K, bt.r[u], D, lane, kv[u]);
+                load4<T>(V, bt.r[u], D, lane, vx);
+            } else {
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const int d = lane + 32 * t;
+                for (int c = 0; c < 4; ++c) kv[u][c] = vx[c] = 0.0f;
+            }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                kv[u][t] = 0.0f;
-                if (d < D && u < bt.n) {
-                    kv[u][t] = Elem<T>::to_f(K[bt.r[u] + d]);
-                    zq[u] = fmaf(q[t], kv[u][t], zq[u]);
-                    zv[u] = fmaf(go[t], Elem<T>::to_f(V[bt.r[u] + d]), zv[u]);
-                }
+            for (int c = 0; c < 4; ++c) {
+                zq[u] = fmaf(q[c], kv[u][c], zq[u]);
+                zv[u] = fmaf(go[c], vx[c], zv[u]);
             }
         }
         warp_sum8(zq, zv);
@@ -229,11 +245,8 @@ __global__ void __launch_bounds__(kWarps * 32) k_bwd_rows(const BwdParams P) {
     branch_rows<T>(
         P, [&](auto&& f) { visit_list(P.nbr_idx + w0, P.nbr_off[i + 1] - w0, H, h, D, f); }, g[2], q, go, dq,
         lane, lse_w, pdp_w);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int d = lane + 32 * t;
-        if (d < D) P.dq32[(i * H + h) * D + d] = dq[t];
-    }
+    if (4 * lane < D)
+        *reinterpret_cast<float4*>(P.dq32 + (i * H + h) * D + 4 * lane) = make_float4(dq[0], dq[1], dq[2], dq[3]);
     if (lane == 0) *reinterpret_cast<float4*>(P.stats + (i * H + h) * 4) = make_float4(lse_s, pdp_s, lse_w, pdp_w);
 }
 
@@ -260,15 +273,18 @@ __global__ void __launch_bounds__(kWarps * 32) k_bwd_keys(const BwdParams P) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             zq[u] = zv[u] = 0.0f;
-            const int64_t r = u < n ? ((int64_t)tk[u] * H + h) * D : 0;
+            if (u < n) {
+                const int64_t r = ((int64_t)tk[u] * H + h) * D;
+                load4<T>(Q, r, D, lane, qi[u]);
+                load4<T>(dO, r, D, lane, goi[u]);
+            } else {
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int d = lane + 32 * t;
-                const bool ok = u < n && d < D;
-                qi[u][t] = ok ? Elem<T>::to_f(Q[r + d]) : 0.0f;
-                goi[u][t] = ok ? Elem<T>::to_f(dO[r + d]) : 0.0f;
-                zq[u] = fmaf(qi[u][t], kj[t], zq[u]);
-                zv[u] = fmaf(goi[u][t], vj[t], zv[u]);
+                for (int c = 0; c < 4; ++c) qi[u][c] = goi[u][c] = 0.0f;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                zq[u] = fmaf(qi[u][c], kj[c], zq[u]);
+                zv[u] = fmaf(goi[u][c], vj[c], zv[u]);
             }
         }
         warp_sum8(zq, zv);
@@ -296,13 +312,9 @@ __global__ void __launch_bounds__(kWarps * 32) k_bwd_keys(const BwdParams P) {
     // window: the token's neighbours (j is in i's window exactly when i is in j's)
     const int32_t w0 = P.nbr_off[j], w1 = P.nbr_off[j + 1];
     for (int32_t e = w0; e < w1; e += 4) quad(P.nbr_idx + e, min(4, w1 - e), 2, 2);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int d = lane + 32 * t;
-        if (d < D) {
-            P.dk32[(j * H + h) * D + d] = dk[t];
-            P.dv32[(j * H + h) * D + d] = dv[t];
-        }
+    if (4 * lane < D) {
+        *reinterpret_cast<float4*>(P.dk32 + (j * H + h) * D + 4 * lane) = make_float4(dk[0], dk[1], dk[2], dk[3]);
+        *reinterpret_cast<float4*>(P.dv32 + (j * H + h) * D + 4 * lane) = make_float4(dv[0], dv[1], dv[2], dv[3]);
     }
 }
 
@@ -472,8 +484,9 @@ ssa_status_t run(Plan* p, const Workspace& w, BwdParams P, const void* q, const 
     int64_t most = 1;   // largest rows x blocks of a sequence
     for (int s = 0; s < p->B; ++s)
         most = std::max<int64_t>(most, (p->seqs[s].hi - p->seqs[s].lo) * (p->seq_blk[s + 1] - p->seq_blk[s]));
-    // heads per batch: the two [heads, rows, blocks] fp32 buffers within about 4 GB
-    const int hb = (int)std::max<int64_t>(1, std::min<int64_t>(H, ((int64_t)1 << 29) / most));
+    // heads per batch: each of the two [heads, rows, blocks] fp32 buffers within 16 GB (all 22
+    // heads of a 110k-token sequence at once: the skinny dKc / dVc products get more parallelism)
+    const int hb = (int)std::max<int64_t>(1, std::min<int64_t>(H, ((int64_t)1 << 32) / most));
     float* SB = A(sizeof(float) * (size_t)hb * most);
     float* PB = A(sizeof(float) * (size_t)hb * most);
     if (!SB || !PB) {

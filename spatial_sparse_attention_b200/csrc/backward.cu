@@ -130,15 +130,34 @@ __device__ __forceinline__ void visit_list(const int32_t* idx, int32_t n, int H,
     }
 }
 
-// dots of two per-lane vectors with up to 4 rows each (warp sums, interleaved)
+// Warp sums of eight values (a[0..3], b[0..3]), returned to every lane: a reduce-scatter that
+// halves the values each step (lanes that differ in bit 4, then 3, then 2 exchange the half the
+// other keeps), sums over bits 1 and 0, then a gather from the lane holding each total (17
+// shuffles instead of 40).
 __device__ __forceinline__ void warp_sum8(float (&a)[4], float (&b)[4]) {
+    const int lane = threadIdx.x & 31;
+    const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4;
+    float w4[4], w2[2];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int i = 0; i < 4; ++i) {
+        const float send = h4 ? a[i] : b[i];
+        const float keep = h4 ? b[i] : a[i];
+        w4[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            a[u] += __shfl_xor_sync(0xffffffffu, a[u], o);
-            b[u] += __shfl_xor_sync(0xffffffffu, b[u], o);
-        }
+    for (int i = 0; i < 2; ++i) {
+        const float send = h3 ? w4[i] : w4[2 + i];
+        const float keep = h3 ? w4[2 + i] : w4[i];
+        w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float w1 = (h2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, h2 ? w2[0] : w2[1], 4);
+    w1 += __shfl_xor_sync(0xffffffffu, w1, 2);
+    w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
+    // the total of value k = 4 (bit 4) + 2 (bit 3) + (bit 2) is in lanes 4k .. 4k + 3
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        a[i] = __shfl_sync(0xffffffffu, w1, 4 * i);
+        b[i] = __shfl_sync(0xffffffffu, w1, 16 + 4 * i);
     }
 }
 

@@ -539,13 +539,25 @@ __global__ void __launch_bounds__(kThreads, 2) k_ssa_select_sub(const __grid_con
 #pragma unroll
         for (int u = 0; u < KM; ++u) tk[u] = 0ull;
         float m = -INFINITY, l = 0.0f, lse = 0.0f;
-        bool ok = nseg > 0;
+        bool ok = nseg > 0, p1_ok = true;
         for (int j = 0; j < 2 * nc && ok; ++j) {
             const int b = j & 1, jt = j < nc ? j : j - nc;
-            // one decision for all four row warps, so that they meet the same named barriers
-            ok = named_sync_and(1, 128, wait_or_flag(&bar[SFULL + b], (uint32_t)(j >> 1) & 1u, P.status,
-                                                     abort_flag));
-            if (!ok) break;
+            if (j < nc) {
+                // pass 1 has no named barrier: a warp whose wait ran out skips its tiles, and the
+                // four row warps decide together at the end of the pass
+                const bool wok = p1_ok && __all_sync(0xffffffffu, wait_or_flag(&bar[SFULL + b], (uint32_t)(j >> 1) & 1u,
+                                                                            P.status, abort_flag));
+                p1_ok = wok;
+                if (!wok) {
+                    if (j == nc - 1 && !(ok = named_sync_and(1, 128, false))) break;
+                    continue;
+                }
+            } else {
+                // one decision for all four row warps, so that they meet the same named barriers
+                ok = named_sync_and(1, 128, wait_or_flag(&bar[SFULL + b], (uint32_t)(j >> 1) & 1u, P.status,
+                                                         abort_flag));
+                if (!ok) break;
+            }
             tc::fence_after_sync();
             float s[64];
             tc::tmem_ld64(tmem + lane_base + b * kKT, s);
@@ -571,7 +583,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_ssa_select_sub(const __grid_con
 #pragma unroll
                 for (int e = 0; e < 64; ++e) ls[e & 3] += tc::ex2(fmaf(s[e], sl, -m));
                 l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                if (j == nc - 1) lse = m + __log2f(l);
+                if (j == nc - 1) {
+                    lse = m + __log2f(l);
+                    if (!(ok = named_sync_and(1, 128, true))) break;
+                }
                 continue;
             }
             // pass 2: this row's weights into the stage

@@ -891,3 +891,29 @@ def test_subblock_selection_is_shared_by_all_queries_of_a_subblock():
         m = np.nonzero(grp == gi)[0]
         assert (sel[m] == sel[m[0]]).all()
     assert len(np.unique(grp)) < N   # the tiny shell has sub-blocks with several cells
+
+
+def test_subblock_selection_with_the_centre_tap_is_the_plain_one():
+    """Convolution compression with only the centre tap (W_0 = Wc) gives the plain compressed
+    tokens, hence the same shared selection and summed weights."""
+    c, _ = _tiny_coords()
+    N, H, D = len(c), 2, 8
+    q, k, v = (_rand((N, H, D), 61 + i) for i in range(3))
+    Wc = (_rand((D, D), 64) / np.sqrt(D)).astype(np.float32)
+    a = oracle.select_subblock(c, [0, N], q, k, v, Wc, 4, want_score=True)
+    b = oracle.select_subblock(c, [0, N], q, k, v, Wc, 4, conv=oracle.center_only_conv(Wc), want_score=True)
+    np.testing.assert_array_equal(a["sel"], b["sel"])
+    for x, y in zip(a["score"], b["score"]):
+        np.testing.assert_allclose(y, x, rtol=1e-12, atol=1e-15)
+
+
+def test_subblock_selection_is_invariant_under_block_translation():
+    """Moving every cell by whole 8-cell blocks moves every 4-cell sub-block with its block: the
+    same tokens share a selection, with the same blocks (block indices keep their order)."""
+    c, _ = _tiny_coords()
+    N, H, D = len(c), 2, 8
+    q, k, v = (_rand((N, H, D), 71 + i) for i in range(3))
+    Wc = (_rand((D, D), 74) / np.sqrt(D)).astype(np.float32)
+    a = oracle.select_subblock(c, [0, N], q, k, v, Wc, 4)["sel"]
+    b = oracle.select_subblock(c + np.array([8, 24, 16], np.int32), [0, N], q, k, v, Wc, 4)["sel"]
+    np.testing.assert_array_equal(a, b)
